@@ -1,0 +1,361 @@
+"""Throughput of the ARL2 hybrid attention layer: frames/s per layer at the 480p workload.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one autoregressive frame of one layer: 4 denoising queries (intra-frame softmax
+attention plus the state readout) and the clean-pass commit of the state. This is every
+step of the layer's hot path.
+
+The workload is 480p: B=1, H=12, d=128, T=1560 tokens per frame. Inputs are seeded and
+synthetic (q, k, v ~ N(0,1) in bf16; phi ~ N(0, 1/d); alpha = sigmoid(N(2, 0.5));
+beta = sigmoid(N(0,1))). The timed region cycles through 8 frames of distinct inputs,
+5 passes per frame (4 denoising + 1 clean), about 575 MB. That is larger than the 126 MB
+L2, so no input is L2-resident between frames.
+
+The bench prints one JSON line (rank 0):
+  - value: whole-job frames/s, timed on the device with CUDA events between barriers.
+  - e2e: the same metric through the host-buffer entry points. Each step copies its
+    inputs from pinned host memory and its outputs back.
+  - roofline: the query kernel's achieved TFLOP/s (algorithmic FLOPs / mean launch time,
+    CUDA events on the launching stream) against the measured bf16 peak.
+  - cpu_baseline: the fp64 oracle on this host's cores over a bounded sample.
+  - clocks: SM clocks and throttle reasons sampled with NVML during the timed region.
+With --gpus N under torchrun, each rank runs its own independent layer (the layer has no
+exchange between streams: replicas, weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from softmax_attention_ar_b200 import synth  # noqa: E402
+
+WORKLOAD = synth.WORKLOADS["480p"]
+B, T, H, D = WORKLOAD["B"], WORKLOAD["T"], WORKLOAD["H"], WORKLOAD["d"]
+QUERIES = WORKLOAD["queries"]
+CYCLE = 8                      # distinct frames of inputs in the timed cycle
+METRIC = "frames/s per ARL2 layer at T=1560,H=12,d=128; % bf16 TC peak & % HBM BW"
+UNIT = "frames/s"
+CONFIG = {"workload": "480p single layer: B=1, H=12, d=128, T=1560 tokens/frame; "
+                      "4 denoising queries + 1 clean-pass commit per frame",
+          "B": B, "H": H, "T": T, "d": D, "queries_per_frame": QUERIES,
+          "l2": "inputs larger than L2 (8-frame cycle of distinct q/k/v, 575 MB)"}
+
+# Algorithmic work (only what the layer must do; padding of ragged tiles is not credited).
+QUERY_FLOPS = B * H * (4.0 * T * T * D + 2 * 2.0 * T * D * D)        # QK^T + PV, phi_q + readout
+QUERY_BYTES = B * T * H * D * 2 * 4 + B * H * D * D * (2 + 2)          # q,k,v,o bf16; S bf16 copy, Wq
+COMMIT_FLOPS = B * H * 4 * 2.0 * T * D * D                             # K Wk, V Wv, K'S, K'^T R
+COMMIT_BYTES = B * T * H * D * 2 * 2 + 2 * B * H * T * 4 + B * H * D * D * 4 * 2 + 2 * H * D * D * 2
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML (read-only) in a thread."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self._stop = [], set(), threading.Event()
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                self.reasons.update(n for b, n in self.REASONS.items() if mask & b)
+            except Exception:
+                pass
+            self._stop.wait(0.02)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._nv is not None:
+            self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+def make_inputs(dev):
+    import torch
+
+    def bf(x):
+        return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16)
+
+    frames = []
+    for f in range(CYCLE):
+        passes = [tuple(bf(x) for x in synth.qkv(0, WORKLOAD["config"], f, p, B, T, H, D))
+                  for p in range(QUERIES + 1)]
+        a, b = synth.gates(0, WORKLOAD["config"], f, B, H, T)
+        frames.append((passes, torch.from_numpy(a), torch.from_numpy(b)))
+    wq, wk, wv = (bf(x) for x in synth.feature_maps(0, WORKLOAD["config"], H, D))
+    if dev is None:
+        return frames, (wq, wk, wv)
+    dev_frames = [([tuple(t.to(dev) for t in p) for p in passes], a.to(dev), b.to(dev)) for passes, a, b in frames]
+    return dev_frames, (wq.to(dev), wk.to(dev), wv.to(dev)), frames
+
+
+class OracleSample:
+    """A bounded slice of one 480p frame for the fp64 oracle: the 4 queries of one head on R
+    query rows, and that head's commit over R tokens. Work grows linearly in R, so the slice
+    stands for R / (T * H) of a frame."""
+
+    def __init__(self):
+        import oracle
+        self.oracle = oracle
+        cfg = WORKLOAD["config"]
+        wq, wk, wv = (synth.bf16_to_f64(x)[:1] for x in synth.feature_maps(0, cfg, H, D))
+        self.W = (wq, wk, wv)
+        self.passes = [tuple(synth.bf16_to_f64(x)[:, :, :1] for x in synth.qkv(0, cfg, 0, p, B, T, H, D))
+                       for p in range(QUERIES + 1)]
+        a, b = synth.gates(0, cfg, 0, B, H, T)
+        self.gates = (a[:, :1], b[:, :1])
+        self.S = np.zeros((B, 1, D, D))
+
+    def run(self, R: int) -> float:
+        """Run one slice; return the fraction of a frame it stands for."""
+        rows = np.arange(R)
+        for p in range(QUERIES):
+            self.oracle.frame_query(*self.passes[p], self.W[0], self.S, rows=rows)
+        _, k, v = self.passes[QUERIES]
+        self.S = self.oracle.frame_commit(k[:, :R], v[:, :R], self.gates[0][..., :R], self.gates[1][..., :R],
+                                          self.W[1], self.W[2], self.S)
+        return R / (T * H)
+
+
+def _oracle_rate(steps: int, warmup: int, budget_s: float):
+    """Time `steps` oracle slices sized so the run takes about budget_s; return (frames/s, R, seconds)."""
+    from threadpoolctl import threadpool_info
+    s = OracleSample()
+    t0 = time.perf_counter()
+    s.run(T)                                  # calibrate on one full head
+    full = time.perf_counter() - t0
+    R = int(max(8, min(T, T * budget_s / max(1, steps + warmup) / full)))
+    for _ in range(warmup):
+        s.run(R)
+    t0 = time.perf_counter()
+    frac = sum(s.run(R) for _ in range(steps))
+    dt = time.perf_counter() - t0
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return frac / dt, R, dt, threads
+
+
+def cpu_baseline(budget_s: float = 15.0):
+    """The fp64 oracle, as it stands, on this host's cores: frames/s over a bounded sample."""
+    steps = 12
+    rate, R, dt, threads = _oracle_rate(steps, 1, budget_s)
+    return {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{steps} slices of a 480p frame, each the 4 queries of one head on {R} of {T} query rows "
+                      f"plus that head's commit over {R} tokens ({steps * R / (T * H):.3f} frames in {dt:.1f} s); "
+                      f"fp64 numpy/BLAS, {os.cpu_count()} host cores"}
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the fp64 oracle on the host cores, same metric and workload."""
+    if rank != 0:
+        return
+    rate, R, dt, threads = _oracle_rate(args.steps, args.warmup, budget_s=90.0)
+    base = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"each step: the 4 queries of one head on {R} of {T} query rows plus that head's commit "
+                      f"over {R} tokens (= {R / (T * H):.5f} frame)"}
+    line = {"impl": "reference", "metric": METRIC, "value": rate, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": CONFIG, "cpu_baseline": base,
+            "e2e": {"value": rate, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from softmax_attention_ar_b200.arl2 import ARL2Layer
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    frames, maps, host_frames = make_inputs(dev)
+    layer = ARL2Layer(H, T, D, B)
+    layer.set_feature_maps(*maps)
+    o = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def step(i, ev=None):
+        passes, a, b = frames[i % CYCLE]
+        for p in range(QUERIES):
+            if ev is not None:
+                ev[0].record(stream)
+            layer.query(*passes[p], out=o)
+            if ev is not None:
+                ev[1].record(stream)
+                ev = ev[2:]
+        _, k, v = passes[QUERIES]
+        if ev is not None:
+            ev[0].record(stream)
+        layer.commit(k, v, a, b)
+        if ev is not None:
+            ev[1].record(stream)
+
+    # Device-resident run.
+    for i in range(args.warmup):
+        step(i)
+    ev_all = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * (QUERIES + 1))] for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank)
+    barrier()
+    with clocks:
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for i in range(args.steps):
+            step(args.warmup + i, ev_all[i])
+        end.record(stream)
+        barrier()
+    elapsed_ms = start.elapsed_time(end)
+    q_ms = [ev[2 * p].elapsed_time(ev[2 * p + 1]) for ev in ev_all for p in range(QUERIES)]
+    c_ms = [ev[2 * QUERIES].elapsed_time(ev[2 * QUERIES + 1]) for ev in ev_all]
+    status = layer.status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+
+    # End-to-end through the host-buffer entry points (pinned host memory).
+    pinned = [([tuple(t.pin_memory() for t in p) for p in passes], a.pin_memory(), b.pin_memory())
+              for passes, a, b in host_frames]
+    o_host = torch.empty((B, T, H, D), dtype=torch.bfloat16).pin_memory()
+    layer.reset()
+
+    def host_step(i):
+        passes, a, b = pinned[i % CYCLE]
+        for p in range(QUERIES):
+            layer.query_host(*passes[p], o_host)
+        _, k, v = passes[QUERIES]
+        layer.commit_host(k, v, a, b)
+
+    e2e_steps = max(1, min(args.steps, 200))
+    for i in range(min(args.warmup, 3)):
+        host_step(i)
+    barrier()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for i in range(e2e_steps):
+        host_step(i)
+    e2.record(stream)
+    barrier()
+    e2e_ms = s2.elapsed_time(e2)
+    act = B * T * H * D * 2
+    h2d = (QUERIES * 3 + 2) * act + 2 * B * H * T * 4
+    d2h = QUERIES * act
+
+    # Max over ranks.
+    t = torch.tensor([elapsed_ms, e2e_ms], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed_ms, e2e_ms = t.tolist()
+    if rank != 0:
+        return
+    value = world * B * args.steps / (elapsed_ms / 1e3)
+    e2e_value = world * B * e2e_steps / (e2e_ms / 1e3)
+    peaks = _peaks()
+    q_mean_s = statistics.mean(q_ms) / 1e3
+    c_mean_s = statistics.mean(c_ms) / 1e3
+    q_tflops = QUERY_FLOPS / q_mean_s / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": CONFIG,
+        "roofline": {"bound": "tensor", "achieved": q_tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": q_tflops / peak, "traffic": None,
+                     "kernel": "arl2_query_kernel (one query pass)",
+                     "peak_source": f"bf16_tflops_sustained ({peaks['source']})",
+                     "frac_of_burst_peak": q_tflops / peaks["bf16_tflops"]},
+        "kernels": {"query_us": 1e6 * q_mean_s, "query_p95_us": 1e3 * float(np.percentile(q_ms, 95)),
+                    "commit_us": 1e6 * c_mean_s,
+                    "commit_hbm_gbs": COMMIT_BYTES / c_mean_s / 1e9,
+                    "commit_hbm_frac": COMMIT_BYTES / c_mean_s / 1e9 / peaks["hbm_gbs"],
+                    "commit_tflops": COMMIT_FLOPS / c_mean_s / 1e12},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "gpu_launches": args.steps * (QUERIES * 1 + 2),
+        "clocks": clocks.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    print(json.dumps(line), flush=True)
+    layer.close()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

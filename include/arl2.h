@@ -1,0 +1,160 @@
+/*
+ * arl2.h - C ABI of the ARL2 hybrid per-frame attention layer on NVIDIA B200 (sm_100a).
+ *
+ * The layer is the one described in "Attend Locally, Remember Linearly (ARL2)", the
+ * technical summary of arXiv 2605.16579 (gist.science, zh/pt/fr pages):
+ *   - §2.1: self-attention is split into an intra-frame branch (the original bidirectional
+ *     softmax attention among one frame's tokens) and an inter-frame branch. The
+ *     inter-frame branch replaces the growing KV cache by a fixed-size recurrent state S.
+ *   - §2.1: per-head grouped 1x1 feature maps phi_q, phi_k, phi_v adapt Q, K, V to the
+ *     recurrent branch.
+ *   - §2.1: the state follows a gated-delta rule, and the branch reads out
+ *     O_inter = Q' S_{N-1}.
+ *   - §2.2: every token of frame N reads the same S_{N-1} (frame-level access). The
+ *     denoising passes only read S. S is written once per frame, after the clean pass
+ *     (clean-pass update).
+ * Per (batch, head) this library computes
+ *     query:   O   = softmax(Q K^T / sqrt(d)) V + (Q Wq_h) S_{N-1}
+ *     commit:  S_N = abar S_{N-1} + K'^T diag(beta / T) (V' - K' S_{N-1}),
+ *              K'  = rownorm(K Wk_h),  V' = V Wv_h,  abar = mean_t alpha_t.
+ * The pages print the update without a transpose. They also do not say how the per-token
+ * gates become one factor per frame. Reading K'^T, the mean of alpha and the rate
+ * beta_t / T is this library's convention.
+ *
+ * Conventions for every call:
+ *   - Pointers are device pointers unless a name ends in _host. Every call is
+ *     asynchronous on the given stream (NULL = the legacy default stream) and returns
+ *     after enqueueing the work. Argument checks are synchronous and return a status.
+ *     Faults and wait time-outs inside kernels are reported later by arl2_get_status.
+ *   - bf16 arrays hold bfloat16 bit patterns (uint16_t). q, k, v and o are [B, T, H, d]
+ *     contiguous (token-major, as a linear projection writes them) and 16-byte aligned.
+ *     alpha and beta are fp32 [B, H, T]. The state is fp32 [B, H, d_k, d_v].
+ *   - The caller owns every buffer it passes. The library owns the two state buffers, its
+ *     copies of the feature maps, its scratch and its staging buffers. It allocates all of
+ *     them in arl2_create and frees them in arl2_destroy, so no call allocates memory.
+ *   - Supported shapes: d_k == d_v == d in {32, 64, 128}; 1 <= T <= 4096; B >= 1; H >= 1;
+ *     B * H <= 65535. Other shapes return ARL2_ERR_UNSUPPORTED. The device must be sm_100.
+ *   - A context is not thread-safe. Calls on one context must be ordered by the caller,
+ *     normally by using one stream.
+ */
+#ifndef ARL2_H
+#define ARL2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct arl2_ctx arl2_ctx;        /* opaque; owned by the library */
+typedef struct arl2_kvcache arl2_kvcache; /* opaque; the growing-KV-cache baseline */
+typedef void* arl2_stream;               /* a cudaStream_t; NULL is the legacy default stream */
+typedef uint16_t arl2_bf16;              /* a bfloat16 bit pattern */
+
+typedef enum {
+  ARL2_OK = 0,
+  ARL2_ERR_INVALID_ARG = 1, /* null or misaligned pointer, bad context */
+  ARL2_ERR_UNSUPPORTED = 2, /* shape or device outside the supported set */
+  ARL2_ERR_OOM = 3,         /* a device allocation in a create call failed */
+  ARL2_ERR_CUDA = 4,        /* a CUDA call failed, or a kernel faulted */
+  ARL2_ERR_TIMEOUT = 5,     /* a kernel's bounded wait ran out; the result of that call is invalid */
+  ARL2_ERR_STATE = 6        /* call out of order, such as a query before the feature maps are set */
+} arl2_status;
+
+/* Create a layer for B independent streams of H heads, T tokens per frame and head
+ * dims d_k = d_v. Allocates the fp32 state S (two buffers, which alternate per commit),
+ * a bf16 copy of S, the feature-map copies, scratch and staging. S starts at 0 and the
+ * frame count at 0. On success *out holds the context; on failure *out is NULL. */
+arl2_status arl2_create(int H, int T, int d_k, int d_v, int B, arl2_ctx** out);
+
+/* Copy the per-head feature maps phi_q, phi_k, phi_v into the library (§2.1, the per-head
+ * grouped 1x1 maps). Each is bf16 [H, d, d] and applies as x' = x @ W[h]; no bias, no
+ * activation. Must be called before the first query or commit; it may be called again.
+ * Stream-ordered: the caller's buffers may be reused once the stream has passed the copy. */
+arl2_status arl2_set_feature_maps(arl2_ctx* ctx, const arl2_bf16* Wq, const arl2_bf16* Wk,
+                                  const arl2_bf16* Wv, arl2_stream stream);
+
+/* One query pass of frame N (a denoising step, or the clean pass): (§2.1, §2.2)
+ *   o = softmax(q k^T / sqrt(d)) v  +  (q Wq_h) S_{N-1}    per (batch, head).
+ * q, k, v, o: bf16 [B, T, H, d]. Reads S_{N-1} and never writes the state. o must not
+ * overlap q, k or v. */
+arl2_status arl2_frame_query(arl2_ctx* ctx, const arl2_bf16* q, const arl2_bf16* k,
+                             const arl2_bf16* v, arl2_bf16* o, arl2_stream stream);
+
+/* The clean-pass commit of frame N (§2.1 state update, §2.2 clean-pass update):
+ *   S_N = abar S_{N-1} + K'^T diag(beta / T) (V' - K' S_{N-1}).
+ * k, v: bf16 [B, T, H, d], the clean pass's keys and values. alpha (forget gate, in (0, 1))
+ * and beta (rate): fp32 [B, H, T]. Writes S_N into the other state buffer and advances the
+ * frame count. Later queries read S_N. Queries enqueued before this commit read S_{N-1},
+ * by stream order. */
+arl2_status arl2_frame_commit(arl2_ctx* ctx, const arl2_bf16* k, const arl2_bf16* v,
+                              const float* alpha, const float* beta, arl2_stream stream);
+
+/* Host-buffer forms of the two calls above, for callers whose data is in host memory.
+ * Each call enqueues, on the stream, the host-to-device copies into library-owned staging,
+ * the kernels, and (for the query) the device-to-host copy of o. With pinned host memory
+ * the call returns at once; the caller synchronises the stream before reading o_host or
+ * reusing the inputs. With pageable memory the CUDA copies may block. */
+arl2_status arl2_frame_query_host(arl2_ctx* ctx, const arl2_bf16* q_host, const arl2_bf16* k_host,
+                                  const arl2_bf16* v_host, arl2_bf16* o_host, arl2_stream stream);
+arl2_status arl2_frame_commit_host(arl2_ctx* ctx, const arl2_bf16* k_host, const arl2_bf16* v_host,
+                                   const float* alpha_host, const float* beta_host,
+                                   arl2_stream stream);
+
+/* Reset the state to S_0 = 0 and the frame count to 0 (the start of a new video). */
+arl2_status arl2_reset(arl2_ctx* ctx, arl2_stream stream);
+
+/* Copy the current state (fp32 [B, H, d_k, d_v]) to dst, which may be device or host
+ * memory. Used for checkpointing and tests. */
+arl2_status arl2_get_state(const arl2_ctx* ctx, float* dst, arl2_stream stream);
+
+/* Replace the current state with src (fp32 [B, H, d_k, d_v], device or host memory),
+ * for resuming from a checkpoint and for tests. The frame count is unchanged. */
+arl2_status arl2_set_state(arl2_ctx* ctx, const float* src, arl2_stream stream);
+
+/* Number of commits since creation or the last reset. */
+int arl2_frame_index(const arl2_ctx* ctx);
+
+/* Synchronise the device and return, then clear, the context's device error word.
+ * Returns ARL2_ERR_TIMEOUT if a kernel's bounded wait ran out since the last call, and
+ * ARL2_ERR_CUDA if the device reported an error. Otherwise it returns ARL2_OK. */
+arl2_status arl2_get_status(arl2_ctx* ctx);
+
+/* Limit on every wait inside this context's kernels, in nanoseconds (default 1e9). When
+ * a wait runs out, the kernel abandons the call and returns; arl2_get_status then reports
+ * ARL2_ERR_TIMEOUT. Very small values make ordinary waits run out, which tests use to
+ * exercise that path. */
+arl2_status arl2_set_wait_timeout_ns(arl2_ctx* ctx, uint64_t timeout_ns);
+
+/* Bytes of device memory the context holds (everything allocated in arl2_create). */
+size_t arl2_memory_bytes(const arl2_ctx* ctx);
+
+/* Free everything the context holds. The caller must make sure none of its work is still
+ * in flight. NULL is ignored. */
+void arl2_destroy(arl2_ctx* ctx);
+
+/* ---- Growing-KV-cache baseline (comparison only; §1 problem statement) -----------------
+ * This is full softmax attention of the newest frame over the keys and values of every
+ * frame so far, which is what the layer above replaces. Its cache grows by one frame per
+ * commit, up to max_frames. The cache is preallocated and zero-filled in create.
+ *   query:  writes k, v into the slot of the current frame n (without committing it), then
+ *           o = softmax(q K_{1..n+1}^T / sqrt(d)) V_{1..n+1}, over (n+1) T keys.
+ *   commit: writes k, v into slot n and advances n.
+ * Layouts, alignment and stream rules are as above. */
+arl2_status arl2_kvcache_create(int H, int T, int d, int B, int max_frames, arl2_kvcache** out);
+arl2_status arl2_kvcache_query(arl2_kvcache* c, const arl2_bf16* q, const arl2_bf16* k,
+                               const arl2_bf16* v, arl2_bf16* o, arl2_stream stream);
+arl2_status arl2_kvcache_commit(arl2_kvcache* c, const arl2_bf16* k, const arl2_bf16* v,
+                                arl2_stream stream);
+arl2_status arl2_kvcache_reset(arl2_kvcache* c);
+int arl2_kvcache_frames(const arl2_kvcache* c);
+arl2_status arl2_kvcache_get_status(arl2_kvcache* c);
+size_t arl2_kvcache_memory_bytes(const arl2_kvcache* c);
+void arl2_kvcache_destroy(arl2_kvcache* c);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ARL2_H */

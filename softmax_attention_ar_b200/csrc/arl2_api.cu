@@ -1,0 +1,505 @@
+// C-ABI layer of the ARL2 library: contexts, argument checks, TMA descriptors, state
+// ping-pong and launches. The computation itself lives in arl2_query.cu and arl2_commit.cu.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/arl2.h"
+#include "arl2_kernels.h"
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// A bf16 tensor map with 128-byte swizzle and 64-element-wide boxes; out-of-range elements
+// read as zero (this is how head dims below 128 and ragged token tails are padded).
+bool make_map(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims, const cuuint64_t* strides_bytes,
+              const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims, strides_bytes, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// [B, L, H, d] token-major activations: dims (d, H, L, B), box (64, 1, 128, 1).
+bool make_act_map(CUtensorMap* m, const void* ptr, int B, int L, int H, int d) {
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)B};
+  const cuuint64_t str[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)L * H * d * 2};
+  const cuuint32_t box[4] = {64, 1, 128, 1};
+  return make_map(m, ptr, 4, dims, str, box);
+}
+
+// [n, d, d] row-major square matrices: dims (d, d, n), box (64, 128, 1).
+bool make_mat_map(CUtensorMap* m, const void* ptr, int n, int d) {
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)d, (cuuint64_t)n};
+  const cuuint64_t str[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * d * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  return make_map(m, ptr, 3, dims, str, box);
+}
+
+bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// Small cache of activation maps keyed by base pointer: callers usually reuse buffers.
+struct MapCache {
+  static constexpr int kSlots = 16;
+  const void* ptr[kSlots] = {};
+  CUtensorMap map[kSlots];
+  int next = 0;
+  const CUtensorMap* get(const void* p, int B, int L, int H, int d) {
+    for (int i = 0; i < kSlots; ++i)
+      if (ptr[i] == p) return &map[i];
+    const int i = next;
+    next = (next + 1) % kSlots;
+    ptr[i] = nullptr;
+    if (!make_act_map(&map[i], p, B, L, H, d)) return nullptr;
+    ptr[i] = p;
+    return &map[i];
+  }
+};
+
+std::mutex g_setup_mu;
+bool g_setup_done[64] = {};
+
+cudaError_t device_setup(int dev) {
+  std::lock_guard<std::mutex> lk(g_setup_mu);
+  if (dev >= 0 && dev < 64 && g_setup_done[dev]) return cudaSuccess;
+  cudaError_t e = arl2::query_setup();
+  if (e == cudaSuccess) e = arl2::commit_setup();
+  if (e == cudaSuccess && dev >= 0 && dev < 64) g_setup_done[dev] = true;
+  return e;
+}
+
+arl2_status check_device(int* dev, int* sms) {
+  if (cudaGetDevice(dev) != cudaSuccess) return ARL2_ERR_CUDA;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, *dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, *dev) != cudaSuccess)
+    return ARL2_ERR_CUDA;
+  if (major != 10 || minor != 0) return ARL2_ERR_UNSUPPORTED;
+  if (!encode_fn()) return ARL2_ERR_CUDA;
+  if (device_setup(*dev) != cudaSuccess) return ARL2_ERR_CUDA;
+  return ARL2_OK;
+}
+
+constexpr unsigned long long kDefaultTimeoutNs = 1000000000ull;
+
+}  // namespace
+
+struct arl2_ctx {
+  int B = 0, H = 0, T = 0, d = 0;
+  int device = 0, num_sms = 0;
+  int chunks_per_group = 1, ngroups = 1;
+  uint16_t* W[3] = {};            // phi_q, phi_k, phi_v copies, [H, d, d]
+  float* S[2] = {};               // fp32 state buffers, [B, H, d, d]
+  uint16_t* S_bf16 = nullptr;     // [2][B, H, d, d] bf16 copies of S[0], S[1]
+  float* part = nullptr;          // [B*H*ngroups, d, d]
+  float* alpha_part = nullptr;    // [B*H*ngroups]
+  unsigned int* err = nullptr;
+  uint16_t* stage_bf16[4] = {};   // q, k, v, o staging for the host-buffer calls
+  float* stage_f32[2] = {};       // alpha, beta staging
+  int cur = 0;                    // buffer holding S_{N-1}
+  int frame = 0;
+  bool maps_set = false;
+  unsigned long long timeout_ns = kDefaultTimeoutNs;
+  CUtensorMap tm_w[3];
+  CUtensorMap tm_s;
+  MapCache acts;
+  size_t bytes = 0;
+
+  size_t act_elems() const { return (size_t)B * T * H * d; }
+  size_t state_elems() const { return (size_t)B * H * d * d; }
+};
+
+struct arl2_kvcache {
+  int B = 0, H = 0, T = 0, d = 0, max_frames = 0;
+  int n = 0;
+  int device = 0;
+  uint16_t* K = nullptr;   // [B, max_frames*T, H, d]
+  uint16_t* V = nullptr;
+  unsigned int* err = nullptr;
+  CUtensorMap tm_k, tm_v;
+  MapCache acts;
+  size_t bytes = 0;
+  unsigned long long timeout_ns = kDefaultTimeoutNs;
+};
+
+namespace {
+
+template <typename T>
+bool dev_alloc(T** p, size_t count, size_t* total) {
+  if (cudaMalloc(reinterpret_cast<void**>(p), count * sizeof(T)) != cudaSuccess) {
+    *p = nullptr;
+    return false;
+  }
+  *total += count * sizeof(T);
+  return true;
+}
+
+void free_ctx(arl2_ctx* c) {
+  if (!c) return;
+  for (auto& p : c->W) cudaFree(p);
+  for (auto& p : c->S) cudaFree(p);
+  cudaFree(c->S_bf16);
+  cudaFree(c->part);
+  cudaFree(c->alpha_part);
+  cudaFree(c->err);
+  for (auto& p : c->stage_bf16) cudaFree(p);
+  for (auto& p : c->stage_f32) cudaFree(p);
+  delete c;
+}
+
+arl2_status query_impl(arl2_ctx* c, const void* q, const void* k, const void* v, void* o, cudaStream_t st) {
+  const CUtensorMap* mq = c->acts.get(q, c->B, c->T, c->H, c->d);
+  const CUtensorMap* mk = c->acts.get(k, c->B, c->T, c->H, c->d);
+  const CUtensorMap* mv = c->acts.get(v, c->B, c->T, c->H, c->d);
+  if (!mq || !mk || !mv) return ARL2_ERR_CUDA;
+  arl2::QueryArgs a{};
+  a.o = static_cast<uint16_t*>(o);
+  a.T = c->T;
+  a.kv_len = c->T;
+  a.B = c->B;
+  a.H = c->H;
+  a.d = c->d;
+  a.state_slot = c->cur;
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->d)));
+  a.err = c->err;
+  a.timeout_ns = c->timeout_ns;
+  return arl2::launch_query(true, *mq, *mk, *mv, c->tm_w[0], c->tm_s, a, st) == cudaSuccess ? ARL2_OK
+                                                                                           : ARL2_ERR_CUDA;
+}
+
+arl2_status commit_impl(arl2_ctx* c, const void* k, const void* v, const float* alpha, const float* beta,
+                        cudaStream_t st) {
+  const CUtensorMap* mk = c->acts.get(k, c->B, c->T, c->H, c->d);
+  const CUtensorMap* mv = c->acts.get(v, c->B, c->T, c->H, c->d);
+  if (!mk || !mv) return ARL2_ERR_CUDA;
+  arl2::CommitArgs a{};
+  a.alpha = alpha;
+  a.beta = beta;
+  a.part = c->part;
+  a.alpha_part = c->alpha_part;
+  a.T = c->T;
+  a.B = c->B;
+  a.H = c->H;
+  a.d = c->d;
+  a.chunks_per_group = c->chunks_per_group;
+  a.ngroups = c->ngroups;
+  a.state_slot = c->cur;
+  a.inv_T = 1.0f / static_cast<float>(c->T);
+  a.err = c->err;
+  a.timeout_ns = c->timeout_ns;
+  arl2::ReduceArgs r{};
+  r.part = c->part;
+  r.alpha_part = c->alpha_part;
+  r.S_old = c->S[c->cur];
+  r.S_new = c->S[c->cur ^ 1];
+  r.S_new_bf16 = c->S_bf16 + (size_t)(c->cur ^ 1) * c->state_elems();
+  r.d = c->d;
+  r.ngroups = c->ngroups;
+  r.BH = c->B * c->H;
+  r.inv_T = a.inv_T;
+  if (arl2::launch_commit(*mk, *mv, c->tm_w[1], c->tm_w[2], c->tm_s, a, r, st) != cudaSuccess) return ARL2_ERR_CUDA;
+  c->cur ^= 1;
+  ++c->frame;
+  return ARL2_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+arl2_status arl2_create(int H, int T, int d_k, int d_v, int B, arl2_ctx** out) {
+  if (!out) return ARL2_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (H < 1 || B < 1 || T < 1 || d_k < 1 || d_v < 1) return ARL2_ERR_INVALID_ARG;
+  if (d_k != d_v || (d_k != 32 && d_k != 64 && d_k != 128) || T > 4096 || (long long)B * H > 65535)
+    return ARL2_ERR_UNSUPPORTED;
+  int dev = 0, sms = 0;
+  arl2_status s = check_device(&dev, &sms);
+  if (s != ARL2_OK) return s;
+  arl2_ctx* c = new (std::nothrow) arl2_ctx();
+  if (!c) return ARL2_ERR_OOM;
+  c->B = B;
+  c->H = H;
+  c->T = T;
+  c->d = d_k;
+  c->device = dev;
+  c->num_sms = sms;
+  // Commit work split: about one CTA per SM, each taking whole 128-token chunks.
+  const int nchunks = (T + 127) / 128;
+  const long long total = (long long)nchunks * H * B;
+  int cpg = (int)std::max<long long>(1, (total + sms - 1) / sms);
+  cpg = std::min(cpg, nchunks);
+  c->ngroups = (nchunks + cpg - 1) / cpg;
+  c->chunks_per_group = (nchunks + c->ngroups - 1) / c->ngroups;
+  const size_t dd = (size_t)d_k * d_k;
+  bool ok = true;
+  for (int i = 0; i < 3 && ok; ++i) ok = dev_alloc(&c->W[i], (size_t)H * dd, &c->bytes);
+  for (int i = 0; i < 2 && ok; ++i) ok = dev_alloc(&c->S[i], c->state_elems(), &c->bytes);
+  ok = ok && dev_alloc(&c->S_bf16, 2 * c->state_elems(), &c->bytes);
+  ok = ok && dev_alloc(&c->part, (size_t)B * H * c->ngroups * dd, &c->bytes);
+  ok = ok && dev_alloc(&c->alpha_part, (size_t)B * H * c->ngroups, &c->bytes);
+  ok = ok && dev_alloc(&c->err, 1, &c->bytes);
+  for (int i = 0; i < 4 && ok; ++i) ok = dev_alloc(&c->stage_bf16[i], c->act_elems(), &c->bytes);
+  for (int i = 0; i < 2 && ok; ++i) ok = dev_alloc(&c->stage_f32[i], (size_t)B * H * T, &c->bytes);
+  if (!ok) {
+    free_ctx(c);
+    return ARL2_ERR_OOM;
+  }
+  ok = cudaMemset(c->S[0], 0, c->state_elems() * 4) == cudaSuccess &&
+       cudaMemset(c->S[1], 0, c->state_elems() * 4) == cudaSuccess &&
+       cudaMemset(c->S_bf16, 0, 2 * c->state_elems() * 2) == cudaSuccess &&
+       cudaMemset(c->err, 0, sizeof(unsigned int)) == cudaSuccess;
+  for (int i = 0; i < 3 && ok; ++i) ok = make_mat_map(&c->tm_w[i], c->W[i], H, d_k);
+  ok = ok && make_mat_map(&c->tm_s, c->S_bf16, 2 * B * H, d_k);
+  if (ok) ok = cudaDeviceSynchronize() == cudaSuccess;
+  if (!ok) {
+    free_ctx(c);
+    return ARL2_ERR_CUDA;
+  }
+  *out = c;
+  return ARL2_OK;
+}
+
+arl2_status arl2_set_feature_maps(arl2_ctx* c, const arl2_bf16* Wq, const arl2_bf16* Wk, const arl2_bf16* Wv,
+                                  arl2_stream stream) {
+  if (!c || !Wq || !Wk || !Wv) return ARL2_ERR_INVALID_ARG;
+  const size_t bytes = (size_t)c->H * c->d * c->d * 2;
+  const arl2_bf16* src[3] = {Wq, Wk, Wv};
+  for (int i = 0; i < 3; ++i)
+    if (cudaMemcpyAsync(c->W[i], src[i], bytes, cudaMemcpyDefault, (cudaStream_t)stream) != cudaSuccess)
+      return ARL2_ERR_CUDA;
+  c->maps_set = true;
+  return ARL2_OK;
+}
+
+arl2_status arl2_frame_query(arl2_ctx* c, const arl2_bf16* q, const arl2_bf16* k, const arl2_bf16* v, arl2_bf16* o,
+                             arl2_stream stream) {
+  if (!c || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ARL2_ERR_INVALID_ARG;
+  if (!c->maps_set) return ARL2_ERR_STATE;
+  return query_impl(c, q, k, v, o, (cudaStream_t)stream);
+}
+
+arl2_status arl2_frame_commit(arl2_ctx* c, const arl2_bf16* k, const arl2_bf16* v, const float* alpha,
+                              const float* beta, arl2_stream stream) {
+  if (!c || !aligned16(k) || !aligned16(v) || !aligned4(alpha) || !aligned4(beta)) return ARL2_ERR_INVALID_ARG;
+  if (!c->maps_set) return ARL2_ERR_STATE;
+  return commit_impl(c, k, v, alpha, beta, (cudaStream_t)stream);
+}
+
+arl2_status arl2_frame_query_host(arl2_ctx* c, const arl2_bf16* q, const arl2_bf16* k, const arl2_bf16* v,
+                                  arl2_bf16* o, arl2_stream stream) {
+  if (!c || !q || !k || !v || !o) return ARL2_ERR_INVALID_ARG;
+  if (!c->maps_set) return ARL2_ERR_STATE;
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t bytes = c->act_elems() * 2;
+  const arl2_bf16* src[3] = {q, k, v};
+  for (int i = 0; i < 3; ++i)
+    if (cudaMemcpyAsync(c->stage_bf16[i], src[i], bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+      return ARL2_ERR_CUDA;
+  arl2_status s = query_impl(c, c->stage_bf16[0], c->stage_bf16[1], c->stage_bf16[2], c->stage_bf16[3], st);
+  if (s != ARL2_OK) return s;
+  return cudaMemcpyAsync(o, c->stage_bf16[3], bytes, cudaMemcpyDeviceToHost, st) == cudaSuccess ? ARL2_OK
+                                                                                                : ARL2_ERR_CUDA;
+}
+
+arl2_status arl2_frame_commit_host(arl2_ctx* c, const arl2_bf16* k, const arl2_bf16* v, const float* alpha,
+                                   const float* beta, arl2_stream stream) {
+  if (!c || !k || !v || !alpha || !beta) return ARL2_ERR_INVALID_ARG;
+  if (!c->maps_set) return ARL2_ERR_STATE;
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t bytes = c->act_elems() * 2, gbytes = (size_t)c->B * c->H * c->T * 4;
+  if (cudaMemcpyAsync(c->stage_bf16[1], k, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(c->stage_bf16[2], v, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(c->stage_f32[0], alpha, gbytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(c->stage_f32[1], beta, gbytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return ARL2_ERR_CUDA;
+  return commit_impl(c, c->stage_bf16[1], c->stage_bf16[2], c->stage_f32[0], c->stage_f32[1], st);
+}
+
+arl2_status arl2_reset(arl2_ctx* c, arl2_stream stream) {
+  if (!c) return ARL2_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaMemsetAsync(c->S[0], 0, c->state_elems() * 4, st) != cudaSuccess ||
+      cudaMemsetAsync(c->S[1], 0, c->state_elems() * 4, st) != cudaSuccess ||
+      cudaMemsetAsync(c->S_bf16, 0, 2 * c->state_elems() * 2, st) != cudaSuccess)
+    return ARL2_ERR_CUDA;
+  c->cur = 0;
+  c->frame = 0;
+  return ARL2_OK;
+}
+
+arl2_status arl2_get_state(const arl2_ctx* c, float* dst, arl2_stream stream) {
+  if (!c || !dst) return ARL2_ERR_INVALID_ARG;
+  return cudaMemcpyAsync(dst, c->S[c->cur], c->state_elems() * 4, cudaMemcpyDefault, (cudaStream_t)stream) ==
+                 cudaSuccess
+             ? ARL2_OK
+             : ARL2_ERR_CUDA;
+}
+
+arl2_status arl2_set_state(arl2_ctx* c, const float* src, arl2_stream stream) {
+  if (!c || !src) return ARL2_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t n = c->state_elems();
+  // Stage through the other buffer so that host sources work too, then convert in place.
+  float* tmp = c->S[c->cur ^ 1];
+  if (cudaMemcpyAsync(tmp, src, n * 4, cudaMemcpyDefault, st) != cudaSuccess) return ARL2_ERR_CUDA;
+  return arl2::launch_state_import(tmp, c->S[c->cur], c->S_bf16 + (size_t)c->cur * n, n, st) == cudaSuccess
+             ? ARL2_OK
+             : ARL2_ERR_CUDA;
+}
+
+int arl2_frame_index(const arl2_ctx* c) { return c ? c->frame : -1; }
+
+static arl2_status read_status(unsigned int* err) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return ARL2_ERR_CUDA;
+  unsigned int h = 0;
+  if (cudaMemcpy(&h, err, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return ARL2_ERR_CUDA;
+  if (h != 0 && cudaMemset(err, 0, sizeof(h)) != cudaSuccess) return ARL2_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return ARL2_ERR_CUDA;
+  return (h & arl2::kErrTimeoutBit) ? ARL2_ERR_TIMEOUT : ARL2_OK;
+}
+
+arl2_status arl2_get_status(arl2_ctx* c) {
+  if (!c) return ARL2_ERR_INVALID_ARG;
+  return read_status(c->err);
+}
+
+arl2_status arl2_set_wait_timeout_ns(arl2_ctx* c, uint64_t timeout_ns) {
+  if (!c || timeout_ns == 0) return ARL2_ERR_INVALID_ARG;
+  c->timeout_ns = timeout_ns;
+  return ARL2_OK;
+}
+
+size_t arl2_memory_bytes(const arl2_ctx* c) { return c ? c->bytes : 0; }
+
+void arl2_destroy(arl2_ctx* c) { free_ctx(c); }
+
+// ------------------------------------------------------------------ KV-cache baseline
+arl2_status arl2_kvcache_create(int H, int T, int d, int B, int max_frames, arl2_kvcache** out) {
+  if (!out) return ARL2_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (H < 1 || B < 1 || T < 1 || d < 1 || max_frames < 1) return ARL2_ERR_INVALID_ARG;
+  if ((d != 32 && d != 64 && d != 128) || (long long)B * H > 65535 || (long long)T * max_frames > (1ll << 30))
+    return ARL2_ERR_UNSUPPORTED;
+  int dev = 0, sms = 0;
+  arl2_status s = check_device(&dev, &sms);
+  if (s != ARL2_OK) return s;
+  arl2_kvcache* c = new (std::nothrow) arl2_kvcache();
+  if (!c) return ARL2_ERR_OOM;
+  c->B = B;
+  c->H = H;
+  c->T = T;
+  c->d = d;
+  c->max_frames = max_frames;
+  c->device = dev;
+  const size_t elems = (size_t)B * max_frames * T * H * d;
+  bool ok = dev_alloc(&c->K, elems, &c->bytes) && dev_alloc(&c->V, elems, &c->bytes) &&
+            dev_alloc(&c->err, 1, &c->bytes);
+  if (ok)
+    ok = cudaMemset(c->K, 0, elems * 2) == cudaSuccess && cudaMemset(c->V, 0, elems * 2) == cudaSuccess &&
+         cudaMemset(c->err, 0, 4) == cudaSuccess && make_act_map(&c->tm_k, c->K, B, max_frames * T, H, d) &&
+         make_act_map(&c->tm_v, c->V, B, max_frames * T, H, d) && cudaDeviceSynchronize() == cudaSuccess;
+  if (!ok) {
+    cudaFree(c->K);
+    cudaFree(c->V);
+    cudaFree(c->err);
+    delete c;
+    return ARL2_ERR_OOM;
+  }
+  *out = c;
+  return ARL2_OK;
+}
+
+static arl2_status kv_write_slot(arl2_kvcache* c, const void* k, const void* v, cudaStream_t st) {
+  const size_t row = (size_t)c->T * c->H * c->d * 2;          // one frame of one batch entry
+  const size_t pitch = (size_t)c->max_frames * row;             // one batch entry of the cache
+  const size_t off = (size_t)c->n * c->T * c->H * c->d;
+  if (cudaMemcpy2DAsync(c->K + off, pitch, k, row, row, c->B, cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
+      cudaMemcpy2DAsync(c->V + off, pitch, v, row, row, c->B, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return ARL2_ERR_CUDA;
+  return ARL2_OK;
+}
+
+arl2_status arl2_kvcache_query(arl2_kvcache* c, const arl2_bf16* q, const arl2_bf16* k, const arl2_bf16* v,
+                               arl2_bf16* o, arl2_stream stream) {
+  if (!c || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ARL2_ERR_INVALID_ARG;
+  if (c->n >= c->max_frames) return ARL2_ERR_STATE;
+  cudaStream_t st = (cudaStream_t)stream;
+  arl2_status s = kv_write_slot(c, k, v, st);
+  if (s != ARL2_OK) return s;
+  const CUtensorMap* mq = c->acts.get(q, c->B, c->T, c->H, c->d);
+  if (!mq) return ARL2_ERR_CUDA;
+  arl2::QueryArgs a{};
+  a.o = o;
+  a.T = c->T;
+  a.kv_len = (c->n + 1) * c->T;
+  a.B = c->B;
+  a.H = c->H;
+  a.d = c->d;
+  a.state_slot = 0;
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->d)));
+  a.err = c->err;
+  a.timeout_ns = c->timeout_ns;
+  return arl2::launch_query(false, *mq, c->tm_k, c->tm_v, c->tm_k, c->tm_k, a, st) == cudaSuccess ? ARL2_OK
+                                                                                                  : ARL2_ERR_CUDA;
+}
+
+arl2_status arl2_kvcache_commit(arl2_kvcache* c, const arl2_bf16* k, const arl2_bf16* v, arl2_stream stream) {
+  if (!c || !aligned16(k) || !aligned16(v)) return ARL2_ERR_INVALID_ARG;
+  if (c->n >= c->max_frames) return ARL2_ERR_STATE;
+  arl2_status s = kv_write_slot(c, k, v, (cudaStream_t)stream);
+  if (s != ARL2_OK) return s;
+  ++c->n;
+  return ARL2_OK;
+}
+
+arl2_status arl2_kvcache_reset(arl2_kvcache* c) {
+  if (!c) return ARL2_ERR_INVALID_ARG;
+  c->n = 0;
+  return ARL2_OK;
+}
+
+int arl2_kvcache_frames(const arl2_kvcache* c) { return c ? c->n : -1; }
+
+arl2_status arl2_kvcache_get_status(arl2_kvcache* c) {
+  if (!c) return ARL2_ERR_INVALID_ARG;
+  return read_status(c->err);
+}
+
+size_t arl2_kvcache_memory_bytes(const arl2_kvcache* c) { return c ? c->bytes : 0; }
+
+void arl2_kvcache_destroy(arl2_kvcache* c) {
+  if (!c) return;
+  cudaFree(c->K);
+  cudaFree(c->V);
+  cudaFree(c->err);
+  delete c;
+}
+
+}  // extern "C"

@@ -1,0 +1,64 @@
+// Internal (C++) interface between the C-ABI layer and the kernels. Not part of the
+// public boundary, which is include/arl2.h.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace arl2 {
+
+constexpr unsigned int kErrTimeoutBit = 1u;  // device error word: a bounded wait ran out
+
+// One query pass (and the growing-KV-cache baseline, which shares the main loop).
+struct QueryArgs {
+  uint16_t* o;            // [B, T, H, d] bf16 output
+  int T;                  // query rows per (batch, head)
+  int kv_len;             // keys attended per (batch, head)
+  int B, H, d;
+  int state_slot;         // which state buffer (0 or 1) the readout uses
+  float scale_log2;       // log2(e) / sqrt(d)
+  unsigned int* err;      // device error word
+  unsigned long long timeout_ns;
+};
+
+// One commit, first kernel: per (group of 128-token chunks, head, batch) partial U and
+// partial sum of alpha.
+struct CommitArgs {
+  const float* alpha;     // [B, H, T]
+  const float* beta;      // [B, H, T]
+  float* part;            // [B*H*ngroups, d, d] partial K'^T diag(beta/T) (V' - K'S)
+  float* alpha_part;      // [B*H*ngroups] partial sums of alpha
+  int T, B, H, d;
+  int chunks_per_group, ngroups;
+  int state_slot;         // state buffer read (S_{N-1})
+  float inv_T;
+  unsigned int* err;
+  unsigned long long timeout_ns;
+};
+
+// Second kernel: S_N = abar * S_{N-1} + sum of partials, fp32 plus its bf16 copy.
+struct ReduceArgs {
+  const float* part;
+  const float* alpha_part;
+  const float* S_old;     // [B*H, d, d]
+  float* S_new;           // [B*H, d, d]
+  uint16_t* S_new_bf16;   // [B*H, d, d]
+  int d, ngroups, BH;
+  float inv_T;
+};
+
+size_t query_smem_bytes();
+size_t commit_smem_bytes();
+cudaError_t query_setup();   // per-device function attributes
+cudaError_t commit_setup();
+
+cudaError_t launch_query(bool hybrid, const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                         const CUtensorMap& tm_w, const CUtensorMap& tm_s, const QueryArgs& a, cudaStream_t stream);
+cudaError_t launch_commit(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const CUtensorMap& tm_wk,
+                          const CUtensorMap& tm_wv, const CUtensorMap& tm_s, const CommitArgs& a,
+                          const ReduceArgs& r, cudaStream_t stream);
+// fp32 state -> state buffer + bf16 copy.
+cudaError_t launch_state_import(const float* src, float* S, uint16_t* S_bf16, size_t n, cudaStream_t stream);
+
+}  // namespace arl2

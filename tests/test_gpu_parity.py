@@ -1,0 +1,238 @@
+"""Parity of the CUDA layer (through the C ABI) with the fp64 oracle, and the layer's
+GPU-side contracts (state untouched by queries, determinism, constant memory, bounded waits).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from arl2_cases import O_TOL, S_TOL, Case, dev_bf16, dev_f32, host_f64, o_errors, s_error, sample_rows
+from softmax_attention_ar_b200 import arl2, synth
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # the gpu marker deselects these on CPU-only machines
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+
+# ------------------------------------------------------------------ parity over frames
+def test_tiny_config_every_call():
+    # Tiny oracle check: B=1, H=2, T=64, d=32, 4 frames of 2 queries + 1 commit.
+    w = synth.WORKLOADS["tiny"]
+    c = Case(w["B"], w["T"], w["H"], w["d"], config=w["config"])
+    c.run(w["frames"], w["queries"])
+
+
+def test_several_tiles_ragged_tail_batched():
+    c = Case(B=2, T=300, H=3, d=128, config=101)
+    c.run(frames=3, queries=2)
+
+
+@pytest.mark.parametrize("d", [32, 64])
+def test_smaller_head_dims(d):
+    c = Case(B=1, T=200, H=2, d=d, config=102)
+    c.run(frames=2, queries=2)
+
+
+@pytest.mark.parametrize("T", [1, 2, 127, 128, 129, 255])
+def test_edge_token_counts(T):
+    c = Case(B=1, T=T, H=2, d=128, config=103)
+    c.run(frames=2, queries=2)
+
+
+def test_480p_21_frames_sampled_rows():
+    # 480p single layer: B=1, H=12, d=128, T=1560, 21 frames of 4 queries + 1 commit.
+    w = synth.WORKLOADS["480p"]
+    c = Case(w["B"], w["T"], w["H"], w["d"], config=w["config"])
+    worst_o, worst_s = c.run(w["frames"], w["queries"], rows=sample_rows(w["T"]))
+    assert worst_o <= O_TOL and worst_s <= S_TOL
+
+
+def test_maximum_tokens_per_frame():
+    c = Case(B=1, T=4096, H=2, d=128, config=104)
+    c.run(frames=2, queries=1, rows=sample_rows(4096))
+
+
+@pytest.mark.parametrize("B,T", [(1, 390), (4, 3600)])
+def test_sweep_shapes(B, T):
+    # Token/batch sweep shapes, H=12, d=128; the largest is checked on sampled rows.
+    c = Case(B=B, T=T, H=12, d=128, config=3)
+    rows = None if T <= 400 else sample_rows(T, n=24)
+    c.run(frames=2, queries=2 if rows is None else 1, rows=rows)
+
+
+# ------------------------------------------------------------------ closed forms on the GPU
+def test_queries_leave_the_state_bit_identical():
+    c = Case(B=1, T=300, H=2, d=128, config=105)
+    c.commit(0)
+    before = c.gpu.get_state().clone()
+    for p in range(4):
+        c.query(1, p)
+    torch.cuda.synchronize()
+    assert torch.equal(c.gpu.get_state(), before)
+
+
+def test_alpha_one_beta_zero_keeps_the_state_bit_identical():
+    c = Case(B=1, T=300, H=2, d=128, config=106)
+    c.gpu.set_state(dev_f32(synth.state(0, 106, 1, 2, 128)))
+    before = c.gpu.get_state().clone()
+    _, k, v = c.inputs(0, synth.CLEAN_PASS)
+    ones = torch.ones((1, 2, 300), device="cuda")
+    c.gpu.commit(dev_bf16(k), dev_bf16(v), ones, torch.zeros_like(ones))
+    assert torch.equal(c.gpu.get_state(), before)
+
+
+def test_readout_branch_with_a_set_state():
+    # A unit-variance state makes the readout dominate O, which isolates phi_q and Q'S.
+    B, T, H, d = 1, 260, 3, 128
+    c = Case(B, T, H, d, config=107)
+    S0 = synth.state(0, 107, B, H, d)
+    c.gpu.set_state(dev_f32(S0))
+    c.ref.S = S0.astype(np.float64)
+    o_gpu, o_ref = c.query(0, 0)
+    assert max(o_errors(o_gpu, o_ref)) <= O_TOL
+    q, k, v = c.inputs(0, 0)
+    o_inter = oracle.readout(synth.bf16_to_f64(q), c.ref.Wq, c.ref.S)
+    assert np.abs(o_inter).max() > 5 * np.abs(o_ref - o_inter).max()  # readout-dominated
+
+
+def test_pure_decay_over_many_frames():
+    # beta = 0 and alpha = c for N frames: S_N = c^N S_0.
+    B, T, H, d = 1, 130, 2, 64
+    c = Case(B, T, H, d, config=108)
+    S0 = synth.state(0, 108, B, H, d)
+    c.gpu.set_state(dev_f32(S0))
+    _, k, v = c.inputs(0, synth.CLEAN_PASS)
+    kk, vv = dev_bf16(k), dev_bf16(v)
+    cst = 0.97
+    alpha = torch.full((B, H, T), cst, device="cuda")
+    beta = torch.zeros_like(alpha)
+    for n in range(1, 61):
+        c.gpu.commit(kk, vv, alpha, beta)
+        if n in (1, 60):
+            S = host_f64(c.gpu.get_state())
+            np.testing.assert_allclose(S, float(np.float32(cst)) ** n * S0, rtol=1e-4, atol=1e-6)
+
+
+def test_single_unit_key_writes_its_value():
+    # T=1, unit key (phi_k = I), beta/T = 1, alpha = 1: K' S_N = V' (= v @ Wv).
+    B, T, H, d = 1, 1, 1, 128
+    layer = arl2.ARL2Layer(H, T, d, B)
+    eye = dev_bf16(synth.bf16_bits(np.eye(d, dtype=np.float32)[None]))
+    _, _, wv = synth.feature_maps(0, 109, H, d)
+    layer.set_feature_maps(eye, eye, dev_bf16(wv))
+    layer.set_state(dev_f32(synth.state(0, 109, B, H, d, scale=0.1)))
+    k = np.zeros((B, T, H, d), np.float32); k[..., 5] = 1.0
+    v = np.random.default_rng(0).standard_normal((B, T, H, d)).astype(np.float32)
+    kb, vb = synth.bf16_bits(k), synth.bf16_bits(v)
+    one = torch.ones((B, H, T), device="cuda")
+    layer.commit(dev_bf16(kb), dev_bf16(vb), one, one)
+    S = host_f64(layer.get_state())
+    vp = synth.bf16_to_f64(vb)[0, 0, 0] @ synth.bf16_to_f64(wv)[0]
+    np.testing.assert_allclose(S[0, 0, 5], vp, rtol=0, atol=2e-2 * np.abs(vp).max())
+
+
+# ------------------------------------------------------------------ contracts
+def test_deterministic_outputs_and_state():
+    results = []
+    for _ in range(2):
+        c = Case(B=1, T=520, H=4, d=128, config=110)
+        outs = []
+        for f in range(2):
+            q, k, v = c.inputs(f, 0)
+            outs.append(c.gpu.query(dev_bf16(q), dev_bf16(k), dev_bf16(v)).clone())
+            c.commit(f)
+        outs.append(c.gpu.get_state().clone())
+        results.append(outs)
+        c.gpu.close()
+    for x, y in zip(*results):
+        assert torch.equal(x, y)
+
+
+def test_long_stream_constant_memory_and_state_parity():
+    # Long streaming: 480p shapes over 240 frames; memory constant; S checked at 1, 60, 240.
+    w = synth.WORKLOADS["stream240"]
+    B, T, H, d = w["B"], w["T"], w["H"], w["d"]
+    c = Case(B, T, H, d, config=w["config"])
+    q, k, v = (dev_bf16(x) for x in c.inputs(0, 0))
+    o = torch.empty_like(q)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    held0 = c.gpu.memory_bytes
+    for f in range(w["frames"]):
+        for _ in range(w["queries"]):
+            c.gpu.query(q, k, v, out=o)
+        s_gpu, s_ref = c.commit(f)   # the oracle replays only the commits
+        if f + 1 in (1, 60, 240):
+            assert s_error(s_gpu, s_ref) <= S_TOL, f"frame {f + 1}"
+    torch.cuda.synchronize()
+    assert c.gpu.memory_bytes == held0
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert c.gpu.frame_index == 240
+    assert c.gpu.status() == arl2.ARL2_OK
+
+
+def test_host_buffer_calls_match_device_calls():
+    B, T, H, d = 1, 300, 2, 128
+    a = Case(B, T, H, d, config=111)
+    b = Case(B, T, H, d, config=111)
+    q, k, v = a.inputs(0, 0)
+    o_dev = a.gpu.query(dev_bf16(q), dev_bf16(k), dev_bf16(v))
+    pin = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    o_host = torch.empty((B, T, H, d), dtype=torch.bfloat16).pin_memory()
+    b.gpu.query_host(pin(q), pin(k), pin(v), o_host)
+    torch.cuda.synchronize()
+    assert torch.equal(o_dev.cpu(), o_host)
+    _, k, v = a.inputs(0, synth.CLEAN_PASS)
+    al, be = a.gates(0)
+    a.gpu.commit(dev_bf16(k), dev_bf16(v), dev_f32(al), dev_f32(be))
+    b.gpu.commit_host(pin(k), pin(v), torch.from_numpy(al).pin_memory(), torch.from_numpy(be).pin_memory())
+    torch.cuda.synchronize()
+    assert torch.equal(a.gpu.get_state(), b.gpu.get_state())
+
+
+def test_reset_and_out_of_order_calls():
+    layer = arl2.ARL2Layer(2, 64, 32, 1)
+    x = torch.zeros((1, 64, 2, 32), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(arl2.Arl2Error) as e:
+        layer.query(x, x, x)
+    assert e.value.status == arl2.ARL2_ERR_STATE
+    c = Case(B=1, T=64, H=2, d=32, config=112)
+    c.commit(0)
+    assert c.gpu.frame_index == 1 and torch.any(c.gpu.get_state() != 0)
+    c.gpu.reset()
+    assert c.gpu.frame_index == 0 and torch.all(c.gpu.get_state() == 0)
+
+
+def test_bounded_waits_report_a_timeout_and_leave_the_context_usable():
+    # A 1 ns wait limit makes ordinary waits run out: the kernels abandon the call and return.
+    c = Case(B=1, T=300, H=2, d=128, config=113)
+    q, k, v = (dev_bf16(x) for x in c.inputs(0, 0))
+    c.gpu.set_wait_timeout_ns(1)
+    c.gpu.query(q, k, v)
+    assert c.gpu.status() == arl2.ARL2_ERR_TIMEOUT
+    c.gpu.set_wait_timeout_ns(1_000_000_000)
+    assert c.gpu.status() == arl2.ARL2_OK
+    o_gpu, o_ref = c.query(0, 0)
+    assert max(o_errors(o_gpu, o_ref)) <= O_TOL
+
+
+# ------------------------------------------------------------------ growing-KV baseline
+def test_kv_cache_baseline_parity():
+    B, T, H, d, frames = 1, 200, 2, 128, 3
+    base = arl2.KVCacheBaseline(H, T, d, B, max_frames=frames)
+    kc, vc = [], []
+    for f in range(frames):
+        for p in range(2):
+            q, k, v = synth.qkv(0, 114, f, p, B, T, H, d)
+            o = host_f64(base.query(dev_bf16(q), dev_bf16(k), dev_bf16(v)))
+            keys = np.concatenate(kc + [synth.bf16_to_f64(k)], axis=1)
+            vals = np.concatenate(vc + [synth.bf16_to_f64(v)], axis=1)
+            ref = oracle.kv_cache_attention(synth.bf16_to_f64(q), keys, vals, (f + 1) * T)
+            assert max(o_errors(o, ref)) <= O_TOL
+        _, k, v = synth.qkv(0, 114, f, synth.CLEAN_PASS, B, T, H, d)
+        base.commit(dev_bf16(k), dev_bf16(v))
+        kc.append(synth.bf16_to_f64(k))
+        vc.append(synth.bf16_to_f64(v))
+    assert base.frames == frames
+    assert base.status() == arl2.ARL2_OK
