@@ -272,17 +272,19 @@ def run_ours(args, rank, world, local_rank):
         _, k, v = passes[QUERIES]
         layer.commit_host(k, v, a, b)
 
-    e2e_steps = max(1, min(args.steps, 200))
-    for i in range(min(args.warmup, 3)):
-        host_step(i)
-    barrier()
-    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s2.record(stream)
-    for i in range(e2e_steps):
-        host_step(i)
-    e2.record(stream)
-    barrier()
-    e2e_ms = s2.elapsed_time(e2)
+    e2e_steps = max(1, min(args.steps, 200)) if not args.no_e2e else 0
+    e2e_ms = float("nan")
+    if e2e_steps:
+        for i in range(min(args.warmup, 3)):
+            host_step(i)
+        barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for i in range(e2e_steps):
+            host_step(i)
+        e2.record(stream)
+        barrier()
+        e2e_ms = s2.elapsed_time(e2)
     act = B * T * H * D * 2
     h2d = (QUERIES * 3 + 2) * act + 2 * B * H * T * 4
     d2h = QUERIES * act
@@ -295,7 +297,7 @@ def run_ours(args, rank, world, local_rank):
     if rank != 0:
         return
     value = world * B * args.steps / (elapsed_ms / 1e3)
-    e2e_value = world * B * e2e_steps / (e2e_ms / 1e3)
+    e2e_value = world * B * e2e_steps / (e2e_ms / 1e3) if e2e_steps else None
     peaks = _peaks()
     q_mean_s = statistics.mean(q_ms) / 1e3
     c_mean_s = statistics.mean(c_ms) / 1e3
@@ -332,7 +334,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer (e2e) measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
