@@ -134,6 +134,41 @@ size_t arl2_memory_bytes(const arl2_ctx* ctx);
  * in flight. NULL is ignored. */
 void arl2_destroy(arl2_ctx* ctx);
 
+/* ---- Allocation-free commit ------------------------------------------------------------
+ * This entry point has no counterpart in the paper. It exists for callers that cannot
+ * call cudaMalloc. Examples: a serving engine that reserved all device memory for its own
+ * pool at start-up; a real-time frame loop that must not take the allocator's locks or
+ * its implicit synchronisation; an embedding that only hands the library memory it owns.
+ *
+ * It computes the same update as arl2_frame_commit without a context:
+ *   S_next = abar S_prev + K'^T diag(beta / T) (V' - K' S_prev)
+ * The arguments are:
+ *   - k, v: bf16 [B, T, H, d].
+ *   - alpha, beta: fp32 [B, H, T].
+ *   - Wk, Wv: bf16 [H, d, d].
+ *   - S_prev, S_next: fp32 [B, H, d, d]. S_next may be S_prev itself (an in-place
+ *     update) or must not overlap it.
+ *   - status: optional device word, ORed with 1 if a kernel's bounded wait ran out. The
+ *     caller zeroes it; NULL uses an internal word.
+ *
+ * The call allocates nothing. Its scratch is a fixed device array of
+ * ARL2_NOALLOC_SCRATCH_BYTES inside the library. Every GPU that loads the library holds
+ * that array until the process exits. Shapes whose scratch would exceed it return
+ * ARL2_ERR_UNSUPPORTED before any work is enqueued. The need is about
+ * B*H*d*d*8 + B*H*g*d*d*4 bytes, with g <= ceil(T/128) chunk groups; B=1, H=12, d=128,
+ * T=1560 needs about 7.1 MB.
+ *
+ * The first call on a device looks the array's device address up, with that device
+ * current. Make that first call before any stream capture. All calls on a device share
+ * the one array and leave their contents in it. Each call clears what it needs at zero.
+ * Calls that overlap on the GPU, for example on two streams, race on the array.
+ * Supported shapes are as for arl2_create. */
+#define ARL2_NOALLOC_SCRATCH_BYTES (16u << 20)
+arl2_status arl2_frame_commit_noalloc(int B, int H, int T, int d, const arl2_bf16* k, const arl2_bf16* v,
+                                      const float* alpha, const float* beta, const arl2_bf16* Wk,
+                                      const arl2_bf16* Wv, const float* S_prev, float* S_next,
+                                      unsigned int* status, arl2_stream stream);
+
 /* ---- Growing-KV-cache baseline (comparison only; §1 problem statement) -----------------
  * This is full softmax attention of the newest frame over the keys and values of every
  * frame so far, which is what the layer above replaces. Its cache grows by one frame per

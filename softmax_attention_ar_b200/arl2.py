@@ -40,6 +40,7 @@ SIGNATURES = {
     "arl2_set_wait_timeout_ns": (_S, [_P, _U64]),
     "arl2_memory_bytes": (_SZ, [_P]),
     "arl2_destroy": (None, [_P]),
+    "arl2_frame_commit_noalloc": (_S, [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "arl2_kvcache_create": (_S, [_I, _I, _I, _I, _I, ctypes.POINTER(_P)]),
     "arl2_kvcache_query": (_S, [_P, _P, _P, _P, _P, _P]),
     "arl2_kvcache_commit": (_S, [_P, _P, _P, _P]),
@@ -210,6 +211,29 @@ class ARL2Layer:
     @property
     def memory_bytes(self) -> int:
         return self._lib.arl2_memory_bytes(self._ctx)
+
+
+def frame_commit_noalloc(k, v, alpha, beta, Wk, Wv, S_prev, S_next, status=None, stream=None) -> None:
+    """Commit without a context or any allocation (arl2_frame_commit_noalloc).
+
+    For callers that cannot allocate device memory: the library's fixed scratch array is
+    used instead. k, v bf16 [B, T, H, d]; alpha, beta fp32 [B, H, T]; Wk, Wv bf16 [H, d, d];
+    S_prev, S_next fp32 [B, H, d, d] (S_next may be S_prev); status an optional int32 [1]
+    device word the caller zeroed.
+    """
+    B, T, H, d = k.shape
+    s, g, w, st = (B, T, H, d), (B, H, T), (H, d, d), (B, H, d, d)
+    status_ptr = None
+    if status is not None:
+        if status.dtype != torch.int32 or status.numel() != 1:
+            raise ValueError("status: expected one int32 element")
+        status_ptr = status.data_ptr()
+    _check(load_library().arl2_frame_commit_noalloc(
+        B, H, T, d, _dev(k, torch.bfloat16, s, "k"), _dev(v, torch.bfloat16, s, "v"),
+        _dev(alpha, torch.float32, g, "alpha"), _dev(beta, torch.float32, g, "beta"),
+        _dev(Wk, torch.bfloat16, w, "Wk"), _dev(Wv, torch.bfloat16, w, "Wv"),
+        _dev(S_prev, torch.float32, st, "S_prev"), _dev(S_next, torch.float32, st, "S_next"),
+        status_ptr, _stream(stream)), "arl2_frame_commit_noalloc")
 
 
 class KVCacheBaseline:

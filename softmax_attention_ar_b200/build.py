@@ -18,7 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libarl2.so")
 BUILD_DIR = os.path.join(PKG, "_build")
-SOURCES = ["arl2_api.cu", "arl2_query.cu", "arl2_commit.cu"]
+SOURCES = ["arl2_api.cu", "arl2_query.cu", "arl2_commit.cu", "arl2_noalloc.cu"]
 HEADERS = ["arl2_device.cuh", "arl2_kernels.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -110,6 +110,15 @@ constexpr unsigned long long kDefaultTimeoutNs = 1000000000ull;
 
 }  // namespace
 
+// Entry points for other translation units of the library (the allocation-free commit).
+namespace arl2 {
+int prepare_device(int* dev, int* sms) { return static_cast<int>(check_device(dev, sms)); }
+bool encode_act_map(CUtensorMap* m, const void* ptr, int B, int L, int H, int d) {
+  return make_act_map(m, ptr, B, L, H, d);
+}
+bool encode_mat_map(CUtensorMap* m, const void* ptr, int n, int d) { return make_mat_map(m, ptr, n, d); }
+}  // namespace arl2
+
 struct arl2_ctx {
   int B = 0, H = 0, T = 0, d = 0;
   int device = 0, num_sms = 0;

@@ -48,6 +48,12 @@ struct ReduceArgs {
   float inv_T;
 };
 
+// Helpers defined in arl2_api.cu: device check and set-up (returns an arl2_status), and
+// the bf16 tensor maps every kernel reads through.
+int prepare_device(int* dev, int* sms);
+bool encode_act_map(CUtensorMap* m, const void* ptr, int B, int L, int H, int d);
+bool encode_mat_map(CUtensorMap* m, const void* ptr, int n, int d);
+
 size_t query_smem_bytes();
 size_t commit_smem_bytes();
 cudaError_t query_setup();   // per-device function attributes
