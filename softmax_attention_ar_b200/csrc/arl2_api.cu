@@ -131,6 +131,9 @@ struct arl2_ctx {
   unsigned int* err = nullptr;
   uint16_t* stage_bf16[4] = {};   // q, k, v, o staging for the host-buffer calls
   float* stage_f32[2] = {};       // alpha, beta staging
+  arl2::QueryPlan qplan{};        // stream-K split of the query kernel
+  float* qscratch = nullptr;      // its partial records
+  int* qcnt = nullptr;            // its per-query-tile counters
   int cur = 0;                    // buffer holding S_{N-1}
   int frame = 0;
   bool maps_set = false;
@@ -155,9 +158,28 @@ struct arl2_kvcache {
   MapCache acts;
   size_t bytes = 0;
   unsigned long long timeout_ns = kDefaultTimeoutNs;
+  int num_sms = 0;
+  float* qscratch = nullptr;      // stream-K partial records, sized for the longest cache
+  size_t qscratch_floats = 0;
+  int* qcnt = nullptr;            // per-query-tile counters
+  long long qtiles = 0;
 };
 
 namespace {
+
+// Point a query launch at its stream-K plan and scratch.
+void set_plan(arl2::QueryArgs* a, const arl2::QueryPlan& p, float* scratch, int* cnt) {
+  a->nq = p.nq;
+  a->nkv = p.nkv;
+  a->units = p.units;
+  a->num_ctas = p.num_ctas;
+  a->max_segs = p.max_segs;
+  const size_t slots = static_cast<size_t>(p.qtiles) * p.max_segs;
+  a->part_o = scratch;
+  a->part_ml = scratch + slots * 128 * 128;
+  a->part_oi = a->part_ml + slots * 2 * 128;
+  a->cnt = cnt;
+}
 
 template <typename T>
 bool dev_alloc(T** p, size_t count, size_t* total) {
@@ -179,6 +201,8 @@ void free_ctx(arl2_ctx* c) {
   cudaFree(c->err);
   for (auto& p : c->stage_bf16) cudaFree(p);
   for (auto& p : c->stage_f32) cudaFree(p);
+  cudaFree(c->qscratch);
+  cudaFree(c->qcnt);
   delete c;
 }
 
@@ -198,6 +222,7 @@ arl2_status query_impl(arl2_ctx* c, const void* q, const void* k, const void* v,
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->d)));
   a.err = c->err;
   a.timeout_ns = c->timeout_ns;
+  set_plan(&a, c->qplan, c->qscratch, c->qcnt);
   return arl2::launch_query(true, *mq, *mk, *mv, c->tm_w[0], c->tm_s, a, st) == cudaSuccess ? ARL2_OK
                                                                                            : ARL2_ERR_CUDA;
 }
@@ -276,6 +301,9 @@ arl2_status arl2_create(int H, int T, int d_k, int d_v, int B, arl2_ctx** out) {
   ok = ok && dev_alloc(&c->err, 1, &c->bytes);
   for (int i = 0; i < 4 && ok; ++i) ok = dev_alloc(&c->stage_bf16[i], c->act_elems(), &c->bytes);
   for (int i = 0; i < 2 && ok; ++i) ok = dev_alloc(&c->stage_f32[i], (size_t)B * H * T, &c->bytes);
+  c->qplan = arl2::plan_query(B, H, T, T, sms);
+  ok = ok && dev_alloc(&c->qscratch, arl2::query_scratch_floats(c->qplan), &c->bytes);
+  ok = ok && dev_alloc(&c->qcnt, (size_t)c->qplan.qtiles, &c->bytes);
   if (!ok) {
     free_ctx(c);
     return ARL2_ERR_OOM;
@@ -283,6 +311,7 @@ arl2_status arl2_create(int H, int T, int d_k, int d_v, int B, arl2_ctx** out) {
   ok = cudaMemset(c->S[0], 0, c->state_elems() * 4) == cudaSuccess &&
        cudaMemset(c->S[1], 0, c->state_elems() * 4) == cudaSuccess &&
        cudaMemset(c->S_bf16, 0, 2 * c->state_elems() * 2) == cudaSuccess &&
+       cudaMemset(c->qcnt, 0, (size_t)c->qplan.qtiles * sizeof(int)) == cudaSuccess &&
        cudaMemset(c->err, 0, sizeof(unsigned int)) == cudaSuccess;
   for (int i = 0; i < 3 && ok; ++i) ok = make_mat_map(&c->tm_w[i], c->W[i], H, d_k);
   ok = ok && make_mat_map(&c->tm_s, c->S_bf16, 2 * B * H, d_k);
@@ -385,18 +414,23 @@ arl2_status arl2_set_state(arl2_ctx* c, const float* src, arl2_stream stream) {
 
 int arl2_frame_index(const arl2_ctx* c) { return c ? c->frame : -1; }
 
-static arl2_status read_status(unsigned int* err) {
+// Synchronise, read and clear the error word. After an abandoned launch the query
+// kernel's tile counters may be left mid-count, so they are cleared too.
+static arl2_status read_status(unsigned int* err, int* cnt, size_t ncnt) {
   if (cudaDeviceSynchronize() != cudaSuccess) return ARL2_ERR_CUDA;
   unsigned int h = 0;
   if (cudaMemcpy(&h, err, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return ARL2_ERR_CUDA;
-  if (h != 0 && cudaMemset(err, 0, sizeof(h)) != cudaSuccess) return ARL2_ERR_CUDA;
+  if (h != 0) {
+    if (cudaMemset(err, 0, sizeof(h)) != cudaSuccess) return ARL2_ERR_CUDA;
+    if (cnt && cudaMemset(cnt, 0, ncnt * sizeof(int)) != cudaSuccess) return ARL2_ERR_CUDA;
+  }
   if (cudaDeviceSynchronize() != cudaSuccess) return ARL2_ERR_CUDA;
   return (h & arl2::kErrTimeoutBit) ? ARL2_ERR_TIMEOUT : ARL2_OK;
 }
 
 arl2_status arl2_get_status(arl2_ctx* c) {
   if (!c) return ARL2_ERR_INVALID_ARG;
-  return read_status(c->err);
+  return read_status(c->err, c->qcnt, (size_t)c->qplan.qtiles);
 }
 
 arl2_status arl2_set_wait_timeout_ns(arl2_ctx* c, uint64_t timeout_ns) {
@@ -427,18 +461,25 @@ arl2_status arl2_kvcache_create(int H, int T, int d, int B, int max_frames, arl2
   c->d = d;
   c->max_frames = max_frames;
   c->device = dev;
+  c->num_sms = sms;
   const size_t elems = (size_t)B * max_frames * T * H * d;
+  // Query scratch for the longest cache any frame reaches.
+  for (int n = 1; n <= max_frames; ++n) {
+    const arl2::QueryPlan p = arl2::plan_query(B, H, T, n * T, sms);
+    c->qscratch_floats = std::max(c->qscratch_floats, arl2::query_scratch_floats(p));
+    c->qtiles = p.qtiles;
+  }
   bool ok = dev_alloc(&c->K, elems, &c->bytes) && dev_alloc(&c->V, elems, &c->bytes) &&
-            dev_alloc(&c->err, 1, &c->bytes);
+            dev_alloc(&c->err, 1, &c->bytes) && dev_alloc(&c->qscratch, c->qscratch_floats, &c->bytes) &&
+            dev_alloc(&c->qcnt, (size_t)c->qtiles, &c->bytes);
   if (ok)
     ok = cudaMemset(c->K, 0, elems * 2) == cudaSuccess && cudaMemset(c->V, 0, elems * 2) == cudaSuccess &&
-         cudaMemset(c->err, 0, 4) == cudaSuccess && make_act_map(&c->tm_k, c->K, B, max_frames * T, H, d) &&
+         cudaMemset(c->err, 0, 4) == cudaSuccess &&
+         cudaMemset(c->qcnt, 0, (size_t)c->qtiles * sizeof(int)) == cudaSuccess &&
+         make_act_map(&c->tm_k, c->K, B, max_frames * T, H, d) &&
          make_act_map(&c->tm_v, c->V, B, max_frames * T, H, d) && cudaDeviceSynchronize() == cudaSuccess;
   if (!ok) {
-    cudaFree(c->K);
-    cudaFree(c->V);
-    cudaFree(c->err);
-    delete c;
+    arl2_kvcache_destroy(c);
     return ARL2_ERR_OOM;
   }
   *out = c;
@@ -475,6 +516,7 @@ arl2_status arl2_kvcache_query(arl2_kvcache* c, const arl2_bf16* q, const arl2_b
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->d)));
   a.err = c->err;
   a.timeout_ns = c->timeout_ns;
+  set_plan(&a, arl2::plan_query(c->B, c->H, c->T, a.kv_len, c->num_sms), c->qscratch, c->qcnt);
   return arl2::launch_query(false, *mq, c->tm_k, c->tm_v, c->tm_k, c->tm_k, a, st) == cudaSuccess ? ARL2_OK
                                                                                                   : ARL2_ERR_CUDA;
 }
@@ -498,7 +540,7 @@ int arl2_kvcache_frames(const arl2_kvcache* c) { return c ? c->n : -1; }
 
 arl2_status arl2_kvcache_get_status(arl2_kvcache* c) {
   if (!c) return ARL2_ERR_INVALID_ARG;
-  return read_status(c->err);
+  return read_status(c->err, c->qcnt, (size_t)c->qtiles);
 }
 
 size_t arl2_kvcache_memory_bytes(const arl2_kvcache* c) { return c ? c->bytes : 0; }
@@ -508,6 +550,8 @@ void arl2_kvcache_destroy(arl2_kvcache* c) {
   cudaFree(c->K);
   cudaFree(c->V);
   cudaFree(c->err);
+  cudaFree(c->qscratch);
+  cudaFree(c->qcnt);
   delete c;
 }
 

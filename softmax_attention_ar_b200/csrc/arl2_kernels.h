@@ -20,7 +20,24 @@ struct QueryArgs {
   float scale_log2;       // log2(e) / sqrt(d)
   unsigned int* err;      // device error word
   unsigned long long timeout_ns;
+  // Persistent stream-K split (see QueryPlan) and its scratch.
+  int nq, nkv;            // query tiles and key tiles per (batch, head)
+  long long units;        // B * H * nq * nkv (query tile, key tile) pairs
+  int num_ctas;           // grid size
+  int max_segs;           // CTAs sharing one query tile, at most
+  float* part_o;          // [qtiles * max_segs, 128, 128] partial O accumulators
+  float* part_ml;         // [qtiles * max_segs, 2, 128] running max (log2 units) and sum
+  float* part_oi;         // [qtiles, 128, 128] O_inter of split query tiles
+  int* cnt;               // [qtiles] arrival counters, zero between launches
 };
+
+// The stream-K split of one query launch: CTA c takes units [c*U/P, (c+1)*U/P).
+struct QueryPlan {
+  int nq, nkv, num_ctas, max_segs;
+  long long units, qtiles;
+};
+QueryPlan plan_query(int B, int H, int T, int kv_len, int num_sms);
+size_t query_scratch_floats(const QueryPlan& p);   // part_o + part_ml + part_oi
 
 // One commit, first kernel: per (group of 128-token chunks, head, batch) partial U and
 // partial sum of alpha.

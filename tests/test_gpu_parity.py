@@ -48,6 +48,14 @@ def test_480p_21_frames_sampled_rows():
     assert worst_o <= O_TOL and worst_s <= S_TOL
 
 
+@pytest.mark.parametrize("B,H,T", [(1, 1, 2048), (1, 2, 200), (2, 3, 300)])
+def test_query_tiles_split_across_many_ctas(B, H, T):
+    # Few query tiles: the persistent split gives each tile to several CTAs (up to its cap
+    # of 8), which merge partial softmax records.
+    c = Case(B=B, T=T, H=H, d=128, config=115)
+    c.run(frames=2, queries=2)
+
+
 def test_maximum_tokens_per_frame():
     c = Case(B=1, T=4096, H=2, d=128, config=104)
     c.run(frames=2, queries=1, rows=sample_rows(4096))
