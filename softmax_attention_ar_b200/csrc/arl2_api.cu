@@ -425,6 +425,7 @@ static arl2_status read_status(unsigned int* err, int* cnt, size_t ncnt) {
     if (cnt && cudaMemset(cnt, 0, ncnt * sizeof(int)) != cudaSuccess) return ARL2_ERR_CUDA;
   }
   if (cudaDeviceSynchronize() != cudaSuccess) return ARL2_ERR_CUDA;
+  if (h & arl2::kErrLayoutBit) return ARL2_ERR_CUDA;
   return (h & arl2::kErrTimeoutBit) ? ARL2_ERR_TIMEOUT : ARL2_OK;
 }
 

@@ -9,6 +9,7 @@
 namespace arl2 {
 
 constexpr unsigned int kErrTimeoutBit = 1u;  // device error word: a bounded wait ran out
+constexpr unsigned int kErrLayoutBit = 2u;   // device error word: shared memory not laid out as required
 
 // One query pass (and the growing-KV-cache baseline, which shares the main loop).
 struct QueryArgs {

@@ -19,25 +19,32 @@
 //     tile in key order and writes O. It then resets the counter. The merge order is
 //     fixed, so the result does not depend on which CTA merges it.
 //
-// Roles (192 threads, one CTA per SM):
-//   warp 0     TMA producer. Per segment: the Q tile, plus Wq_h and the bf16 state copy when
-//              the segment starts the tile. Then K/V tiles into two-stage rings, where K and
-//              V stages are released separately.
-//   warp 1     TMEM owner; lane 0 issues every tcgen05.mma and commit.
-//   warps 2-5  softmax warpgroup: thread = query row = TMEM lane. These threads also pack
-//              Q' to bf16 for the readout MMA, and write outputs and partial records.
+// Roles (384 threads, one CTA per SM):
+//   warp 0      K producer: per segment the Q tile, then K tiles into a three-stage ring.
+//               When a segment starts a tile, Wq_h first goes through the ring like a tile.
+//   warp 1      TMEM owner; lane 0 issues every tcgen05.mma and commit.
+//   warp 2      V producer: V tiles into a three-stage ring. When a segment starts a tile,
+//               the bf16 state copy S_h goes first, through the ring.
+//   warps 4-11  two softmax warpgroups. Thread = query row = TMEM lane; warps 4-7 own
+//               score and output columns 0-63, warps 8-11 columns 64-127. A thread reads
+//               and overwrites only its own 64 columns; the two halves of a row swap
+//               their partial maxima through shared memory once per tile. These threads
+//               also pack Q' to bf16 for the readout MMA and write outputs and partial
+//               records.
 // TMEM (512 columns):
-//   - cols 0 and 128: the two S tiles, double-buffered. P (bf16, 64 columns) overwrites
-//     its own S tile and feeds the P.V MMA straight from TMEM.
+//   - cols 0 and 128: the two S tiles, double-buffered. P (bf16) overwrites its own S tile:
+//     scores 0-63 are packed into columns 0-31 and scores 64-127 into columns 64-95. The
+//     P.V MMA reads them straight from TMEM.
 //   - col 256: O. At the start of a segment that starts a tile, it briefly holds Q' packed
 //     to bf16 for the readout MMA.
 //   - col 384: Q' (fp32), then O_inter.
-// Shared memory: Q | K0 K1 | V0 V1 | Wq | S (32 KiB tiles).
+// Shared memory: Q | K0 K1 K2 | V0 V1 V2 (32 KiB tiles) from its 1 KiB-aligned base, then a
+// small control block (mbarriers, flags, the max/sum exchange slots).
 //
 // Online softmax: scores are kept in log2 units. The running max m is raised only when a
 // tile's max exceeds it by more than 8 (a factor of 256), so O in TMEM is rescaled rarely.
-// Probabilities stay below 2^8. A quarter of the exponentials run on the FMA pipe
-// (exp2_poly) and the rest on the MUFU unit, which would otherwise pace the loop.
+// Probabilities stay below 2^8. Half of the exponentials run on the FMA pipe (exp2_poly)
+// and half on the MUFU unit.
 #include <algorithm>
 
 #include "arl2_device.cuh"
@@ -46,56 +53,59 @@
 namespace arl2 {
 namespace {
 
-constexpr uint32_t kQOff = 0;
-constexpr uint32_t kKOff = kTileBytes;          // two stages
-constexpr uint32_t kVOff = 3 * kTileBytes;      // two stages
-constexpr uint32_t kWOff = 5 * kTileBytes;
-constexpr uint32_t kSOff = 6 * kTileBytes;
-constexpr uint32_t kBarOff = 7 * kTileBytes;
+constexpr int kStages = 3;
+constexpr int kThreads = 384;
+constexpr int kSoftmaxThreads = 256;
 enum : int {
-  kBarQFull = 0,     // Q (+ Wq, S) of a segment landed
-  kBarQEmpty = 1,    // the segment's QK^T MMAs are done with Q
-  kBarWSEmpty = 2,   // the readout MMAs are done with Wq, S
-  kBarKFull = 3,     // +stage
-  kBarVFull = 5,
-  kBarKEmpty = 7,
-  kBarVEmpty = 9,
-  kBarSFull = 11,    // +S buffer
-  kBarPFull = 13,    // +S buffer: P written over it (128 arrivals)
-  kBarPVDone = 15,   // +S buffer: the P.V MMA that read it is done
-  kBarQp = 17,       // Q' = Q Wq is in TMEM
-  kBarQpReady = 18,  // Q' bf16 is packed in TMEM (128 arrivals)
-  kBarOFull = 19,    // the segment's MMAs are all done
-  kBarOEmpty = 20,   // the segment's O / O_inter were read (128 arrivals)
-  kBarFinal = 21,
-  kBarGroup = 22,    // bounded rendezvous of the softmax warpgroup (128 arrivals)
-  kNumBars = 23
+  kBarQFull = 0,      // Q of a segment landed
+  kBarQEmpty = 1,     // the segment's MMAs are done with Q
+  kBarKFull = 2,      // +stage (3)
+  kBarKEmpty = 5,
+  kBarVFull = 8,
+  kBarVEmpty = 11,
+  kBarSFull = 14,     // +S buffer (2)
+  kBarPFull = 16,     // +S buffer: P written over it (256 arrivals)
+  kBarPVDone = 18,    // +S buffer: the P.V MMA that read it is done
+  kBarQp = 20,        // Q' = Q Wq is in TMEM
+  kBarQpReady = 21,   // Q' bf16 is packed in TMEM (256 arrivals)
+  kBarOFull = 22,     // the segment's MMAs are all done
+  kBarOEmpty = 23,    // the segment's O / O_inter were read (256 arrivals)
+  kBarFinal = 24,
+  kBarGroup = 25,     // bounded rendezvous of the softmax threads (256 arrivals)
+  kNumBars = 26
 };
-static_assert(kNumBars * 8 <= 256, "barriers must fit their shared-memory slot");
-constexpr int kMaxSegs = 8;        // the host plan keeps segments per query tile at or below this
+// Tiles at the (1 KiB-aligned) base of dynamic shared memory, then the control block.
+constexpr uint32_t kQOff = 0;
+constexpr uint32_t kKOff = kTileBytes;
+constexpr uint32_t kVOff = kKOff + kStages * kTileBytes;
+constexpr uint32_t kTileRegion = kVOff + kStages * kTileBytes;
+constexpr uint32_t kCtlBars = 0;
+constexpr uint32_t kCtlMisc = 256;           // tmem slot, abort flag, merge flag
+constexpr uint32_t kCtlX = 320;              // [2 buffers][2 halves][128] fp32 exchange slots
+constexpr uint32_t kCtlBytes = kCtlX + 2 * 2 * 128 * 4;
+static_assert(kNumBars * 8 <= kCtlMisc, "barriers must fit their slot");
+constexpr uint32_t kSmemBytes = kTileRegion + kCtlBytes;
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS0 = 0, kColO = 256, kColOI = 384;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kMaxSegs = 8;                // the host plan keeps segments per query tile at or below this
 
-// Rendezvous of the 128 softmax threads with a bounded wait (no hang if a warp aborted).
+struct Smem {
+  uint32_t ctl, tiles;
+  __device__ uint32_t bar(int i) const { return ctl + kCtlBars + 8u * i; }
+  __device__ uint32_t q() const { return tiles + kQOff; }
+  __device__ uint32_t k(int s) const { return tiles + kKOff + s * kTileBytes; }
+  __device__ uint32_t v(int s) const { return tiles + kVOff + s * kTileBytes; }
+};
+
+// Rendezvous of the 256 softmax threads with a bounded wait (no hang if a warp aborted).
 __device__ __forceinline__ bool group_sync(uint32_t bar, uint32_t& phase, const Guard& g) {
   mbar_arrive(bar);
   const bool ok = mbar_wait(bar, phase & 1, g);
   ++phase;
   return __all_sync(0xffffffffu, ok);
 }
-constexpr uint32_t kMiscOff = kBarOff + 256;
-constexpr uint32_t kSmemBytes = kMiscOff + 32 + 1024;  // + slack for 1 KiB alignment
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColO = 256, kColOI = 384;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
-
-struct Smem {
-  uint32_t base;
-  __device__ uint32_t bar(int i) const { return base + kBarOff + 8u * i; }
-  __device__ uint32_t q() const { return base + kQOff; }
-  __device__ uint32_t k(int s) const { return base + kKOff + s * kTileBytes; }
-  __device__ uint32_t v(int s) const { return base + kVOff + s * kTileBytes; }
-  __device__ uint32_t w() const { return base + kWOff; }
-  __device__ uint32_t s() const { return base + kSOff; }
-};
 
 // One segment of a CTA's unit range: key tiles [kb, ke) of query tile Q.
 struct Seg {
@@ -132,56 +142,59 @@ __device__ __forceinline__ int owner(long long u, const QueryArgs& a) {
   return static_cast<int>(((u + 1) * a.num_ctas - 1) / a.units);
 }
 
-template <bool kHybrid>
-__device__ void producer(const Smem& sm, const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
-                         const CUtensorMap* tm_w, const CUtensorMap* tm_s, const QueryArgs& a, const Guard& g) {
-  uint32_t nk[2] = {0, 0}, nv[2] = {0, 0};
-  uint32_t nseg = 0, nhead = 0, tile = 0;
+// Ring slot g: stage g % 3, used for the (g / 3)-th time.
+__device__ __forceinline__ int ring_stage(uint32_t g) { return static_cast<int>(g % kStages); }
+__device__ __forceinline__ uint32_t ring_phase(uint32_t g) { return (g / kStages) & 1; }
+
+// K producer (kIsK) or V producer. Per segment: [the readout operand (Wq or S) when the
+// segment starts a tile], then its key tiles, all through this producer's ring. The K
+// producer also loads each segment's Q tile.
+template <bool kHybrid, bool kIsK>
+__device__ void producer(const Smem& sm, const CUtensorMap* tm_q, const CUtensorMap* tm_kv, const CUtensorMap* tm_rd,
+                         const QueryArgs& a, const Guard& g) {
+  const int full0 = kIsK ? kBarKFull : kBarVFull, empty0 = kIsK ? kBarKEmpty : kBarVEmpty;
+  uint32_t nissued[kStages] = {0, 0, 0};
+  uint32_t nseg = 0, ring = 0;
   Sched sch(a, blockIdx.x);
   Seg sg;
   bool ok = true;
+  auto slot_wait = [&](uint32_t gidx) -> bool {
+    return gidx < kStages || mbar_wait(sm.bar(empty0 + ring_stage(gidx)), ring_phase(gidx - kStages), g);
+  };
+  auto tile_addr = [&](int s) { return kIsK ? sm.k(s) : sm.v(s); };
   while (ok && sch.next(sg)) {
-    const bool rd = kHybrid && sg.head;
-    if (nseg > 0 && !mbar_wait(sm.bar(kBarQEmpty), (nseg - 1) & 1, g)) break;
-    if (rd && nhead > 0 && !mbar_wait(sm.bar(kBarWSEmpty), (nhead - 1) & 1, g)) break;
-    mbar_expect_tx(sm.bar(kBarQFull), (rd ? 3 : 1) * kTileBytes);
-    for (int p = 0; p < 2; ++p)
-      tma_load_4d(sm.q() + p * kPanelBytes, tm_q, sm.bar(kBarQFull), 64 * p, sg.h, sg.qt * kRows, sg.b);
-    if (rd) {
-      const int slot = a.state_slot * a.B * a.H + sg.b * a.H + sg.h;
-      for (int p = 0; p < 2; ++p) {
-        tma_load_3d(sm.w() + p * kPanelBytes, tm_w, sm.bar(kBarQFull), 64 * p, 0, sg.h);
-        tma_load_3d(sm.s() + p * kPanelBytes, tm_s, sm.bar(kBarQFull), 64 * p, 0, slot);
-      }
-      ++nhead;
+    if (kIsK) {
+      if (nseg > 0 && !mbar_wait(sm.bar(kBarQEmpty), (nseg - 1) & 1, g)) break;
+      mbar_expect_tx(sm.bar(kBarQFull), kTileBytes);
+      for (int p = 0; p < 2; ++p)
+        tma_load_4d(sm.q() + p * kPanelBytes, tm_q, sm.bar(kBarQFull), 64 * p, sg.h, sg.qt * kRows, sg.b);
     }
     ++nseg;
-    for (int j = sg.kb; j < sg.ke; ++j, ++tile) {
-      const int s = tile & 1;
-      if (tile >= 2 && !mbar_wait(sm.bar(kBarKEmpty + s), ((tile - 2) >> 1) & 1, g)) {
+    if (kHybrid && sg.head) {
+      if (!slot_wait(ring)) break;
+      const int s = ring_stage(ring);
+      mbar_expect_tx(sm.bar(full0 + s), kTileBytes);
+      const int c2 = kIsK ? sg.h : a.state_slot * a.B * a.H + sg.b * a.H + sg.h;
+      for (int p = 0; p < 2; ++p) tma_load_3d(tile_addr(s) + p * kPanelBytes, tm_rd, sm.bar(full0 + s), 64 * p, 0, c2);
+      ++nissued[s];
+      ++ring;
+    }
+    for (int j = sg.kb; j < sg.ke; ++j, ++ring) {
+      if (!slot_wait(ring)) {
         ok = false;
         break;
       }
-      mbar_expect_tx(sm.bar(kBarKFull + s), kTileBytes);
+      const int s = ring_stage(ring);
+      mbar_expect_tx(sm.bar(full0 + s), kTileBytes);
       for (int p = 0; p < 2; ++p)
-        tma_load_4d(sm.k(s) + p * kPanelBytes, tm_k, sm.bar(kBarKFull + s), 64 * p, sg.h, j * kRows, sg.b);
-      ++nk[s];
-      if (tile >= 2 && !mbar_wait(sm.bar(kBarVEmpty + s), ((tile - 2) >> 1) & 1, g)) {
-        ok = false;
-        break;
-      }
-      mbar_expect_tx(sm.bar(kBarVFull + s), kTileBytes);
-      for (int p = 0; p < 2; ++p)
-        tma_load_4d(sm.v(s) + p * kPanelBytes, tm_v, sm.bar(kBarVFull + s), 64 * p, sg.h, j * kRows, sg.b);
-      ++nv[s];
+        tma_load_4d(tile_addr(s) + p * kPanelBytes, tm_kv, sm.bar(full0 + s), 64 * p, sg.h, j * kRows, sg.b);
+      ++nissued[s];
     }
   }
   // Every load issued must land before the CTA may exit (matters only after an abort).
-  if (nseg > 0) mbar_wait_drain(sm.bar(kBarQFull), (nseg - 1) & 1);
-  for (int s = 0; s < 2; ++s) {
-    if (nk[s]) mbar_wait_drain(sm.bar(kBarKFull + s), (nk[s] - 1) & 1);
-    if (nv[s]) mbar_wait_drain(sm.bar(kBarVFull + s), (nv[s] - 1) & 1);
-  }
+  if (kIsK && nseg > 0) mbar_wait_drain(sm.bar(kBarQFull), (nseg - 1) & 1);
+  for (int s = 0; s < kStages; ++s)
+    if (nissued[s]) mbar_wait_drain(sm.bar(full0 + s), (nissued[s] - 1) & 1);
 }
 
 template <bool kHybrid>
@@ -189,118 +202,275 @@ __device__ void mma_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, co
   constexpr uint32_t id_kk = idesc_bf16(128, 128, false, false);   // A, B K-major
   constexpr uint32_t id_kmn = idesc_bf16(128, 128, false, true);   // A K-major (smem or TMEM), B MN-major
   const uint32_t tO = tmem + kColO, tOI = tmem + kColOI;
-  uint32_t nseg = 0, nhead = 0, tile = 0;
+  uint32_t nseg = 0, nhead = 0, tile = 0, ring = 0;
   Sched sch(a, blockIdx.x);
   Seg sg;
-  auto issue_qk = [&](uint32_t t) -> bool {
-    const int st = t & 1;
-    if (!mbar_wait(sm.bar(kBarKFull + st), (t >> 1) & 1, g)) return false;
+  // Score tile t (S buffer t & 1) from the K tile in ring slot r.
+  auto issue_qk = [&](uint32_t t, uint32_t r) -> bool {
+    const int st = t & 1, ks = ring_stage(r);
+    if (!mbar_wait(sm.bar(kBarKFull + ks), ring_phase(r), g)) return false;
     tc_fence_after();
     const uint32_t tS = tmem + kColS0 + 128u * st;
 #pragma unroll
-    for (int s = 0; s < 8; ++s) mma_bf16(tS, desc_kmajor(sm.q(), s), desc_kmajor(sm.k(st), s), id_kk, s > 0);
-    mma_commit(sm.bar(kBarKEmpty + st));
+    for (int s = 0; s < 8; ++s) mma_bf16(tS, desc_kmajor(sm.q(), s), desc_kmajor(sm.k(ks), s), id_kk, s > 0);
+    mma_commit(sm.bar(kBarKEmpty + ks));
     mma_commit(sm.bar(kBarSFull + st));
     return true;
   };
   while (sch.next(sg)) {
     const bool rd = kHybrid && sg.head;
     const uint32_t t0 = tile, n = sg.ke - sg.kb;
+    const uint32_t r_rd = ring, r0 = ring + (rd ? 1 : 0);   // readout operands' slot, first key tile's slot
     if (!mbar_wait(sm.bar(kBarQFull), nseg & 1, g)) return;
     tc_fence_after();
     // The first two score tiles only need free S buffers; they overlap the previous
     // segment's epilogue.
-    if (!issue_qk(t0)) return;
-    if (n > 1 && !issue_qk(t0 + 1)) return;
+    if (!issue_qk(t0, r0)) return;
+    if (n > 1 && !issue_qk(t0 + 1, r0 + 1)) return;
     // O and O_inter of the previous segment must have been read before they are rewritten.
     if (nseg > 0 && !mbar_wait(sm.bar(kBarOEmpty), (nseg - 1) & 1, g)) return;
     tc_fence_after();
     if (rd) {
-      // Q' = Q Wq_h (phi_q) into the O_inter columns.
+      // Q' = Q Wq_h (phi_q) into the O_inter columns; Wq_h sits in K slot r_rd.
+      const int ws = ring_stage(r_rd);
+      if (!mbar_wait(sm.bar(kBarKFull + ws), ring_phase(r_rd), g)) return;
+      tc_fence_after();
 #pragma unroll
-      for (int s = 0; s < 8; ++s) mma_bf16(tOI, desc_kmajor(sm.q(), s), desc_mnmajor(sm.w(), s), id_kmn, s > 0);
+      for (int s = 0; s < 8; ++s) mma_bf16(tOI, desc_kmajor(sm.q(), s), desc_mnmajor(sm.k(ws), s), id_kmn, s > 0);
+      mma_commit(sm.bar(kBarKEmpty + ws));
       mma_commit(sm.bar(kBarQp));
     }
     if (n <= 2) mma_commit(sm.bar(kBarQEmpty));
     if (rd) {
-      // O_inter = Q' S_{N-1}, with Q' packed to bf16 in the O columns.
+      // O_inter = Q' S_{N-1}: Q' packed to bf16 in the O columns, S_h in V slot r_rd.
+      const int ss = ring_stage(r_rd);
       if (!mbar_wait(sm.bar(kBarQpReady), nhead & 1, g)) return;
+      if (!mbar_wait(sm.bar(kBarVFull + ss), ring_phase(r_rd), g)) return;
       tc_fence_after();
 #pragma unroll
-      for (int s = 0; s < 8; ++s) mma_bf16_ts(tOI, tO + 8u * s, desc_mnmajor(sm.s(), s), id_kmn, s > 0);
-      mma_commit(sm.bar(kBarWSEmpty));
+      for (int s = 0; s < 8; ++s) mma_bf16_ts(tOI, tO + 8u * s, desc_mnmajor(sm.v(ss), s), id_kmn, s > 0);
+      mma_commit(sm.bar(kBarVEmpty + ss));
       ++nhead;
     }
     for (uint32_t i = 0; i < n; ++i) {
-      const uint32_t t = t0 + i;
-      const int st = t & 1;
-      const uint32_t ph = (t >> 1) & 1;
-      if (!mbar_wait(sm.bar(kBarPFull + st), ph, g)) return;
-      if (!mbar_wait(sm.bar(kBarVFull + st), ph, g)) return;
+      const uint32_t t = t0 + i, r = r0 + i;
+      const int st = t & 1, vs = ring_stage(r);
+      if (!mbar_wait(sm.bar(kBarPFull + st), (t >> 1) & 1, g)) return;
+      if (!mbar_wait(sm.bar(kBarVFull + vs), ring_phase(r), g)) return;
       tc_fence_after();
       const uint32_t tP = tmem + kColS0 + 128u * st;
 #pragma unroll
       for (int s = 0; s < 8; ++s)
-        mma_bf16_ts(tO, tP + 8u * s, desc_mnmajor(sm.v(st), s), id_kmn, (i > 0 || s > 0) ? 1u : 0u);
+        mma_bf16_ts(tO, tP + (s < 4 ? 8u * s : 64u + 8u * (s - 4)), desc_mnmajor(sm.v(vs), s), id_kmn,
+                    (i > 0 || s > 0) ? 1u : 0u);
       mma_commit(sm.bar(kBarPVDone + st));
-      mma_commit(sm.bar(kBarVEmpty + st));
+      mma_commit(sm.bar(kBarVEmpty + vs));
       if (i + 2 < n) {
-        if (!issue_qk(t + 2)) return;
+        if (!issue_qk(t + 2, r + 2)) return;
         if (i + 3 == n) mma_commit(sm.bar(kBarQEmpty));
       }
     }
     mma_commit(sm.bar(kBarOFull));
     tile += n;
+    ring = r0 + n;
     ++nseg;
   }
 }
 
-// Softmax of one 128-key tile for this thread's row: scores sv (raw fp32) -> P (bf16) in
-// TMEM over the same columns. Returns the row sum of P; m is the log2-unit max in use.
-__device__ __forceinline__ float tile_probs(uint32_t (&sv)[4][32], float m, float scale_log2, uint32_t tP) {
+// Row max (log2 units) of a 64-column score half, with keys at or beyond `valid` masked.
+__device__ __forceinline__ float half_max(uint32_t (&sv)[2][32], int col0, int valid) {
+  if (valid < col0 + 64) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        if (col0 + 32 * c + e >= valid) sv[c][e] = __float_as_uint(-INFINITY);
+  }
+  float mx[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < 2; ++c)
+#pragma unroll
+    for (int e = 0; e < 32; ++e) mx[e & 7] = fmaxf(mx[e & 7], __uint_as_float(sv[c][e]));
+  return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+}
+
+// P for this thread's 64 score columns (raw fp32 in sv) -> 32 packed bf16 pairs in TMEM at
+// tP. Returns their sum; m is the log2-unit max in use.
+__device__ __forceinline__ float half_probs(const uint32_t (&sv)[2][32], float m, float scale_log2, uint32_t tP) {
   const float neg_m = -m;
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  // Two halves of 64 score columns; each becomes 32 packed bf16 pairs stored to TMEM at
-  // once, so only one half's packed words are live.
+  uint32_t pk[32];
 #pragma unroll
-  for (int hlf = 0; hlf < 2; ++hlf) {
-    uint32_t pk[32];   // pk[w]: score columns 64*hlf + 2w, 64*hlf + 2w + 1
+  for (int c = 0; c < 2; ++c) {
 #pragma unroll
-    for (int cc = 0; cc < 2; ++cc) {
-      const int c = 2 * hlf + cc;
+    for (int i = 0; i < 32; i += 2) {
+      float p2[2];
 #pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        float p2[2];
+      for (int e = 0; e < 2; ++e) {
+        const int col = i + e;
+        const float x = fmaf(__uint_as_float(sv[c][col]), scale_log2, neg_m);
+        // Odd columns on the FMA pipe, even columns on MUFU.
+        p2[e] = (col & 1) ? exp2_poly(x) : ex2_approx(x);
+        acc[col & 7] += p2[e];
+      }
+      pk[16 * c + (i >> 1)] = pack_bf16x2(p2[0], p2[1]);
+    }
+  }
+  tmem_st32(tP, pk);
+  return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+}
+
+// End of a segment: write O (whole query tile), or this segment's partial record and,
+// for the CTA completing the tile, the merge of all its records. Kept out of line so its
+// registers do not compete with the softmax loop. Returns false if a wait gave up.
+template <bool kHybrid>
+__device__ __noinline__ bool segment_epilogue(const Smem& sm, const QueryArgs& a, const Seg& sg, uint32_t r, int half,
+                                              int c0, int ncols, uint32_t tO, uint32_t tOI, float m, float l_row,
+                                              uint32_t& gphase, volatile int* merge_flag, const Guard& g) {
+  const int d = a.d;
+  const int t_row = sg.qt * kRows + static_cast<int>(r);
+  const bool row_ok = t_row < a.T;
+  uint16_t* out_row = a.o + ((static_cast<size_t>(sg.b) * a.T + t_row) * a.H + sg.h) * d;
+  if (sg.head && sg.tail) {
+    const float inv_l = 1.f / l_row;
+    for (int c = 0; 16 * c < ncols; ++c) {
+      uint32_t ov[16], iv[16];
+      tmem_ld16(tO + c0 + 16u * c, ov);
+      if (kHybrid) tmem_ld16(tOI + c0 + 16u * c, iv);
+      tmem_wait_ld();
+      reg_fence16(ov);
+      if (kHybrid) reg_fence16(iv);
+      if (row_ok) {
+        uint4* dst = reinterpret_cast<uint4*>(out_row + c0 + 16 * c);
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int col = i + e;
-          const float x = fmaf(__uint_as_float(sv[c][col]), scale_log2, neg_m);
-          // Every fourth column on the FMA pipe, the rest on MUFU.
-          p2[e] = ((col & 3) == 3) ? exp2_poly(x) : ex2_approx(x);
-          acc[col & 7] += p2[e];
+        for (int q = 0; q < 2; ++q) {
+          float y[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            y[e] = __uint_as_float(ov[8 * q + e]) * inv_l;
+            if (kHybrid) y[e] += __uint_as_float(iv[8 * q + e]);
+          }
+          dst[q] = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                              pack_bf16x2(y[6], y[7]));
         }
-        pk[16 * cc + (i >> 1)] = pack_bf16x2(p2[0], p2[1]);
       }
     }
-    tmem_st32(tP + 32u * hlf, pk);
-  }
-  float s = 0.f;
+    tc_fence_before();
+    mbar_arrive(sm.bar(kBarOEmpty));
+  } else {
+    // Partial record of this segment: O_acc, m, l (and O_inter if it holds key tile 0).
+    const long long first = static_cast<long long>(sg.Q) * a.nkv;
+    const int c_first = owner(first, a);
+    const int nsegs = owner(first + a.nkv - 1, a) - c_first + 1;
+    const int slot = sg.Q * a.max_segs + (static_cast<int>(blockIdx.x) - c_first);
+    float* po = a.part_o + (static_cast<size_t>(slot) * kRows + r) * kDP + c0;
+    float* poi = a.part_oi + (static_cast<size_t>(sg.Q) * kRows + r) * kDP + c0;
+    for (int c = 0; 16 * c < ncols; ++c) {
+      uint32_t ov[16], iv[16];
+      tmem_ld16(tO + c0 + 16u * c, ov);
+      if (kHybrid && sg.head) tmem_ld16(tOI + c0 + 16u * c, iv);
+      tmem_wait_ld();
+      reg_fence16(ov);
+      if (kHybrid && sg.head) reg_fence16(iv);
+      float4* d4 = reinterpret_cast<float4*>(po + 16 * c);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) s += acc[i];
-  return s;
+      for (int q = 0; q < 4; ++q)
+        d4[q] = make_float4(__uint_as_float(ov[4 * q]), __uint_as_float(ov[4 * q + 1]),
+                            __uint_as_float(ov[4 * q + 2]), __uint_as_float(ov[4 * q + 3]));
+      if (kHybrid && sg.head) {
+        float4* i4 = reinterpret_cast<float4*>(poi + 16 * c);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          i4[q] = make_float4(__uint_as_float(iv[4 * q]), __uint_as_float(iv[4 * q + 1]),
+                              __uint_as_float(iv[4 * q + 2]), __uint_as_float(iv[4 * q + 3]));
+      }
+    }
+    if (half == 0) {
+      a.part_ml[(static_cast<size_t>(slot) * 2) * kRows + r] = m;
+      a.part_ml[(static_cast<size_t>(slot) * 2 + 1) * kRows + r] = l_row;
+    }
+    // TMEM is read: the next segment's MMAs may reuse O and O_inter.
+    tc_fence_before();
+    mbar_arrive(sm.bar(kBarOEmpty));
+    // Publish, then count this segment in; the CTA completing the count merges.
+    __threadfence();
+    if (!group_sync(sm.bar(kBarGroup), gphase, g)) return false;
+    if (half == 0 && r == 0) {
+      const int prev = atomicAdd(a.cnt + sg.Q, 1);
+      *merge_flag = (prev == nsegs - 1) ? 1 : 0;
+    }
+    if (!group_sync(sm.bar(kBarGroup), gphase, g)) return false;
+    if (*merge_flag) {
+      __threadfence();
+      float M = -INFINITY;
+      for (int s = 0; s < nsegs; ++s)
+        M = fmaxf(M, __ldcg(a.part_ml + (static_cast<size_t>(sg.Q * a.max_segs + s) * 2) * kRows + r));
+      float L = 0.f, wgt[kMaxSegs];
+      for (int s = 0; s < nsegs && s < kMaxSegs; ++s) {
+        const size_t sl = static_cast<size_t>(sg.Q * a.max_segs + s);
+        wgt[s] = ex2_approx(__ldcg(a.part_ml + (sl * 2) * kRows + r) - M);
+        L += wgt[s] * __ldcg(a.part_ml + (sl * 2 + 1) * kRows + r);
+      }
+      const float inv_L = 1.f / L;
+      for (int c = 0; 8 * c < ncols; ++c) {
+        float y[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) y[e] = 0.f;
+        for (int s = 0; s < nsegs && s < kMaxSegs; ++s) {
+          const float4* src = reinterpret_cast<const float4*>(
+              a.part_o + (static_cast<size_t>(sg.Q * a.max_segs + s) * kRows + r) * kDP + c0 + 8 * c);
+          const float4 u0 = __ldcg(src), u1 = __ldcg(src + 1);
+          y[0] += wgt[s] * u0.x;
+          y[1] += wgt[s] * u0.y;
+          y[2] += wgt[s] * u0.z;
+          y[3] += wgt[s] * u0.w;
+          y[4] += wgt[s] * u1.x;
+          y[5] += wgt[s] * u1.y;
+          y[6] += wgt[s] * u1.z;
+          y[7] += wgt[s] * u1.w;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) y[e] *= inv_L;
+        if (kHybrid) {
+          const float4* src = reinterpret_cast<const float4*>(poi + 8 * c);
+          const float4 u0 = __ldcg(src), u1 = __ldcg(src + 1);
+          y[0] += u0.x;
+          y[1] += u0.y;
+          y[2] += u0.z;
+          y[3] += u0.w;
+          y[4] += u1.x;
+          y[5] += u1.y;
+          y[6] += u1.z;
+          y[7] += u1.w;
+        }
+        if (row_ok)
+          *reinterpret_cast<uint4*>(out_row + c0 + 8 * c) = make_uint4(
+              pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
+      }
+      if (half == 0 && r == 0) a.cnt[sg.Q] = 0;   // ready for the next launch
+    }
+  }
+  return true;
 }
 
 template <bool kHybrid>
-__device__ void softmax_role(const Smem& sm, uint32_t tmem, const QueryArgs& a, int warp, int lane,
-                             volatile int* bcast, const Guard& g) {
+__device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const QueryArgs& a, int warp, int lane,
+                             const Guard& g) {
   const int quarter = warp & 3;
-  const uint32_t r = quarter * 32 + lane;                  // tile row == TMEM lane
+  const int half = (warp - 4) >> 2;                         // 0: columns 0-63, 1: columns 64-127
+  const uint32_t r = quarter * 32 + lane;                   // tile row == TMEM lane
   const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
   const uint32_t tO = tmem + lane_off + kColO;
   const uint32_t tOI = tmem + lane_off + kColOI;
+  float* xch = reinterpret_cast<float*>(ctl + kCtlX);            // [2 buffers][2 halves][128]
+  volatile int* merge_flag = reinterpret_cast<volatile int*>(ctl + kCtlMisc + 8);
   const int d = a.d;
+  const int c0 = 64 * half;                                 // first column of this thread's half
+  const int ncols = max(0, min(64, d - c0));                // output columns of this half
   uint32_t nseg = 0, nhead = 0, tile = 0, gphase = 0;
   Sched sch(a, blockIdx.x);
   Seg sg;
@@ -312,14 +482,14 @@ __device__ void softmax_role(const Smem& sm, uint32_t tmem, const QueryArgs& a, 
       if (!mbar_wait_warp(sm.bar(kBarQp), nhead & 1, g)) return;
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t x[32], pk[16];
-        tmem_ld32(tOI + 32u * c, x);
+        tmem_ld32(tOI + c0 + 32u * c, x);
         tmem_wait_ld();
         reg_fence(x);
 #pragma unroll
         for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(x[2 * i]), __uint_as_float(x[2 * i + 1]));
-        tmem_st16(tO + 16u * c, pk);
+        tmem_st16(tO + c0 / 2 + 16u * c, pk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -333,32 +503,21 @@ __device__ void softmax_role(const Smem& sm, uint32_t tmem, const QueryArgs& a, 
       const int st = t & 1;
       if (!mbar_wait_warp(sm.bar(kBarSFull + st), (t >> 1) & 1, g)) return;
       tc_fence_after();
-      uint32_t sv[4][32];
       const uint32_t tS = tmem + lane_off + kColS0 + 128u * st;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32u * c, sv[c]);
-      tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < 4; ++c) reg_fence(sv[c]);
-
-      // Tile max of the raw scores (eight independent chains); keys >= kv_len are masked.
       const int valid = a.kv_len - (sg.kb + static_cast<int>(i)) * kRows;   // >= 1
-      if (valid < kRows) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (32 * c + e >= valid) sv[c][e] = __float_as_uint(-INFINITY);
-      }
-      float mx[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int e = 0; e < 32; ++e) mx[e & 7] = fmaxf(mx[e & 7], __uint_as_float(sv[c][e]));
-      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * a.scale_log2;
+      // This half's 64 scores; the row max is combined with the other half's through
+      // shared memory (each half reads and overwrites only its own columns).
+      uint32_t sv[2][32];
+      tmem_ld32(tS + c0, sv[0]);
+      tmem_ld32(tS + c0 + 32, sv[1]);
+      tmem_wait_ld();
+      reg_fence(sv[0]);
+      reg_fence(sv[1]);
+      const float mh = half_max(sv, c0, valid);
+      float* xb = xch + (t & 1) * 256;
+      xb[half * 128 + r] = mh;
+      if (!group_sync(sm.bar(kBarGroup), gphase, g)) return;
+      const float mt = fmaxf(mh, xb[(half ^ 1) * 128 + r]) * a.scale_log2;
       float m_new = m;
       bool rescale = false;
       if (i == 0) {
@@ -368,203 +527,95 @@ __device__ void softmax_role(const Smem& sm, uint32_t tmem, const QueryArgs& a, 
         rescale = true;
       }
       if (__any_sync(0xffffffffu, rescale)) {
-        // O holds the sum up to tile t-1: wait for that P.V MMA, then scale this row of O.
+        // O holds the sum up to tile t-1: wait for that P.V MMA, then scale this half-row.
         if (!mbar_wait_warp(sm.bar(kBarPVDone + ((t - 1) & 1)), ((t - 1) >> 1) & 1, g)) return;
         tc_fence_after();
         const float corr = rescale ? ex2_approx(m - m_new) : 1.f;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t ov[32];
-          tmem_ld32(tO + 32u * c, ov);
+          tmem_ld32(tO + c0 + 32u * c, ov);
           tmem_wait_ld();
           reg_fence(ov);
 #pragma unroll
           for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
-          tmem_st32(tO + 32u * c, ov);
+          tmem_st32(tO + c0 + 32u * c, ov);
         }
         l *= corr;
       }
       m = m_new;
-      l += tile_probs(sv, m, a.scale_log2, tS);
+      l += half_probs(sv, m, a.scale_log2, tS + c0);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(sm.bar(kBarPFull + st));
     }
     tile += n;
 
-    // ---- end of segment: every MMA of it is done.
+    // ---- end of segment: every MMA of it is done; combine the two half-row sums.
     if (!mbar_wait_warp(sm.bar(kBarOFull), nseg & 1, g)) return;
     tc_fence_after();
-    const int t_row = sg.qt * kRows + static_cast<int>(r);
-    const bool row_ok = t_row < a.T;
-    uint16_t* out_row = a.o + ((static_cast<size_t>(sg.b) * a.T + t_row) * a.H + sg.h) * d;
-    if (sg.head && sg.tail) {
-      const float inv_l = 1.f / l;
-      for (int c = 0; 16 * c < d; ++c) {
-        uint32_t ov[16], iv[16];
-        tmem_ld16(tO + 16u * c, ov);
-        if (kHybrid) tmem_ld16(tOI + 16u * c, iv);
-        tmem_wait_ld();
-        reg_fence16(ov);
-        if (kHybrid) reg_fence16(iv);
-        if (row_ok) {
-          uint4* dst = reinterpret_cast<uint4*>(out_row + 16 * c);
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            float y[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              y[e] = __uint_as_float(ov[8 * q + e]) * inv_l;
-              if (kHybrid) y[e] += __uint_as_float(iv[8 * q + e]);
-            }
-            dst[q] = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
-                                pack_bf16x2(y[6], y[7]));
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(sm.bar(kBarOEmpty));
-    } else {
-      // Partial record of this segment: O_acc, m, l (and O_inter if it holds key tile 0).
-      const long long first = static_cast<long long>(sg.Q) * a.nkv;
-      const int c_first = owner(first, a);
-      const int nsegs = owner(first + a.nkv - 1, a) - c_first + 1;
-      const int slot = sg.Q * a.max_segs + (static_cast<int>(blockIdx.x) - c_first);
-      float* po = a.part_o + (static_cast<size_t>(slot) * kRows + r) * kDP;
-      float* poi = a.part_oi + (static_cast<size_t>(sg.Q) * kRows + r) * kDP;
-      for (int c = 0; 16 * c < d; ++c) {
-        uint32_t ov[16], iv[16];
-        tmem_ld16(tO + 16u * c, ov);
-        if (kHybrid && sg.head) tmem_ld16(tOI + 16u * c, iv);
-        tmem_wait_ld();
-        reg_fence16(ov);
-        if (kHybrid && sg.head) reg_fence16(iv);
-        float4* d4 = reinterpret_cast<float4*>(po + 16 * c);
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          d4[q] = make_float4(__uint_as_float(ov[4 * q]), __uint_as_float(ov[4 * q + 1]),
-                              __uint_as_float(ov[4 * q + 2]), __uint_as_float(ov[4 * q + 3]));
-        if (kHybrid && sg.head) {
-          float4* i4 = reinterpret_cast<float4*>(poi + 16 * c);
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            i4[q] = make_float4(__uint_as_float(iv[4 * q]), __uint_as_float(iv[4 * q + 1]),
-                                __uint_as_float(iv[4 * q + 2]), __uint_as_float(iv[4 * q + 3]));
-        }
-      }
-      a.part_ml[(static_cast<size_t>(slot) * 2) * kRows + r] = m;
-      a.part_ml[(static_cast<size_t>(slot) * 2 + 1) * kRows + r] = l;
-      // TMEM is read: the next segment's MMAs may reuse O and O_inter.
-      tc_fence_before();
-      mbar_arrive(sm.bar(kBarOEmpty));
-      // Publish, then count this segment in; the CTA completing the count merges.
-      __threadfence();
-      if (!group_sync(sm.bar(kBarGroup), gphase, g)) return;
-      if (r == 0) {
-        const int prev = atomicAdd(a.cnt + sg.Q, 1);
-        *bcast = (prev == nsegs - 1) ? 1 : 0;
-      }
-      if (!group_sync(sm.bar(kBarGroup), gphase, g)) return;
-      if (*bcast) {
-        __threadfence();
-        float M = -INFINITY;
-        for (int s = 0; s < nsegs; ++s)
-          M = fmaxf(M, __ldcg(a.part_ml + (static_cast<size_t>(sg.Q * a.max_segs + s) * 2) * kRows + r));
-        float L = 0.f, wgt[kMaxSegs];
-        for (int s = 0; s < nsegs && s < kMaxSegs; ++s) {
-          const size_t sl = static_cast<size_t>(sg.Q * a.max_segs + s);
-          wgt[s] = ex2_approx(__ldcg(a.part_ml + (sl * 2) * kRows + r) - M);
-          L += wgt[s] * __ldcg(a.part_ml + (sl * 2 + 1) * kRows + r);
-        }
-        const float inv_L = 1.f / L;
-        for (int c = 0; 8 * c < d; ++c) {
-          float y[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) y[e] = 0.f;
-          for (int s = 0; s < nsegs && s < kMaxSegs; ++s) {
-            const float4* src = reinterpret_cast<const float4*>(
-                a.part_o + (static_cast<size_t>(sg.Q * a.max_segs + s) * kRows + r) * kDP + 8 * c);
-            const float4 u0 = __ldcg(src), u1 = __ldcg(src + 1);
-            y[0] += wgt[s] * u0.x;
-            y[1] += wgt[s] * u0.y;
-            y[2] += wgt[s] * u0.z;
-            y[3] += wgt[s] * u0.w;
-            y[4] += wgt[s] * u1.x;
-            y[5] += wgt[s] * u1.y;
-            y[6] += wgt[s] * u1.z;
-            y[7] += wgt[s] * u1.w;
-          }
-#pragma unroll
-          for (int e = 0; e < 8; ++e) y[e] *= inv_L;
-          if (kHybrid) {
-            const float4* src = reinterpret_cast<const float4*>(poi + 8 * c);
-            const float4 u0 = __ldcg(src), u1 = __ldcg(src + 1);
-            y[0] += u0.x;
-            y[1] += u0.y;
-            y[2] += u0.z;
-            y[3] += u0.w;
-            y[4] += u1.x;
-            y[5] += u1.y;
-            y[6] += u1.z;
-            y[7] += u1.w;
-          }
-          if (row_ok)
-            *reinterpret_cast<uint4*>(out_row + 8 * c) = make_uint4(
-                pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
-        }
-        if (r == 0) a.cnt[sg.Q] = 0;   // ready for the next launch
-      }
-    }
+    // The exchange buffer of the next tile's parity is idle: no thread writes it again
+    // before the extra rendezvous below.
+    float* xs = xch + (tile & 1) * 256;
+    xs[half * 128 + r] = l;
+    if (!group_sync(sm.bar(kBarGroup), gphase, g)) return;
+    const float l_row = xs[r] + xs[128 + r];
+    if (!group_sync(sm.bar(kBarGroup), gphase, g)) return;
+    if (!segment_epilogue<kHybrid>(sm, a, sg, r, half, c0, ncols, tO, tOI, m, l_row, gphase, merge_flag, g)) return;
     ++nseg;
   }
 }
 
 template <bool kHybrid>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     arl2_query_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
                       const __grid_constant__ CUtensorMap tm_s, const QueryArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  uint8_t* gbase = smem_raw + (base - raw);
-  const Smem sm{base};
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kMiscOff);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + kMiscOff + 4);
-  volatile int* bcast = reinterpret_cast<volatile int*>(gbase + kMiscOff + 8);
+  const uint32_t tiles = smem_u32(smem_raw);
+  if (tiles & 1023u) {   // the swizzled tiles need a 1 KiB-aligned base: report, do nothing
+    if (threadIdx.x == 0) atomicOr(a.err, kErrLayoutBit);
+    return;
+  }
+  const uint32_t ctl = tiles + kTileRegion;
+  uint8_t* ctl_ptr = smem_raw + kTileRegion;
+  const Smem sm{ctl, tiles};
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl_ptr + kCtlMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl_ptr + kCtlMisc + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Guard g{abort_flag, a.err, a.timeout_ns};
 
   if (threadIdx.x == 0) {
     mbar_init(sm.bar(kBarQFull), 1);
     mbar_init(sm.bar(kBarQEmpty), 1);
-    mbar_init(sm.bar(kBarWSEmpty), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(sm.bar(kBarKFull + s), 1);
-      mbar_init(sm.bar(kBarVFull + s), 1);
       mbar_init(sm.bar(kBarKEmpty + s), 1);
+      mbar_init(sm.bar(kBarVFull + s), 1);
       mbar_init(sm.bar(kBarVEmpty + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(sm.bar(kBarSFull + s), 1);
-      mbar_init(sm.bar(kBarPFull + s), 128);
+      mbar_init(sm.bar(kBarPFull + s), kSoftmaxThreads);
       mbar_init(sm.bar(kBarPVDone + s), 1);
     }
     mbar_init(sm.bar(kBarQp), 1);
-    mbar_init(sm.bar(kBarQpReady), 128);
+    mbar_init(sm.bar(kBarQpReady), kSoftmaxThreads);
     mbar_init(sm.bar(kBarOFull), 1);
-    mbar_init(sm.bar(kBarOEmpty), 128);
+    mbar_init(sm.bar(kBarOEmpty), kSoftmaxThreads);
     mbar_init(sm.bar(kBarFinal), 1);
-    mbar_init(sm.bar(kBarGroup), 128);
+    mbar_init(sm.bar(kBarGroup), kSoftmaxThreads);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
+    if (kHybrid) prefetch_tmap(&tm_w);
+  }
+  if (warp == 2 && lane == 0) {
     prefetch_tmap(&tm_v);
-    if (kHybrid) {
-      prefetch_tmap(&tm_w);
-      prefetch_tmap(&tm_s);
-    }
+    if (kHybrid) prefetch_tmap(&tm_s);
   }
   if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
   tc_fence_before();
@@ -573,15 +624,17 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) producer<kHybrid>(sm, &tm_q, &tm_k, &tm_v, &tm_w, &tm_s, a, g);
+    if (lane == 0) producer<kHybrid, true>(sm, &tm_q, &tm_k, &tm_w, a, g);
   } else if (warp == 1) {
     if (lane == 0) {
       mma_issuer<kHybrid>(sm, tmem, a, g);
       mma_commit(sm.bar(kBarFinal));   // arrives once every MMA issued above has finished
     }
     __syncwarp();
-  } else {
-    softmax_role<kHybrid>(sm, tmem, a, warp, lane, bcast, g);
+  } else if (warp == 2) {
+    if (lane == 0) producer<kHybrid, false>(sm, &tm_q, &tm_v, &tm_s, a, g);
+  } else if (warp >= 4) {
+    softmax_role<kHybrid>(sm, ctl_ptr, tmem, a, warp, lane, g);
   }
 
   tc_fence_before();
@@ -641,9 +694,9 @@ cudaError_t launch_query(bool hybrid, const CUtensorMap& tm_q, const CUtensorMap
                          const CUtensorMap& tm_w, const CUtensorMap& tm_s, const QueryArgs& a, cudaStream_t stream) {
   const dim3 grid(a.num_ctas);
   if (hybrid)
-    arl2_query_kernel<true><<<grid, 192, kSmemBytes, stream>>>(tm_q, tm_k, tm_v, tm_w, tm_s, a);
+    arl2_query_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_k, tm_v, tm_w, tm_s, a);
   else
-    arl2_query_kernel<false><<<grid, 192, kSmemBytes, stream>>>(tm_q, tm_k, tm_v, tm_w, tm_s, a);
+    arl2_query_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_k, tm_v, tm_w, tm_s, a);
   return cudaGetLastError();
 }
 
