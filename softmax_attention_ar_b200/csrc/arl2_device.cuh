@@ -206,6 +206,64 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int s) {
   return sdesc_sw128(tile + s * 2048, kPanelBytes, 1024);
 }
 
+// A whole 128-deep contraction (8 K-steps of 16) as one issue block: the single issuing
+// thread is the tensor pipe's only feeder, so every instruction it spends per MMA counts.
+// Descriptors advance by constant offsets (in 16-byte units) from their step-0 value.
+//   K-major operand: step s at (s / 4) panels + (s % 4) * 32 bytes.
+//   MN-major operand: step s at s * 2048 bytes.
+//   TMEM operand (packed bf16): step s at column kPackedCol[s].
+__host__ __device__ constexpr uint32_t kmajor_step16(int s) { return (s >> 2) * (kPanelBytes >> 4) + (s & 3) * 2; }
+__host__ __device__ constexpr uint32_t mnmajor_step16(int s) { return s * (2048 >> 4); }
+
+template <bool kAMN, bool kBMN>
+__device__ __forceinline__ void mma8_ss(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc, uint32_t acc) {
+  uint64_t a[8], b[8];
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    a[s] = a0 + (kAMN ? mnmajor_step16(s) : kmajor_step16(s));
+    b[s] = b0 + (kBMN ? mnmajor_step16(s) : kmajor_step16(s));
+  }
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %18, 0;\n\t"
+      "setp.ne.b32 q, 1, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %9, %17, p;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %10, %17, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %11, %17, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %12, %17, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %13, %17, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %6, %14, %17, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %15, %17, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %8, %16, %17, q;\n\t}" ::"r"(d_tmem),
+      "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(a[4]), "l"(a[5]), "l"(a[6]), "l"(a[7]), "l"(b[0]), "l"(b[1]),
+      "l"(b[2]), "l"(b[3]), "l"(b[4]), "l"(b[5]), "l"(b[6]), "l"(b[7]), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+// A from TMEM: 8 K-steps whose packed columns are a0 + col[s]; B MN-major from shared memory.
+__device__ __forceinline__ void mma8_ts(uint32_t d_tmem, uint32_t a0, const uint32_t (&col)[8], uint64_t b0,
+                                        uint32_t idesc, uint32_t acc) {
+  uint64_t b[8];
+#pragma unroll
+  for (int s = 0; s < 8; ++s) b[s] = b0 + mnmajor_step16(s);
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %18, 0;\n\t"
+      "setp.ne.b32 q, 1, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %9, %17, p;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %10, %17, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %11, %17, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %12, %17, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%5], %13, %17, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%6], %14, %17, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%7], %15, %17, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%8], %16, %17, q;\n\t}" ::"r"(d_tmem),
+      "r"(a0 + col[0]), "r"(a0 + col[1]), "r"(a0 + col[2]), "r"(a0 + col[3]), "r"(a0 + col[4]), "r"(a0 + col[5]),
+      "r"(a0 + col[6]), "r"(a0 + col[7]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "l"(b[4]), "l"(b[5]), "l"(b[6]),
+      "l"(b[7]), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
 // 32 lanes x 32 consecutive 32-bit columns: thread i of the warp gets TMEM lane
 // (warp's lane quarter base + i), columns [col, col + 32).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {

@@ -26,9 +26,9 @@ struct QueryArgs {
   long long units;        // B * H * nq * nkv (query tile, key tile) pairs
   int num_ctas;           // grid size
   int max_segs;           // CTAs sharing one query tile, at most
-  float* part_o;          // [qtiles * max_segs, 128, 128] partial O accumulators
+  float* part_o;          // [qtiles * max_segs][32 column quads][128 rows] float4: partial O accumulators
   float* part_ml;         // [qtiles * max_segs, 2, 128] running max (log2 units) and sum
-  float* part_oi;         // [qtiles, 128, 128] O_inter of split query tiles
+  float* part_oi;         // [qtiles][32 column quads][128 rows] float4: O_inter of each query tile
   int* cnt;               // [qtiles] arrival counters, zero between launches
 };
 

@@ -13,11 +13,14 @@
 // [c*U/P, (c+1)*U/P), so every SM gets the same number of tile pairs. A CTA's range falls
 // into segments, each a key range of one query tile:
 //   - A segment that covers a whole query tile writes O directly.
-//   - Otherwise the CTA writes a partial record (O_acc, running max m and sum l) to scratch
-//     and bumps the tile's counter. The segment holding key tile 0 also stores O_inter.
+//   - Otherwise the CTA writes a partial record (O_acc, running max m, sum l) to scratch
+//     and bumps the tile's counter.
 //   - The CTA that brings the counter to the segment count merges every record of that
 //     tile in key order and writes O. It then resets the counter. The merge order is
 //     fixed, so the result does not depend on which CTA merges it.
+//   - The segment holding key tile 0 computes the readout O_inter first and stores it
+//     (fp32) in the tile's scratch record; whoever finishes the tile adds it.
+// Scratch records are column-quad-major, so every scratch access of a warp is coalesced.
 //
 // Roles (384 threads, one CTA per SM):
 //   warp 0      K producer: per segment the Q tile, then K tiles into a three-stage ring.
@@ -27,24 +30,25 @@
 //               the bf16 state copy S_h goes first, through the ring.
 //   warps 4-11  two softmax warpgroups. Thread = query row = TMEM lane; warps 4-7 own
 //               score and output columns 0-63, warps 8-11 columns 64-127. A thread reads
-//               and overwrites only its own 64 columns; the two halves of a row swap
-//               their partial maxima through shared memory once per tile. These threads
-//               also pack Q' to bf16 for the readout MMA and write outputs and partial
-//               records.
+//               the whole score row for its max but writes P only over its own columns,
+//               after both halves have read the tile. These threads also pack Q' for the
+//               readout MMA and write outputs and partial records.
 // TMEM (512 columns):
-//   - cols 0 and 128: the two S tiles, double-buffered. P (bf16) overwrites its own S tile:
-//     scores 0-63 are packed into columns 0-31 and scores 64-127 into columns 64-95. The
-//     P.V MMA reads them straight from TMEM.
-//   - col 256: O. At the start of a segment that starts a tile, it briefly holds Q' packed
-//     to bf16 for the readout MMA.
-//   - col 384: Q' (fp32), then O_inter.
+//   - cols 0, 128, 256: three S tiles. The score MMA of tile t+2 is queued right behind
+//     the P.V MMA of tile t and writes the buffer last read two MMA groups earlier, so no
+//     MMA group overwrites TMEM columns that the group just ahead of it still reads (that
+//     stalls the tensor pipe). P (bf16) overwrites its own S tile, scores 0-63 packed into
+//     columns 0-31 and scores 64-127 into columns 64-95, and feeds the P.V MMA straight
+//     from TMEM.
+//   - col 384: O. At the start of a segment that starts a tile, it first holds Q' (fp32,
+//     then packed to bf16 for the readout MMA, whose result goes to a free S tile).
 // Shared memory: Q | K0 K1 K2 | V0 V1 V2 (32 KiB tiles) from its 1 KiB-aligned base, then a
-// small control block (mbarriers, flags, the max/sum exchange slots).
+// small control block (mbarriers, flags, the row-sum exchange).
 //
 // Online softmax: scores are kept in log2 units. The running max m is raised only when a
 // tile's max exceeds it by more than 8 (a factor of 256), so O in TMEM is rescaled rarely.
-// Probabilities stay below 2^8. Half of the exponentials run on the FMA pipe (exp2_poly)
-// and half on the MUFU unit.
+// Probabilities stay below 2^8. A quarter of the exponentials run on the FMA pipe
+// (exp2_poly) and the rest on the MUFU unit.
 #include <algorithm>
 
 #include "arl2_device.cuh"
@@ -53,7 +57,8 @@
 namespace arl2 {
 namespace {
 
-constexpr int kStages = 3;
+constexpr int kStages = 3;      // K and V ring depth
+constexpr int kSBufs = 3;       // score tiles in TMEM
 constexpr int kThreads = 384;
 constexpr int kSoftmaxThreads = 256;
 enum : int {
@@ -63,16 +68,19 @@ enum : int {
   kBarKEmpty = 5,
   kBarVFull = 8,
   kBarVEmpty = 11,
-  kBarSFull = 14,     // +S buffer (2)
-  kBarPFull = 16,     // +S buffer: P written over it (256 arrivals)
-  kBarPVDone = 18,    // +S buffer: the P.V MMA that read it is done
-  kBarQp = 20,        // Q' = Q Wq is in TMEM
-  kBarQpReady = 21,   // Q' bf16 is packed in TMEM (256 arrivals)
-  kBarOFull = 22,     // the segment's MMAs are all done
-  kBarOEmpty = 23,    // the segment's O / O_inter were read (256 arrivals)
-  kBarFinal = 24,
-  kBarGroup = 25,     // bounded rendezvous of the softmax threads (256 arrivals)
-  kNumBars = 26
+  kBarSFull = 14,     // +S buffer (3): scores of a tile are in TMEM
+  kBarSRead = 17,     // +S buffer: both halves have read them (256 arrivals)
+  kBarPFull = 20,     // +S buffer: P written over them (256 arrivals)
+  kBarPVDone = 23,    // +S buffer: the P.V MMA that read P is done
+  kBarQp = 26,        // Q' = Q Wq is in TMEM (O columns)
+  kBarQpReady = 27,   // Q' is packed to bf16 (256 arrivals)
+  kBarOIReady = 28,   // O_inter is in TMEM (a free S buffer)
+  kBarOIFree = 29,    // O_inter was read out (256 arrivals)
+  kBarOFull = 30,     // the segment's MMAs are all done
+  kBarOEmpty = 31,    // the segment's O was read (256 arrivals)
+  kBarFinal = 32,
+  kBarGroup = 33,     // bounded rendezvous of the softmax threads (256 arrivals)
+  kNumBars = 34
 };
 // Tiles at the (1 KiB-aligned) base of dynamic shared memory, then the control block.
 constexpr uint32_t kQOff = 0;
@@ -80,14 +88,14 @@ constexpr uint32_t kKOff = kTileBytes;
 constexpr uint32_t kVOff = kKOff + kStages * kTileBytes;
 constexpr uint32_t kTileRegion = kVOff + kStages * kTileBytes;
 constexpr uint32_t kCtlBars = 0;
-constexpr uint32_t kCtlMisc = 256;           // tmem slot, abort flag, merge flag
-constexpr uint32_t kCtlX = 320;              // [2 buffers][2 halves][128] fp32 exchange slots
-constexpr uint32_t kCtlBytes = kCtlX + 2 * 2 * 128 * 4;
+constexpr uint32_t kCtlMisc = 320;           // tmem slot, abort flag, merge flag
+constexpr uint32_t kCtlX = 384;              // [2 halves][128] fp32 row-sum exchange
+constexpr uint32_t kCtlBytes = kCtlX + 2 * 128 * 4;
 static_assert(kNumBars * 8 <= kCtlMisc, "barriers must fit their slot");
 constexpr uint32_t kSmemBytes = kTileRegion + kCtlBytes;
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColO = 256, kColOI = 384;
+constexpr uint32_t kColO = 384;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kMaxSegs = 8;                // the host plan keeps segments per query tile at or below this
 
@@ -142,9 +150,11 @@ __device__ __forceinline__ int owner(long long u, const QueryArgs& a) {
   return static_cast<int>(((u + 1) * a.num_ctas - 1) / a.units);
 }
 
-// Ring slot g: stage g % 3, used for the (g / 3)-th time.
+// Ring slot g: stage g % 3, used for the (g / 3)-th time. S buffers cycle the same way.
 __device__ __forceinline__ int ring_stage(uint32_t g) { return static_cast<int>(g % kStages); }
 __device__ __forceinline__ uint32_t ring_phase(uint32_t g) { return (g / kStages) & 1; }
+__device__ __forceinline__ int sbuf(uint32_t t) { return static_cast<int>(t % kSBufs); }
+__device__ __forceinline__ uint32_t sphase(uint32_t t) { return (t / kSBufs) & 1; }
 
 // K producer (kIsK) or V producer. Per segment: [the readout operand (Wq or S) when the
 // segment starts a tile], then its key tiles, all through this producer's ring. The K
@@ -197,77 +207,87 @@ __device__ void producer(const Smem& sm, const CUtensorMap* tm_q, const CUtensor
     if (nissued[s]) mbar_wait_drain(sm.bar(full0 + s), (nissued[s] - 1) & 1);
 }
 
+
+
 template <bool kHybrid>
 __device__ void mma_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, const Guard& g) {
   constexpr uint32_t id_kk = idesc_bf16(128, 128, false, false);   // A, B K-major
   constexpr uint32_t id_kmn = idesc_bf16(128, 128, false, true);   // A K-major (smem or TMEM), B MN-major
-  const uint32_t tO = tmem + kColO, tOI = tmem + kColOI;
+  const uint32_t tO = tmem + kColO;
+  const uint32_t kPacked[8] = {0, 8, 16, 24, 64, 72, 80, 88};   // see the TMEM layout above
   uint32_t nseg = 0, nhead = 0, tile = 0, ring = 0;
   Sched sch(a, blockIdx.x);
   Seg sg;
-  // Score tile t (S buffer t & 1) from the K tile in ring slot r.
+  // Score tile t (S buffer t % 3) from the K tile in ring slot r. The buffer's previous
+  // tile (t - 3) was consumed by a P.V MMA issued earlier, so in-order execution keeps it.
   auto issue_qk = [&](uint32_t t, uint32_t r) -> bool {
-    const int st = t & 1, ks = ring_stage(r);
+    const int sb = sbuf(t), ks = ring_stage(r);
     if (!mbar_wait(sm.bar(kBarKFull + ks), ring_phase(r), g)) return false;
     tc_fence_after();
-    const uint32_t tS = tmem + kColS0 + 128u * st;
-#pragma unroll
-    for (int s = 0; s < 8; ++s) mma_bf16(tS, desc_kmajor(sm.q(), s), desc_kmajor(sm.k(ks), s), id_kk, s > 0);
+    const uint32_t tS = tmem + 128u * sb;
+    mma8_ss<false, false>(tS, desc_kmajor(sm.q(), 0), desc_kmajor(sm.k(ks), 0), id_kk, 0u);
     mma_commit(sm.bar(kBarKEmpty + ks));
-    mma_commit(sm.bar(kBarSFull + st));
+    mma_commit(sm.bar(kBarSFull + sb));
     return true;
   };
   while (sch.next(sg)) {
     const bool rd = kHybrid && sg.head;
     const uint32_t t0 = tile, n = sg.ke - sg.kb;
     const uint32_t r_rd = ring, r0 = ring + (rd ? 1 : 0);   // readout operands' slot, first key tile's slot
+    // Score tiles issued before the P.V loop: two. Afterwards the scores of tile t + 2 are
+    // issued right behind the P.V MMA of tile t: they go to the buffer whose P was read by
+    // the P.V MMA before that one, so adjacent MMA groups never touch the same TMEM columns
+    // (an MMA that overwrites columns the MMA just ahead of it still reads stalls the pipe).
+    const uint32_t npre = min(n, 2u);
     if (!mbar_wait(sm.bar(kBarQFull), nseg & 1, g)) return;
     tc_fence_after();
-    // The first two score tiles only need free S buffers; they overlap the previous
-    // segment's epilogue.
-    if (!issue_qk(t0, r0)) return;
-    if (n > 1 && !issue_qk(t0 + 1, r0 + 1)) return;
-    // O and O_inter of the previous segment must have been read before they are rewritten.
+    for (uint32_t i = 0; i < npre; ++i)
+      if (!issue_qk(t0 + i, r0 + i)) return;
+    // O of the previous segment must have been read before it is rewritten.
     if (nseg > 0 && !mbar_wait(sm.bar(kBarOEmpty), (nseg - 1) & 1, g)) return;
     tc_fence_after();
     if (rd) {
-      // Q' = Q Wq_h (phi_q) into the O_inter columns; Wq_h sits in K slot r_rd.
+      // Q' = Q Wq_h (phi_q) into the O columns; Wq_h sits in K slot r_rd.
       const int ws = ring_stage(r_rd);
       if (!mbar_wait(sm.bar(kBarKFull + ws), ring_phase(r_rd), g)) return;
       tc_fence_after();
-#pragma unroll
-      for (int s = 0; s < 8; ++s) mma_bf16(tOI, desc_kmajor(sm.q(), s), desc_mnmajor(sm.k(ws), s), id_kmn, s > 0);
+      mma8_ss<false, true>(tO, desc_kmajor(sm.q(), 0), desc_mnmajor(sm.k(ws), 0), id_kmn, 0u);
       mma_commit(sm.bar(kBarKEmpty + ws));
       mma_commit(sm.bar(kBarQp));
     }
-    if (n <= 2) mma_commit(sm.bar(kBarQEmpty));
+    if (n <= npre) mma_commit(sm.bar(kBarQEmpty));
     if (rd) {
-      // O_inter = Q' S_{N-1}: Q' packed to bf16 in the O columns, S_h in V slot r_rd.
+      // O_inter = Q' S_{N-1}: Q' packed to bf16 in the O columns, S_h in V slot r_rd, the
+      // result in the S buffer of tile t0 + 2 (free until that tile's scores are issued).
       const int ss = ring_stage(r_rd);
       if (!mbar_wait(sm.bar(kBarQpReady), nhead & 1, g)) return;
       if (!mbar_wait(sm.bar(kBarVFull + ss), ring_phase(r_rd), g)) return;
       tc_fence_after();
-#pragma unroll
-      for (int s = 0; s < 8; ++s) mma_bf16_ts(tOI, tO + 8u * s, desc_mnmajor(sm.v(ss), s), id_kmn, s > 0);
+      const uint32_t tX = tmem + 128u * sbuf(t0 + 2);
+      mma8_ts(tX, tO, kPacked, desc_mnmajor(sm.v(ss), 0), id_kmn, 0u);
       mma_commit(sm.bar(kBarVEmpty + ss));
+      mma_commit(sm.bar(kBarOIReady));
+      // Whatever tile next scores into that buffer (this segment's or a later one's) must
+      // wait for the read-out. It costs nothing here: the first P.V of the segment needs
+      // the softmax threads, which read O_inter out first.
+      if (!mbar_wait(sm.bar(kBarOIFree), nhead & 1, g)) return;
+      tc_fence_after();
       ++nhead;
     }
+    const uint32_t nissued = npre;   // score tiles issued ahead of the P.V loop
     for (uint32_t i = 0; i < n; ++i) {
       const uint32_t t = t0 + i, r = r0 + i;
-      const int st = t & 1, vs = ring_stage(r);
-      if (!mbar_wait(sm.bar(kBarPFull + st), (t >> 1) & 1, g)) return;
+      const int sb = sbuf(t), vs = ring_stage(r);
+      if (!mbar_wait(sm.bar(kBarPFull + sb), sphase(t), g)) return;
       if (!mbar_wait(sm.bar(kBarVFull + vs), ring_phase(r), g)) return;
       tc_fence_after();
-      const uint32_t tP = tmem + kColS0 + 128u * st;
-#pragma unroll
-      for (int s = 0; s < 8; ++s)
-        mma_bf16_ts(tO, tP + (s < 4 ? 8u * s : 64u + 8u * (s - 4)), desc_mnmajor(sm.v(vs), s), id_kmn,
-                    (i > 0 || s > 0) ? 1u : 0u);
-      mma_commit(sm.bar(kBarPVDone + st));
+      const uint32_t tP = tmem + 128u * sb;
+      mma8_ts(tO, tP, kPacked, desc_mnmajor(sm.v(vs), 0), id_kmn, i > 0 ? 1u : 0u);
+      mma_commit(sm.bar(kBarPVDone + sb));
       mma_commit(sm.bar(kBarVEmpty + vs));
-      if (i + 2 < n) {
-        if (!issue_qk(t + 2, r + 2)) return;
-        if (i + 3 == n) mma_commit(sm.bar(kBarQEmpty));
+      if (i + nissued < n) {
+        if (!issue_qk(t + nissued, r + nissued)) return;
+        if (i + nissued + 1 == n) mma_commit(sm.bar(kBarQEmpty));
       }
     }
     mma_commit(sm.bar(kBarOFull));
@@ -277,7 +297,7 @@ __device__ void mma_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, co
   }
 }
 
-// Row max (log2 units) of a 64-column score half, with keys at or beyond `valid` masked.
+// Row max of 64 score columns (raw units), with keys at or beyond `valid` masked.
 __device__ __forceinline__ float half_max(uint32_t (&sv)[2][32], int col0, int valid) {
   if (valid < col0 + 64) {
 #pragma unroll
@@ -296,14 +316,14 @@ __device__ __forceinline__ float half_max(uint32_t (&sv)[2][32], int col0, int v
   return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
 }
 
-// P for this thread's 64 score columns (raw fp32 in sv) -> 32 packed bf16 pairs in TMEM at
-// tP. Returns their sum; m is the log2-unit max in use.
-__device__ __forceinline__ float half_probs(const uint32_t (&sv)[2][32], float m, float scale_log2, uint32_t tP) {
+// P for 64 score columns (raw fp32 in sv; masked ones are -inf) as 32 packed bf16 pairs
+// in pk. Returns their sum; m is the log2-unit max in use.
+__device__ __forceinline__ float half_probs(const uint32_t (&sv)[2][32], float m, float scale_log2,
+                                            uint32_t (&pk)[32]) {
   const float neg_m = -m;
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  uint32_t pk[32];
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
 #pragma unroll
@@ -313,147 +333,170 @@ __device__ __forceinline__ float half_probs(const uint32_t (&sv)[2][32], float m
       for (int e = 0; e < 2; ++e) {
         const int col = i + e;
         const float x = fmaf(__uint_as_float(sv[c][col]), scale_log2, neg_m);
-        // Odd columns on the FMA pipe, even columns on MUFU.
-        p2[e] = (col & 1) ? exp2_poly(x) : ex2_approx(x);
+        // Every fourth column on the FMA pipe, the rest on MUFU.
+        p2[e] = ((col & 3) == 3) ? exp2_poly(x) : ex2_approx(x);
         acc[col & 7] += p2[e];
       }
       pk[16 * c + (i >> 1)] = pack_bf16x2(p2[0], p2[1]);
     }
   }
-  tmem_st32(tP, pk);
   return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 }
 
+// Scratch records are stored column-quad-major: float4 (record, quad q of 4 columns, row r)
+// sits at ((record * 32 + q) * 128 + r), so a warp's 32 rows move 512 contiguous bytes.
+__device__ __forceinline__ float4* quad_ptr(float* base, size_t record, int q, uint32_t r) {
+  return reinterpret_cast<float4*>(base) + ((record * 32 + q) * kRows + r);
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&y)[8]) {
+  return make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                    pack_bf16x2(y[6], y[7]));
+}
+
 // End of a segment: write O (whole query tile), or this segment's partial record and,
-// for the CTA completing the tile, the merge of all its records. Kept out of line so its
-// registers do not compete with the softmax loop. Returns false if a wait gave up.
+// for the CTA completing the tile, the merge of all its records. O_inter (fp32 scratch,
+// written by the segment that started the tile) is added by whoever finishes the tile.
+// Loads are issued in batches of 16 quads so their latencies overlap. Kept out of line so
+// its registers do not compete with the softmax loop. Returns false if a wait gave up.
 template <bool kHybrid>
 __device__ __noinline__ bool segment_epilogue(const Smem& sm, const QueryArgs& a, const Seg& sg, uint32_t r, int half,
-                                              int c0, int ncols, uint32_t tO, uint32_t tOI, float m, float l_row,
+                                              int c0, int ncols, uint32_t tO, float m, float l_row,
                                               uint32_t& gphase, volatile int* merge_flag, const Guard& g) {
   const int d = a.d;
+  const int q0 = c0 / 4, nquads = ncols / 4;   // this half's column quads
   const int t_row = sg.qt * kRows + static_cast<int>(r);
   const bool row_ok = t_row < a.T;
-  uint16_t* out_row = a.o + ((static_cast<size_t>(sg.b) * a.T + t_row) * a.H + sg.h) * d;
+  uint16_t* out_row = a.o + ((static_cast<size_t>(sg.b) * a.T + t_row) * a.H + sg.h) * d + c0;
   if (sg.head && sg.tail) {
     const float inv_l = 1.f / l_row;
-    for (int c = 0; 16 * c < ncols; ++c) {
-      uint32_t ov[16], iv[16];
-      tmem_ld16(tO + c0 + 16u * c, ov);
-      if (kHybrid) tmem_ld16(tOI + c0 + 16u * c, iv);
-      tmem_wait_ld();
-      reg_fence16(ov);
-      if (kHybrid) reg_fence16(iv);
-      if (row_ok) {
-        uint4* dst = reinterpret_cast<uint4*>(out_row + c0 + 16 * c);
+    // Two passes of 8 column quads (32 columns): O_inter loads first, then O from TMEM.
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          float y[8];
+    for (int hp = 0; hp < 2; ++hp) {
+      if (32 * hp >= ncols) break;
+      float4 oi[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            y[e] = __uint_as_float(ov[8 * q + e]) * inv_l;
-            if (kHybrid) y[e] += __uint_as_float(iv[8 * q + e]);
+      for (int q = 0; q < 8; ++q) {
+        oi[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (kHybrid && 8 * hp + q < nquads) oi[q] = __ldcg(quad_ptr(a.part_oi, sg.Q, q0 + 8 * hp + q, r));
+      }
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = 2 * hp + cc;
+        if (16 * c >= ncols) break;
+        uint32_t ov[16];
+        tmem_ld16(tO + c0 + 16u * c, ov);
+        tmem_wait_ld();
+        reg_fence16(ov);
+        if (row_ok) {
+#pragma unroll
+          for (int h8 = 0; h8 < 2; ++h8) {
+            const float4 i0 = oi[4 * cc + 2 * h8], i1 = oi[4 * cc + 2 * h8 + 1];
+            const float y[8] = {__uint_as_float(ov[8 * h8]) * inv_l + i0.x,     __uint_as_float(ov[8 * h8 + 1]) * inv_l + i0.y,
+                                __uint_as_float(ov[8 * h8 + 2]) * inv_l + i0.z, __uint_as_float(ov[8 * h8 + 3]) * inv_l + i0.w,
+                                __uint_as_float(ov[8 * h8 + 4]) * inv_l + i1.x, __uint_as_float(ov[8 * h8 + 5]) * inv_l + i1.y,
+                                __uint_as_float(ov[8 * h8 + 6]) * inv_l + i1.z, __uint_as_float(ov[8 * h8 + 7]) * inv_l + i1.w};
+            reinterpret_cast<uint4*>(out_row + 16 * c)[h8] = pack8(y);
           }
-          dst[q] = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
-                              pack_bf16x2(y[6], y[7]));
         }
       }
     }
     tc_fence_before();
     mbar_arrive(sm.bar(kBarOEmpty));
-  } else {
-    // Partial record of this segment: O_acc, m, l (and O_inter if it holds key tile 0).
-    const long long first = static_cast<long long>(sg.Q) * a.nkv;
-    const int c_first = owner(first, a);
-    const int nsegs = owner(first + a.nkv - 1, a) - c_first + 1;
-    const int slot = sg.Q * a.max_segs + (static_cast<int>(blockIdx.x) - c_first);
-    float* po = a.part_o + (static_cast<size_t>(slot) * kRows + r) * kDP + c0;
-    float* poi = a.part_oi + (static_cast<size_t>(sg.Q) * kRows + r) * kDP + c0;
-    for (int c = 0; 16 * c < ncols; ++c) {
-      uint32_t ov[16], iv[16];
-      tmem_ld16(tO + c0 + 16u * c, ov);
-      if (kHybrid && sg.head) tmem_ld16(tOI + c0 + 16u * c, iv);
-      tmem_wait_ld();
-      reg_fence16(ov);
-      if (kHybrid && sg.head) reg_fence16(iv);
-      float4* d4 = reinterpret_cast<float4*>(po + 16 * c);
+    return true;
+  }
+  // Partial record of this segment: O_acc (coalesced quads), m, l.
+  const long long first = static_cast<long long>(sg.Q) * a.nkv;
+  const int c_first = owner(first, a);
+  const int nsegs = owner(first + a.nkv - 1, a) - c_first + 1;
+  const size_t slot0 = static_cast<size_t>(sg.Q) * a.max_segs;
+  const size_t slot = slot0 + (static_cast<int>(blockIdx.x) - c_first);
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        d4[q] = make_float4(__uint_as_float(ov[4 * q]), __uint_as_float(ov[4 * q + 1]),
-                            __uint_as_float(ov[4 * q + 2]), __uint_as_float(ov[4 * q + 3]));
-      if (kHybrid && sg.head) {
-        float4* i4 = reinterpret_cast<float4*>(poi + 16 * c);
+  for (int c = 0; c < 4; ++c) {
+    if (16 * c >= ncols) break;
+    uint32_t ov[16];
+    tmem_ld16(tO + c0 + 16u * c, ov);
+    tmem_wait_ld();
+    reg_fence16(ov);
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          i4[q] = make_float4(__uint_as_float(iv[4 * q]), __uint_as_float(iv[4 * q + 1]),
-                              __uint_as_float(iv[4 * q + 2]), __uint_as_float(iv[4 * q + 3]));
-      }
-    }
-    if (half == 0) {
-      a.part_ml[(static_cast<size_t>(slot) * 2) * kRows + r] = m;
-      a.part_ml[(static_cast<size_t>(slot) * 2 + 1) * kRows + r] = l_row;
-    }
-    // TMEM is read: the next segment's MMAs may reuse O and O_inter.
-    tc_fence_before();
-    mbar_arrive(sm.bar(kBarOEmpty));
-    // Publish, then count this segment in; the CTA completing the count merges.
-    __threadfence();
-    if (!group_sync(sm.bar(kBarGroup), gphase, g)) return false;
-    if (half == 0 && r == 0) {
-      const int prev = atomicAdd(a.cnt + sg.Q, 1);
-      *merge_flag = (prev == nsegs - 1) ? 1 : 0;
-    }
-    if (!group_sync(sm.bar(kBarGroup), gphase, g)) return false;
-    if (*merge_flag) {
-      __threadfence();
-      float M = -INFINITY;
-      for (int s = 0; s < nsegs; ++s)
-        M = fmaxf(M, __ldcg(a.part_ml + (static_cast<size_t>(sg.Q * a.max_segs + s) * 2) * kRows + r));
-      float L = 0.f, wgt[kMaxSegs];
-      for (int s = 0; s < nsegs && s < kMaxSegs; ++s) {
-        const size_t sl = static_cast<size_t>(sg.Q * a.max_segs + s);
-        wgt[s] = ex2_approx(__ldcg(a.part_ml + (sl * 2) * kRows + r) - M);
-        L += wgt[s] * __ldcg(a.part_ml + (sl * 2 + 1) * kRows + r);
-      }
-      const float inv_L = 1.f / L;
-      for (int c = 0; 8 * c < ncols; ++c) {
-        float y[8];
+    for (int q = 0; q < 4; ++q)
+      *quad_ptr(a.part_o, slot, q0 + 4 * c + q, r) =
+          make_float4(__uint_as_float(ov[4 * q]), __uint_as_float(ov[4 * q + 1]), __uint_as_float(ov[4 * q + 2]),
+                      __uint_as_float(ov[4 * q + 3]));
+  }
+  if (half == 0) {
+    a.part_ml[(slot * 2) * kRows + r] = m;
+    a.part_ml[(slot * 2 + 1) * kRows + r] = l_row;
+  }
+  // TMEM is read: the next segment's MMAs may reuse O.
+  tc_fence_before();
+  mbar_arrive(sm.bar(kBarOEmpty));
+  // Publish, then count this segment in; the CTA completing the count merges.
+  __threadfence();
+  if (!group_sync(sm.bar(kBarGroup), gphase, g)) return false;
+  if (half == 0 && r == 0) {
+    const int prev = atomicAdd(a.cnt + sg.Q, 1);
+    *merge_flag = (prev == nsegs - 1) ? 1 : 0;
+  }
+  if (!group_sync(sm.bar(kBarGroup), gphase, g)) return false;
+  if (!*merge_flag) return true;
+  __threadfence();
+  float ms[kMaxSegs], ls[kMaxSegs];
+  float M = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) y[e] = 0.f;
-        for (int s = 0; s < nsegs && s < kMaxSegs; ++s) {
-          const float4* src = reinterpret_cast<const float4*>(
-              a.part_o + (static_cast<size_t>(sg.Q * a.max_segs + s) * kRows + r) * kDP + c0 + 8 * c);
-          const float4 u0 = __ldcg(src), u1 = __ldcg(src + 1);
-          y[0] += wgt[s] * u0.x;
-          y[1] += wgt[s] * u0.y;
-          y[2] += wgt[s] * u0.z;
-          y[3] += wgt[s] * u0.w;
-          y[4] += wgt[s] * u1.x;
-          y[5] += wgt[s] * u1.y;
-          y[6] += wgt[s] * u1.z;
-          y[7] += wgt[s] * u1.w;
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) y[e] *= inv_L;
-        if (kHybrid) {
-          const float4* src = reinterpret_cast<const float4*>(poi + 8 * c);
-          const float4 u0 = __ldcg(src), u1 = __ldcg(src + 1);
-          y[0] += u0.x;
-          y[1] += u0.y;
-          y[2] += u0.z;
-          y[3] += u0.w;
-          y[4] += u1.x;
-          y[5] += u1.y;
-          y[6] += u1.z;
-          y[7] += u1.w;
-        }
-        if (row_ok)
-          *reinterpret_cast<uint4*>(out_row + c0 + 8 * c) = make_uint4(
-              pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
-      }
-      if (half == 0 && r == 0) a.cnt[sg.Q] = 0;   // ready for the next launch
+  for (int s = 0; s < kMaxSegs; ++s) {
+    if (s < nsegs) {
+      ms[s] = __ldcg(a.part_ml + ((slot0 + s) * 2) * kRows + r);
+      ls[s] = __ldcg(a.part_ml + ((slot0 + s) * 2 + 1) * kRows + r);
+      M = fmaxf(M, ms[s]);
     }
   }
+  float L = 0.f;
+#pragma unroll
+  for (int s = 0; s < kMaxSegs; ++s)
+    if (s < nsegs) L += ex2_approx(ms[s] - M) * ls[s];
+  const float inv_L = 1.f / L;
+  // Two passes of 8 column quads; each pass issues one segment's 8 loads at a time.
+#pragma unroll
+  for (int hp = 0; hp < 2; ++hp) {
+    if (32 * hp >= ncols) break;
+    float4 acc[8], oi[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      oi[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (kHybrid && 8 * hp + q < nquads) oi[q] = __ldcg(quad_ptr(a.part_oi, sg.Q, q0 + 8 * hp + q, r));
+    }
+#pragma unroll
+    for (int s = 0; s < kMaxSegs; ++s) {
+      if (s < nsegs) {
+        const float w = ex2_approx(ms[s] - M);
+        float4 v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          v[q] = (8 * hp + q < nquads) ? __ldcg(quad_ptr(a.part_o, slot0 + s, q0 + 8 * hp + q, r))
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          acc[q].x += w * v[q].x;
+          acc[q].y += w * v[q].y;
+          acc[q].z += w * v[q].z;
+          acc[q].w += w * v[q].w;
+        }
+      }
+    }
+    if (row_ok) {
+#pragma unroll
+      for (int h8 = 0; h8 < 4; ++h8) {
+        if (32 * hp + 8 * h8 >= ncols) break;
+        const float4 a0 = acc[2 * h8], a1 = acc[2 * h8 + 1], i0 = oi[2 * h8], i1 = oi[2 * h8 + 1];
+        const float y[8] = {a0.x * inv_L + i0.x, a0.y * inv_L + i0.y, a0.z * inv_L + i0.z, a0.w * inv_L + i0.w,
+                            a1.x * inv_L + i1.x, a1.y * inv_L + i1.y, a1.z * inv_L + i1.z, a1.w * inv_L + i1.w};
+        reinterpret_cast<uint4*>(out_row + 32 * hp)[h8] = pack8(y);
+      }
+    }
+  }
+  if (half == 0 && r == 0) a.cnt[sg.Q] = 0;   // ready for the next launch
   return true;
 }
 
@@ -465,59 +508,90 @@ __device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const 
   const uint32_t r = quarter * 32 + lane;                   // tile row == TMEM lane
   const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
   const uint32_t tO = tmem + lane_off + kColO;
-  const uint32_t tOI = tmem + lane_off + kColOI;
-  float* xch = reinterpret_cast<float*>(ctl + kCtlX);            // [2 buffers][2 halves][128]
+  float* xch = reinterpret_cast<float*>(ctl + kCtlX);      // [2 halves][128]
   volatile int* merge_flag = reinterpret_cast<volatile int*>(ctl + kCtlMisc + 8);
   const int d = a.d;
   const int c0 = 64 * half;                                 // first column of this thread's half
+  const int oc = 64 - c0;                                   // first column of the other half
   const int ncols = max(0, min(64, d - c0));                // output columns of this half
   uint32_t nseg = 0, nhead = 0, tile = 0, gphase = 0;
   Sched sch(a, blockIdx.x);
   Seg sg;
   while (sch.next(sg)) {
-    const bool rd = kHybrid && sg.head;
     const uint32_t t0 = tile, n = sg.ke - sg.kb;
-    if (rd) {
-      // Q' (fp32, O_inter columns) -> bf16 pairs in the O columns, the readout MMA's A operand.
+    if (kHybrid && sg.head) {
+      // Q' (fp32, O columns) -> bf16 pairs over this half's own O columns: the readout
+      // MMA's A operand.
       if (!mbar_wait_warp(sm.bar(kBarQp), nhead & 1, g)) return;
       tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t x[32], pk[16];
-        tmem_ld32(tOI + c0 + 32u * c, x);
+      {
+        uint32_t x0[32], x1[32], pk[32];
+        tmem_ld32(tO + c0, x0);
+        tmem_ld32(tO + c0 + 32, x1);
         tmem_wait_ld();
-        reg_fence(x);
+        reg_fence(x0);
+        reg_fence(x1);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(x[2 * i]), __uint_as_float(x[2 * i + 1]));
-        tmem_st16(tO + c0 / 2 + 16u * c, pk);
+        for (int i = 0; i < 16; ++i) {
+          pk[i] = pack_bf16x2(__uint_as_float(x0[2 * i]), __uint_as_float(x0[2 * i + 1]));
+          pk[16 + i] = pack_bf16x2(__uint_as_float(x1[2 * i]), __uint_as_float(x1[2 * i + 1]));
+        }
+        tmem_st32(tO + c0, pk);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(sm.bar(kBarQpReady));
+      // O_inter (fp32, the S buffer of tile t0 + 2) -> this half's quads of the tile's
+      // O_inter record in scratch.
+      if (!mbar_wait_warp(sm.bar(kBarOIReady), nhead & 1, g)) return;
+      tc_fence_after();
+      {
+        const uint32_t tX = tmem + lane_off + 128u * sbuf(t0 + 2);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (16 * c >= ncols) break;
+          uint32_t x[16];
+          tmem_ld16(tX + c0 + 16u * c, x);
+          tmem_wait_ld();
+          reg_fence16(x);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            *quad_ptr(a.part_oi, sg.Q, c0 / 4 + 4 * c + q, r) =
+                make_float4(__uint_as_float(x[4 * q]), __uint_as_float(x[4 * q + 1]), __uint_as_float(x[4 * q + 2]),
+                            __uint_as_float(x[4 * q + 3]));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(sm.bar(kBarOIFree));
       ++nhead;
     }
 
     float m = -INFINITY, l = 0.f;
     for (uint32_t i = 0; i < n; ++i) {
       const uint32_t t = t0 + i;
-      const int st = t & 1;
-      if (!mbar_wait_warp(sm.bar(kBarSFull + st), (t >> 1) & 1, g)) return;
+      const int sb = sbuf(t);
+      if (!mbar_wait_warp(sm.bar(kBarSFull + sb), sphase(t), g)) return;
       tc_fence_after();
-      const uint32_t tS = tmem + lane_off + kColS0 + 128u * st;
+      const uint32_t tS = tmem + lane_off + 128u * sb;
       const int valid = a.kv_len - (sg.kb + static_cast<int>(i)) * kRows;   // >= 1
-      // This half's 64 scores; the row max is combined with the other half's through
-      // shared memory (each half reads and overwrites only its own columns).
+      // Row max over both halves: the other half's scores are read first and dropped,
+      // then this half's are kept. Both halves leave the scores intact until every
+      // thread has read them (kBarSRead).
       uint32_t sv[2][32];
+      tmem_ld32(tS + oc, sv[0]);
+      tmem_ld32(tS + oc + 32, sv[1]);
+      tmem_wait_ld();
+      reg_fence(sv[0]);
+      reg_fence(sv[1]);
+      float mt = half_max(sv, oc, valid);
       tmem_ld32(tS + c0, sv[0]);
       tmem_ld32(tS + c0 + 32, sv[1]);
       tmem_wait_ld();
       reg_fence(sv[0]);
       reg_fence(sv[1]);
-      const float mh = half_max(sv, c0, valid);
-      float* xb = xch + (t & 1) * 256;
-      xb[half * 128 + r] = mh;
-      if (!group_sync(sm.bar(kBarGroup), gphase, g)) return;
-      const float mt = fmaxf(mh, xb[(half ^ 1) * 128 + r]) * a.scale_log2;
+      tc_fence_before();
+      mbar_arrive(sm.bar(kBarSRead + sb));
+      mt = fmaxf(mt, half_max(sv, c0, valid)) * a.scale_log2;
       float m_new = m;
       bool rescale = false;
       if (i == 0) {
@@ -528,7 +602,7 @@ __device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const 
       }
       if (__any_sync(0xffffffffu, rescale)) {
         // O holds the sum up to tile t-1: wait for that P.V MMA, then scale this half-row.
-        if (!mbar_wait_warp(sm.bar(kBarPVDone + ((t - 1) & 1)), ((t - 1) >> 1) & 1, g)) return;
+        if (!mbar_wait_warp(sm.bar(kBarPVDone + sbuf(t - 1)), sphase(t - 1), g)) return;
         tc_fence_after();
         const float corr = rescale ? ex2_approx(m - m_new) : 1.f;
 #pragma unroll
@@ -544,24 +618,26 @@ __device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const 
         l *= corr;
       }
       m = m_new;
-      l += half_probs(sv, m, a.scale_log2, tS + c0);
+      uint32_t pk[32];
+      l += half_probs(sv, m, a.scale_log2, pk);
+      // P overwrites the first 32 of this half's score columns once both halves read them.
+      if (!mbar_wait_warp(sm.bar(kBarSRead + sb), sphase(t), g)) return;
+      tc_fence_after();
+      tmem_st32(tS + c0, pk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(sm.bar(kBarPFull + st));
+      mbar_arrive(sm.bar(kBarPFull + sb));
     }
     tile += n;
 
     // ---- end of segment: every MMA of it is done; combine the two half-row sums.
     if (!mbar_wait_warp(sm.bar(kBarOFull), nseg & 1, g)) return;
     tc_fence_after();
-    // The exchange buffer of the next tile's parity is idle: no thread writes it again
-    // before the extra rendezvous below.
-    float* xs = xch + (tile & 1) * 256;
-    xs[half * 128 + r] = l;
+    xch[half * 128 + r] = l;
     if (!group_sync(sm.bar(kBarGroup), gphase, g)) return;
-    const float l_row = xs[r] + xs[128 + r];
-    if (!group_sync(sm.bar(kBarGroup), gphase, g)) return;
-    if (!segment_epilogue<kHybrid>(sm, a, sg, r, half, c0, ncols, tO, tOI, m, l_row, gphase, merge_flag, g)) return;
+    const float l_row = xch[r] + xch[128 + r];
+    if (!group_sync(sm.bar(kBarGroup), gphase, g)) return;   // before anyone rewrites xch
+    if (!segment_epilogue<kHybrid>(sm, a, sg, r, half, c0, ncols, tO, m, l_row, gphase, merge_flag, g)) return;
     ++nseg;
   }
 }
@@ -594,13 +670,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(sm.bar(kBarVFull + s), 1);
       mbar_init(sm.bar(kBarVEmpty + s), 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kSBufs; ++s) {
       mbar_init(sm.bar(kBarSFull + s), 1);
+      mbar_init(sm.bar(kBarSRead + s), kSoftmaxThreads);
       mbar_init(sm.bar(kBarPFull + s), kSoftmaxThreads);
       mbar_init(sm.bar(kBarPVDone + s), 1);
     }
     mbar_init(sm.bar(kBarQp), 1);
     mbar_init(sm.bar(kBarQpReady), kSoftmaxThreads);
+    mbar_init(sm.bar(kBarOIReady), 1);
+    mbar_init(sm.bar(kBarOIFree), kSoftmaxThreads);
     mbar_init(sm.bar(kBarOFull), 1);
     mbar_init(sm.bar(kBarOEmpty), kSoftmaxThreads);
     mbar_init(sm.bar(kBarFinal), 1);
