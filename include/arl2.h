@@ -123,9 +123,16 @@ arl2_status arl2_get_status(arl2_ctx* ctx);
 
 /* Limit on every wait inside this context's kernels, in nanoseconds (default 1e9). When
  * a wait runs out, the kernel abandons the call and returns; arl2_get_status then reports
- * ARL2_ERR_TIMEOUT. Very small values make ordinary waits run out, which tests use to
- * exercise that path. */
+ * ARL2_ERR_TIMEOUT. Returns ARL2_ERR_INVALID_ARG for NULL or 0. */
 arl2_status arl2_set_wait_timeout_ns(arl2_ctx* ctx, uint64_t timeout_ns);
+
+/* Failure-detection test hook. The next arl2_frame_query (or arl2_frame_query_host)
+ * launch makes its softmax threads wait on an mbarrier that nothing signals. That wait
+ * runs out after the context's wait limit; every role of the kernel then stops, drains
+ * what it issued and frees its tensor memory, and arl2_get_status reports
+ * ARL2_ERR_TIMEOUT. The output of that call is undefined. The hook clears itself after
+ * that one launch. Returns ARL2_ERR_INVALID_ARG for NULL. */
+arl2_status arl2_test_stall_next_query(arl2_ctx* ctx);
 
 /* Bytes of device memory the context holds (everything allocated in arl2_create). */
 size_t arl2_memory_bytes(const arl2_ctx* ctx);

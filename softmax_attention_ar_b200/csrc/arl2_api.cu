@@ -137,6 +137,7 @@ struct arl2_ctx {
   int cur = 0;                    // buffer holding S_{N-1}
   int frame = 0;
   bool maps_set = false;
+  bool stall_next = false;        // failure-detection test hook (next query only)
   unsigned long long timeout_ns = kDefaultTimeoutNs;
   CUtensorMap tm_w[3];
   CUtensorMap tm_s;
@@ -222,6 +223,8 @@ arl2_status query_impl(arl2_ctx* c, const void* q, const void* k, const void* v,
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->d)));
   a.err = c->err;
   a.timeout_ns = c->timeout_ns;
+  a.stall = c->stall_next ? 1 : 0;
+  c->stall_next = false;
   set_plan(&a, c->qplan, c->qscratch, c->qcnt);
   return arl2::launch_query(true, *mq, *mk, *mv, c->tm_w[0], c->tm_s, a, st) == cudaSuccess ? ARL2_OK
                                                                                            : ARL2_ERR_CUDA;
@@ -437,6 +440,12 @@ arl2_status arl2_get_status(arl2_ctx* c) {
 arl2_status arl2_set_wait_timeout_ns(arl2_ctx* c, uint64_t timeout_ns) {
   if (!c || timeout_ns == 0) return ARL2_ERR_INVALID_ARG;
   c->timeout_ns = timeout_ns;
+  return ARL2_OK;
+}
+
+arl2_status arl2_test_stall_next_query(arl2_ctx* c) {
+  if (!c) return ARL2_ERR_INVALID_ARG;
+  c->stall_next = true;
   return ARL2_OK;
 }
 

@@ -21,6 +21,7 @@ struct QueryArgs {
   float scale_log2;       // log2(e) / sqrt(d)
   unsigned int* err;      // device error word
   unsigned long long timeout_ns;
+  int stall;              // test hook: the softmax threads wait on a barrier nothing signals
   // Persistent stream-K split (see QueryPlan) and its scratch.
   int nq, nkv;            // query tiles and key tiles per (batch, head)
   long long units;        // B * H * nq * nkv (query tile, key tile) pairs

@@ -30,9 +30,10 @@
 //               the bf16 state copy S_h goes first, through the ring.
 //   warps 4-11  two softmax warpgroups. Thread = query row = TMEM lane; warps 4-7 own
 //               score and output columns 0-63, warps 8-11 columns 64-127. A thread reads
-//               the whole score row for its max but writes P only over its own columns,
-//               after both halves have read the tile. These threads also pack Q' for the
-//               readout MMA and write outputs and partial records.
+//               and writes only its own half-row; warps w and w+4 (same rows, same SM
+//               sub-partition) swap half-row maxima through shared memory each tile.
+//               These threads also pack Q' for the readout MMA and write outputs and
+//               partial records.
 // TMEM (512 columns):
 //   - cols 0, 128, 256: three S tiles. The score MMA of tile t+2 is queued right behind
 //     the P.V MMA of tile t and writes the buffer last read two MMA groups earlier, so no
@@ -47,8 +48,9 @@
 //
 // Online softmax: scores are kept in log2 units. The running max m is raised only when a
 // tile's max exceeds it by more than 8 (a factor of 256), so O in TMEM is rescaled rarely.
-// Probabilities stay below 2^8. A quarter of the exponentials run on the FMA pipe
-// (exp2_poly) and the rest on the MUFU unit.
+// Probabilities stay below 2^8. Three column pairs in eight take their exponentials on
+// the FMA pipe (exp2_poly2) and the rest on the MUFU unit; scaling, sums and the
+// polynomial use the paired fp32 instructions.
 #include <algorithm>
 
 #include "arl2_device.cuh"
@@ -69,18 +71,19 @@ enum : int {
   kBarVFull = 8,
   kBarVEmpty = 11,
   kBarSFull = 14,     // +S buffer (3): scores of a tile are in TMEM
-  kBarSRead = 17,     // +S buffer: both halves have read them (256 arrivals)
-  kBarPFull = 20,     // +S buffer: P written over them (256 arrivals)
-  kBarPVDone = 23,    // +S buffer: the P.V MMA that read P is done
-  kBarQp = 26,        // Q' = Q Wq is in TMEM (O columns)
-  kBarQpReady = 27,   // Q' is packed to bf16 (256 arrivals)
-  kBarOIReady = 28,   // O_inter is in TMEM (a free S buffer)
-  kBarOIFree = 29,    // O_inter was read out (256 arrivals)
-  kBarOFull = 30,     // the segment's MMAs are all done
-  kBarOEmpty = 31,    // the segment's O was read (256 arrivals)
-  kBarFinal = 32,
-  kBarGroup = 33,     // bounded rendezvous of the softmax threads (256 arrivals)
-  kNumBars = 34
+  kBarPFull = 17,     // +S buffer: P written over them (256 arrivals)
+  kBarPVDone = 20,    // +S buffer: the P.V MMA that read P is done
+  kBarQp = 23,        // Q' = Q Wq is in TMEM (O columns)
+  kBarQpReady = 24,   // Q' is packed to bf16 (256 arrivals)
+  kBarOIReady = 25,   // O_inter is in TMEM (a free S buffer)
+  kBarOIFree = 26,    // O_inter was read out (256 arrivals)
+  kBarOFull = 27,     // the segment's MMAs are all done
+  kBarOEmpty = 28,    // the segment's O was read (256 arrivals)
+  kBarFinal = 29,
+  kBarGroup = 30,     // bounded rendezvous of the softmax threads (256 arrivals)
+  kBarPair = 31,      // +row quarter (4): the two warps of those rows swapped half-row maxima
+  kBarNever = 35,     // never signalled: target of the failure-detection test hook
+  kNumBars = 36
 };
 // Tiles at the (1 KiB-aligned) base of dynamic shared memory, then the control block.
 constexpr uint32_t kQOff = 0;
@@ -89,8 +92,10 @@ constexpr uint32_t kVOff = kKOff + kStages * kTileBytes;
 constexpr uint32_t kTileRegion = kVOff + kStages * kTileBytes;
 constexpr uint32_t kCtlBars = 0;
 constexpr uint32_t kCtlMisc = 320;           // tmem slot, abort flag, merge flag
-constexpr uint32_t kCtlX = 384;              // [2 halves][128] fp32 row-sum exchange
-constexpr uint32_t kCtlBytes = kCtlX + 2 * 128 * 4;
+// [2 slots][2 halves][128] fp32: per-tile half-row maxima (slot = tile parity); slot 0
+// also carries the end-of-segment row sums.
+constexpr uint32_t kCtlX = 384;
+constexpr uint32_t kCtlBytes = kCtlX + 2 * 2 * 128 * 4;
 static_assert(kNumBars * 8 <= kCtlMisc, "barriers must fit their slot");
 constexpr uint32_t kSmemBytes = kTileRegion + kCtlBytes;
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
@@ -161,7 +166,7 @@ __device__ __forceinline__ uint32_t sphase(uint32_t t) { return (t / kSBufs) & 1
 // producer also loads each segment's Q tile.
 template <bool kHybrid, bool kIsK>
 __device__ void producer(const Smem& sm, const CUtensorMap* tm_q, const CUtensorMap* tm_kv, const CUtensorMap* tm_rd,
-                         const QueryArgs& a, const Guard& g) {
+                         const QueryArgs& a, const Guard& g, bool lead) {
   const int full0 = kIsK ? kBarKFull : kBarVFull, empty0 = kIsK ? kBarKEmpty : kBarVEmpty;
   uint32_t nissued[kStages] = {0, 0, 0};
   uint32_t nseg = 0, ring = 0;
@@ -169,23 +174,27 @@ __device__ void producer(const Smem& sm, const CUtensorMap* tm_q, const CUtensor
   Seg sg;
   bool ok = true;
   auto slot_wait = [&](uint32_t gidx) -> bool {
-    return gidx < kStages || mbar_wait(sm.bar(empty0 + ring_stage(gidx)), ring_phase(gidx - kStages), g);
+    return gidx < kStages || mbar_wait_warp(sm.bar(empty0 + ring_stage(gidx)), ring_phase(gidx - kStages), g);
   };
   auto tile_addr = [&](int s) { return kIsK ? sm.k(s) : sm.v(s); };
   while (ok && sch.next(sg)) {
     if (kIsK) {
-      if (nseg > 0 && !mbar_wait(sm.bar(kBarQEmpty), (nseg - 1) & 1, g)) break;
-      mbar_expect_tx(sm.bar(kBarQFull), kTileBytes);
-      for (int p = 0; p < 2; ++p)
-        tma_load_4d(sm.q() + p * kPanelBytes, tm_q, sm.bar(kBarQFull), 64 * p, sg.h, sg.qt * kRows, sg.b);
+      if (nseg > 0 && !mbar_wait_warp(sm.bar(kBarQEmpty), (nseg - 1) & 1, g)) break;
+      if (lead) {
+        mbar_expect_tx(sm.bar(kBarQFull), kTileBytes);
+        for (int p = 0; p < 2; ++p)
+          tma_load_4d(sm.q() + p * kPanelBytes, tm_q, sm.bar(kBarQFull), 64 * p, sg.h, sg.qt * kRows, sg.b);
+      }
     }
     ++nseg;
     if (kHybrid && sg.head) {
       if (!slot_wait(ring)) break;
       const int s = ring_stage(ring);
-      mbar_expect_tx(sm.bar(full0 + s), kTileBytes);
       const int c2 = kIsK ? sg.h : a.state_slot * a.B * a.H + sg.b * a.H + sg.h;
-      for (int p = 0; p < 2; ++p) tma_load_3d(tile_addr(s) + p * kPanelBytes, tm_rd, sm.bar(full0 + s), 64 * p, 0, c2);
+      if (lead) {
+        mbar_expect_tx(sm.bar(full0 + s), kTileBytes);
+        for (int p = 0; p < 2; ++p) tma_load_3d(tile_addr(s) + p * kPanelBytes, tm_rd, sm.bar(full0 + s), 64 * p, 0, c2);
+      }
       ++nissued[s];
       ++ring;
     }
@@ -195,9 +204,11 @@ __device__ void producer(const Smem& sm, const CUtensorMap* tm_q, const CUtensor
         break;
       }
       const int s = ring_stage(ring);
-      mbar_expect_tx(sm.bar(full0 + s), kTileBytes);
-      for (int p = 0; p < 2; ++p)
-        tma_load_4d(tile_addr(s) + p * kPanelBytes, tm_kv, sm.bar(full0 + s), 64 * p, sg.h, j * kRows, sg.b);
+      if (lead) {
+        mbar_expect_tx(sm.bar(full0 + s), kTileBytes);
+        for (int p = 0; p < 2; ++p)
+          tma_load_4d(tile_addr(s) + p * kPanelBytes, tm_kv, sm.bar(full0 + s), 64 * p, sg.h, j * kRows, sg.b);
+      }
       ++nissued[s];
     }
   }
@@ -210,7 +221,7 @@ __device__ void producer(const Smem& sm, const CUtensorMap* tm_q, const CUtensor
 
 
 template <bool kHybrid>
-__device__ void mma_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, const Guard& g) {
+__device__ void mma_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, const Guard& g, bool lead) {
   constexpr uint32_t id_kk = idesc_bf16(128, 128, false, false);   // A, B K-major
   constexpr uint32_t id_kmn = idesc_bf16(128, 128, false, true);   // A K-major (smem or TMEM), B MN-major
   const uint32_t tO = tmem + kColO;
@@ -222,12 +233,14 @@ __device__ void mma_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, co
   // tile (t - 3) was consumed by a P.V MMA issued earlier, so in-order execution keeps it.
   auto issue_qk = [&](uint32_t t, uint32_t r) -> bool {
     const int sb = sbuf(t), ks = ring_stage(r);
-    if (!mbar_wait(sm.bar(kBarKFull + ks), ring_phase(r), g)) return false;
+    if (!mbar_wait_warp(sm.bar(kBarKFull + ks), ring_phase(r), g)) return false;
     tc_fence_after();
     const uint32_t tS = tmem + 128u * sb;
-    mma8_ss<false, false>(tS, desc_kmajor(sm.q(), 0), desc_kmajor(sm.k(ks), 0), id_kk, 0u);
-    mma_commit(sm.bar(kBarKEmpty + ks));
-    mma_commit(sm.bar(kBarSFull + sb));
+    if (lead) {
+      mma8_ss<false, false>(tS, desc_kmajor(sm.q(), 0), desc_kmajor(sm.k(ks), 0), id_kk, 0u);
+      mma_commit(sm.bar(kBarKEmpty + ks));
+      mma_commit(sm.bar(kBarSFull + sb));
+    }
     return true;
   };
   while (sch.next(sg)) {
@@ -239,38 +252,42 @@ __device__ void mma_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, co
     // the P.V MMA before that one, so adjacent MMA groups never touch the same TMEM columns
     // (an MMA that overwrites columns the MMA just ahead of it still reads stalls the pipe).
     const uint32_t npre = min(n, 2u);
-    if (!mbar_wait(sm.bar(kBarQFull), nseg & 1, g)) return;
+    if (!mbar_wait_warp(sm.bar(kBarQFull), nseg & 1, g)) return;
     tc_fence_after();
     for (uint32_t i = 0; i < npre; ++i)
       if (!issue_qk(t0 + i, r0 + i)) return;
     // O of the previous segment must have been read before it is rewritten.
-    if (nseg > 0 && !mbar_wait(sm.bar(kBarOEmpty), (nseg - 1) & 1, g)) return;
+    if (nseg > 0 && !mbar_wait_warp(sm.bar(kBarOEmpty), (nseg - 1) & 1, g)) return;
     tc_fence_after();
     if (rd) {
       // Q' = Q Wq_h (phi_q) into the O columns; Wq_h sits in K slot r_rd.
       const int ws = ring_stage(r_rd);
-      if (!mbar_wait(sm.bar(kBarKFull + ws), ring_phase(r_rd), g)) return;
+      if (!mbar_wait_warp(sm.bar(kBarKFull + ws), ring_phase(r_rd), g)) return;
       tc_fence_after();
-      mma8_ss<false, true>(tO, desc_kmajor(sm.q(), 0), desc_mnmajor(sm.k(ws), 0), id_kmn, 0u);
-      mma_commit(sm.bar(kBarKEmpty + ws));
-      mma_commit(sm.bar(kBarQp));
+      if (lead) {
+        mma8_ss<false, true>(tO, desc_kmajor(sm.q(), 0), desc_mnmajor(sm.k(ws), 0), id_kmn, 0u);
+        mma_commit(sm.bar(kBarKEmpty + ws));
+        mma_commit(sm.bar(kBarQp));
+      }
     }
-    if (n <= npre) mma_commit(sm.bar(kBarQEmpty));
+    if (lead && n <= npre) mma_commit(sm.bar(kBarQEmpty));
     if (rd) {
       // O_inter = Q' S_{N-1}: Q' packed to bf16 in the O columns, S_h in V slot r_rd, the
       // result in the S buffer of tile t0 + 2 (free until that tile's scores are issued).
       const int ss = ring_stage(r_rd);
-      if (!mbar_wait(sm.bar(kBarQpReady), nhead & 1, g)) return;
-      if (!mbar_wait(sm.bar(kBarVFull + ss), ring_phase(r_rd), g)) return;
+      if (!mbar_wait_warp(sm.bar(kBarQpReady), nhead & 1, g)) return;
+      if (!mbar_wait_warp(sm.bar(kBarVFull + ss), ring_phase(r_rd), g)) return;
       tc_fence_after();
       const uint32_t tX = tmem + 128u * sbuf(t0 + 2);
-      mma8_ts(tX, tO, kPacked, desc_mnmajor(sm.v(ss), 0), id_kmn, 0u);
-      mma_commit(sm.bar(kBarVEmpty + ss));
-      mma_commit(sm.bar(kBarOIReady));
+      if (lead) {
+        mma8_ts(tX, tO, kPacked, desc_mnmajor(sm.v(ss), 0), id_kmn, 0u);
+        mma_commit(sm.bar(kBarVEmpty + ss));
+        mma_commit(sm.bar(kBarOIReady));
+      }
       // Whatever tile next scores into that buffer (this segment's or a later one's) must
       // wait for the read-out. It costs nothing here: the first P.V of the segment needs
       // the softmax threads, which read O_inter out first.
-      if (!mbar_wait(sm.bar(kBarOIFree), nhead & 1, g)) return;
+      if (!mbar_wait_warp(sm.bar(kBarOIFree), nhead & 1, g)) return;
       tc_fence_after();
       ++nhead;
     }
@@ -278,26 +295,29 @@ __device__ void mma_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, co
     for (uint32_t i = 0; i < n; ++i) {
       const uint32_t t = t0 + i, r = r0 + i;
       const int sb = sbuf(t), vs = ring_stage(r);
-      if (!mbar_wait(sm.bar(kBarPFull + sb), sphase(t), g)) return;
-      if (!mbar_wait(sm.bar(kBarVFull + vs), ring_phase(r), g)) return;
+      if (!mbar_wait_warp(sm.bar(kBarPFull + sb), sphase(t), g)) return;
+      if (!mbar_wait_warp(sm.bar(kBarVFull + vs), ring_phase(r), g)) return;
       tc_fence_after();
       const uint32_t tP = tmem + 128u * sb;
-      mma8_ts(tO, tP, kPacked, desc_mnmajor(sm.v(vs), 0), id_kmn, i > 0 ? 1u : 0u);
-      mma_commit(sm.bar(kBarPVDone + sb));
-      mma_commit(sm.bar(kBarVEmpty + vs));
+      if (lead) {
+        mma8_ts(tO, tP, kPacked, desc_mnmajor(sm.v(vs), 0), id_kmn, i > 0 ? 1u : 0u);
+        mma_commit(sm.bar(kBarPVDone + sb));
+        mma_commit(sm.bar(kBarVEmpty + vs));
+      }
       if (i + nissued < n) {
         if (!issue_qk(t + nissued, r + nissued)) return;
-        if (i + nissued + 1 == n) mma_commit(sm.bar(kBarQEmpty));
+        if (lead && i + nissued + 1 == n) mma_commit(sm.bar(kBarQEmpty));
       }
     }
-    mma_commit(sm.bar(kBarOFull));
+    if (lead) mma_commit(sm.bar(kBarOFull));
     tile += n;
     ring = r0 + n;
     ++nseg;
   }
 }
 
-// Row max of 64 score columns (raw units), with keys at or beyond `valid` masked.
+// Max of this half's 64 score columns (raw units), with keys at or beyond `valid` masked
+// to -inf. Three-input maxima, four independent chains.
 __device__ __forceinline__ float half_max(uint32_t (&sv)[2][32], int col0, int valid) {
   if (valid < col0 + 64) {
 #pragma unroll
@@ -306,41 +326,41 @@ __device__ __forceinline__ float half_max(uint32_t (&sv)[2][32], int col0, int v
       for (int e = 0; e < 32; ++e)
         if (col0 + 32 * c + e >= valid) sv[c][e] = __float_as_uint(-INFINITY);
   }
-  float mx[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
+  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
   for (int c = 0; c < 2; ++c)
 #pragma unroll
-    for (int e = 0; e < 32; ++e) mx[e & 7] = fmaxf(mx[e & 7], __uint_as_float(sv[c][e]));
-  return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+    for (int e = 0; e < 32; e += 2)
+      mx[(e >> 1) & 3] = fmax3(mx[(e >> 1) & 3], __uint_as_float(sv[c][e]), __uint_as_float(sv[c][e + 1]));
+  return fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
 }
 
+// Column pairs (of every 8) whose exponentials run on the FMA pipe (exp2_poly2); the
+// rest go to the MUFU unit. Three of eight balances the two units for d = 128.
+constexpr uint32_t kPolyPairs = 0xA4u;   // pairs 2, 5, 7
+__host__ __device__ constexpr bool poly_pair(int j) { return (kPolyPairs >> (j & 7)) & 1u; }
+
 // P for 64 score columns (raw fp32 in sv; masked ones are -inf) as 32 packed bf16 pairs
-// in pk. Returns their sum; m is the log2-unit max in use.
+// in pk. Returns their sum; m is the log2-unit max in use. Scaling and sums run on
+// column pairs.
 __device__ __forceinline__ float half_probs(const uint32_t (&sv)[2][32], float m, float scale_log2,
                                             uint32_t (&pk)[32]) {
-  const float neg_m = -m;
-  float acc[8];
+  const float2 sc = make_float2(scale_log2, scale_log2), nm = make_float2(-m, -m);
+  float2 acc[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
 #pragma unroll
-    for (int i = 0; i < 32; i += 2) {
-      float p2[2];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int col = i + e;
-        const float x = fmaf(__uint_as_float(sv[c][col]), scale_log2, neg_m);
-        // Every fourth column on the FMA pipe, the rest on MUFU.
-        p2[e] = ((col & 3) == 3) ? exp2_poly(x) : ex2_approx(x);
-        acc[col & 7] += p2[e];
-      }
-      pk[16 * c + (i >> 1)] = pack_bf16x2(p2[0], p2[1]);
+    for (int j = 0; j < 16; ++j) {
+      const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[c][2 * j]), __uint_as_float(sv[c][2 * j + 1])), sc, nm);
+      const float2 p = poly_pair(j) ? exp2_poly2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+      acc[j & 3] = __fadd2_rn(acc[j & 3], p);
+      pk[16 * c + j] = pack_bf16x2(p.x, p.y);
     }
   }
-  return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+  const float2 s = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+  return s.x + s.y;
 }
 
 // Scratch records are stored column-quad-major: float4 (record, quad q of 4 columns, row r)
@@ -508,13 +528,15 @@ __device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const 
   const uint32_t r = quarter * 32 + lane;                   // tile row == TMEM lane
   const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
   const uint32_t tO = tmem + lane_off + kColO;
-  float* xch = reinterpret_cast<float*>(ctl + kCtlX);      // [2 halves][128]
+  float* xch = reinterpret_cast<float*>(ctl + kCtlX);      // [2 slots][2 halves][128]
   volatile int* merge_flag = reinterpret_cast<volatile int*>(ctl + kCtlMisc + 8);
   const int d = a.d;
   const int c0 = 64 * half;                                 // first column of this thread's half
   const int oc = 64 - c0;                                   // first column of the other half
   const int ncols = max(0, min(64, d - c0));                // output columns of this half
   uint32_t nseg = 0, nhead = 0, tile = 0, gphase = 0;
+  // Test hook: a wait that can only run out (the bounded-wait path, without a fault).
+  if (a.stall && !mbar_wait_warp(sm.bar(kBarNever), 0, g)) return;
   Sched sch(a, blockIdx.x);
   Seg sg;
   while (sch.next(sg)) {
@@ -574,24 +596,21 @@ __device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const 
       tc_fence_after();
       const uint32_t tS = tmem + lane_off + 128u * sb;
       const int valid = a.kv_len - (sg.kb + static_cast<int>(i)) * kRows;   // >= 1
-      // Row max over both halves: the other half's scores are read first and dropped,
-      // then this half's are kept. Both halves leave the scores intact until every
-      // thread has read them (kBarSRead).
+      // This half's scores, then the row max: the two warps holding these rows (one per
+      // half) swap their half-row maxima through shared memory, double-buffered by tile
+      // parity. Each half reads and writes only its own columns.
       uint32_t sv[2][32];
-      tmem_ld32(tS + oc, sv[0]);
-      tmem_ld32(tS + oc + 32, sv[1]);
-      tmem_wait_ld();
-      reg_fence(sv[0]);
-      reg_fence(sv[1]);
-      float mt = half_max(sv, oc, valid);
       tmem_ld32(tS + c0, sv[0]);
       tmem_ld32(tS + c0 + 32, sv[1]);
       tmem_wait_ld();
       reg_fence(sv[0]);
       reg_fence(sv[1]);
-      tc_fence_before();
-      mbar_arrive(sm.bar(kBarSRead + sb));
-      mt = fmaxf(mt, half_max(sv, c0, valid)) * a.scale_log2;
+      float* xm = xch + (t & 1) * 256;
+      xm[half * 128 + r] = half_max(sv, c0, valid);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.bar(kBarPair + quarter));
+      if (!mbar_wait_warp(sm.bar(kBarPair + quarter), t & 1, g)) return;
+      const float mt = fmaxf(xm[r], xm[128 + r]) * a.scale_log2;
       float m_new = m;
       bool rescale = false;
       if (i == 0) {
@@ -620,9 +639,7 @@ __device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const 
       m = m_new;
       uint32_t pk[32];
       l += half_probs(sv, m, a.scale_log2, pk);
-      // P overwrites the first 32 of this half's score columns once both halves read them.
-      if (!mbar_wait_warp(sm.bar(kBarSRead + sb), sphase(t), g)) return;
-      tc_fence_after();
+      // P overwrites the first 32 of this half's score columns.
       tmem_st32(tS + c0, pk);
       tmem_wait_st();
       tc_fence_before();
@@ -672,7 +689,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < kSBufs; ++s) {
       mbar_init(sm.bar(kBarSFull + s), 1);
-      mbar_init(sm.bar(kBarSRead + s), kSoftmaxThreads);
       mbar_init(sm.bar(kBarPFull + s), kSoftmaxThreads);
       mbar_init(sm.bar(kBarPVDone + s), 1);
     }
@@ -684,6 +700,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(sm.bar(kBarOEmpty), kSoftmaxThreads);
     mbar_init(sm.bar(kBarFinal), 1);
     mbar_init(sm.bar(kBarGroup), kSoftmaxThreads);
+    for (int q = 0; q < 4; ++q) mbar_init(sm.bar(kBarPair + q), 2);   // one arrival per warp
+    mbar_init(sm.bar(kBarNever), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -702,16 +720,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // Producers and the MMA issuer run warp-wide (uniform control flow and waits); one
+  // elected lane issues each TMA copy, MMA and commit.
   if (warp == 0) {
-    if (lane == 0) producer<kHybrid, true>(sm, &tm_q, &tm_k, &tm_w, a, g);
+    producer<kHybrid, true>(sm, &tm_q, &tm_k, &tm_w, a, g, elect_one());
   } else if (warp == 1) {
-    if (lane == 0) {
-      mma_issuer<kHybrid>(sm, tmem, a, g);
-      mma_commit(sm.bar(kBarFinal));   // arrives once every MMA issued above has finished
-    }
+    const bool lead = elect_one();
+    mma_issuer<kHybrid>(sm, tmem, a, g, lead);
+    if (lead) mma_commit(sm.bar(kBarFinal));   // arrives once every MMA issued above has finished
     __syncwarp();
   } else if (warp == 2) {
-    if (lane == 0) producer<kHybrid, false>(sm, &tm_q, &tm_v, &tm_s, a, g);
+    producer<kHybrid, false>(sm, &tm_q, &tm_v, &tm_s, a, g, elect_one());
   } else if (warp >= 4) {
     softmax_role<kHybrid>(sm, ctl_ptr, tmem, a, warp, lane, g);
   }

@@ -213,15 +213,29 @@ def test_reset_and_out_of_order_calls():
 
 
 def test_bounded_waits_report_a_timeout_and_leave_the_context_usable():
-    # A 1 ns wait limit makes ordinary waits run out: the kernels abandon the call and return.
+    # The test hook makes one launch wait on a barrier nothing signals: its bounded wait
+    # runs out (1 ms limit), every role stops, and the status says so. The context (TMEM,
+    # counters, barriers of later launches) stays usable.
     c = Case(B=1, T=300, H=2, d=128, config=113)
     q, k, v = (dev_bf16(x) for x in c.inputs(0, 0))
-    c.gpu.set_wait_timeout_ns(1)
+    c.gpu.set_wait_timeout_ns(1_000_000)
+    c.gpu.test_stall_next_query()
     c.gpu.query(q, k, v)
     assert c.gpu.status() == arl2.ARL2_ERR_TIMEOUT
     c.gpu.set_wait_timeout_ns(1_000_000_000)
     assert c.gpu.status() == arl2.ARL2_OK
     o_gpu, o_ref = c.query(0, 0)
+    assert max(o_errors(o_gpu, o_ref)) <= O_TOL
+    # Several stalled launches in a row, on a split plan (partial records and counters).
+    big = Case(B=1, T=1560, H=4, d=128, config=115)
+    q, k, v = (dev_bf16(x) for x in big.inputs(0, 0))
+    big.gpu.set_wait_timeout_ns(1_000_000)
+    for _ in range(3):
+        big.gpu.test_stall_next_query()
+        big.gpu.query(q, k, v)
+        assert big.gpu.status() == arl2.ARL2_ERR_TIMEOUT
+    big.gpu.set_wait_timeout_ns(1_000_000_000)
+    o_gpu, o_ref = big.query(0, 0, rows=sample_rows(1560, 64, seed=5))
     assert max(o_errors(o_gpu, o_ref)) <= O_TOL
 
 
