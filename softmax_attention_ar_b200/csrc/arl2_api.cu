@@ -133,7 +133,8 @@ struct arl2_ctx {
   float* stage_f32[2] = {};       // alpha, beta staging
   arl2::QueryPlan qplan{};        // stream-K split of the query kernel
   float* qscratch = nullptr;      // its partial records
-  int* qcnt = nullptr;            // its per-query-tile counters
+  int* qflags = nullptr;          // their published flags
+  int qepoch = 0;                 // epoch of the last query launch
   int cur = 0;                    // buffer holding S_{N-1}
   int frame = 0;
   bool maps_set = false;
@@ -162,14 +163,21 @@ struct arl2_kvcache {
   int num_sms = 0;
   float* qscratch = nullptr;      // stream-K partial records, sized for the longest cache
   size_t qscratch_floats = 0;
-  int* qcnt = nullptr;            // per-query-tile counters
-  long long qtiles = 0;
+  int* qflags = nullptr;          // record flags, sized for the longest cache
+  size_t qflag_count = 0;
+  int qepoch = 0;
 };
 
 namespace {
 
 // Point a query launch at its stream-K plan and scratch.
-void set_plan(arl2::QueryArgs* a, const arl2::QueryPlan& p, float* scratch, int* cnt) {
+// Epochs of successive launches on one set of flags: nonzero, never the previous one.
+int next_epoch(int* e) {
+  *e = (*e == 0x7fffffff) ? 1 : *e + 1;
+  return *e;
+}
+
+void set_plan(arl2::QueryArgs* a, const arl2::QueryPlan& p, float* scratch, int* flags, int epoch) {
   a->nq = p.nq;
   a->nkv = p.nkv;
   a->units = p.units;
@@ -178,8 +186,8 @@ void set_plan(arl2::QueryArgs* a, const arl2::QueryPlan& p, float* scratch, int*
   const size_t slots = static_cast<size_t>(p.qtiles) * p.max_segs;
   a->part_o = scratch;
   a->part_ml = scratch + slots * 128 * 128;
-  a->part_oi = a->part_ml + slots * 2 * 128;
-  a->cnt = cnt;
+  a->flags = flags;
+  a->epoch = epoch;
 }
 
 template <typename T>
@@ -203,7 +211,7 @@ void free_ctx(arl2_ctx* c) {
   for (auto& p : c->stage_bf16) cudaFree(p);
   for (auto& p : c->stage_f32) cudaFree(p);
   cudaFree(c->qscratch);
-  cudaFree(c->qcnt);
+  cudaFree(c->qflags);
   delete c;
 }
 
@@ -225,7 +233,7 @@ arl2_status query_impl(arl2_ctx* c, const void* q, const void* k, const void* v,
   a.timeout_ns = c->timeout_ns;
   a.stall = c->stall_next ? 1 : 0;
   c->stall_next = false;
-  set_plan(&a, c->qplan, c->qscratch, c->qcnt);
+  set_plan(&a, c->qplan, c->qscratch, c->qflags, next_epoch(&c->qepoch));
   return arl2::launch_query(true, *mq, *mk, *mv, c->tm_w[0], c->tm_s, a, st) == cudaSuccess ? ARL2_OK
                                                                                            : ARL2_ERR_CUDA;
 }
@@ -306,7 +314,7 @@ arl2_status arl2_create(int H, int T, int d_k, int d_v, int B, arl2_ctx** out) {
   for (int i = 0; i < 2 && ok; ++i) ok = dev_alloc(&c->stage_f32[i], (size_t)B * H * T, &c->bytes);
   c->qplan = arl2::plan_query(B, H, T, T, sms);
   ok = ok && dev_alloc(&c->qscratch, arl2::query_scratch_floats(c->qplan), &c->bytes);
-  ok = ok && dev_alloc(&c->qcnt, (size_t)c->qplan.qtiles, &c->bytes);
+  ok = ok && dev_alloc(&c->qflags, arl2::query_flag_count(c->qplan), &c->bytes);
   if (!ok) {
     free_ctx(c);
     return ARL2_ERR_OOM;
@@ -314,7 +322,7 @@ arl2_status arl2_create(int H, int T, int d_k, int d_v, int B, arl2_ctx** out) {
   ok = cudaMemset(c->S[0], 0, c->state_elems() * 4) == cudaSuccess &&
        cudaMemset(c->S[1], 0, c->state_elems() * 4) == cudaSuccess &&
        cudaMemset(c->S_bf16, 0, 2 * c->state_elems() * 2) == cudaSuccess &&
-       cudaMemset(c->qcnt, 0, (size_t)c->qplan.qtiles * sizeof(int)) == cudaSuccess &&
+       cudaMemset(c->qflags, 0, arl2::query_flag_count(c->qplan) * sizeof(int)) == cudaSuccess &&
        cudaMemset(c->err, 0, sizeof(unsigned int)) == cudaSuccess;
   for (int i = 0; i < 3 && ok; ++i) ok = make_mat_map(&c->tm_w[i], c->W[i], H, d_k);
   ok = ok && make_mat_map(&c->tm_s, c->S_bf16, 2 * B * H, d_k);
@@ -417,16 +425,13 @@ arl2_status arl2_set_state(arl2_ctx* c, const float* src, arl2_stream stream) {
 
 int arl2_frame_index(const arl2_ctx* c) { return c ? c->frame : -1; }
 
-// Synchronise, read and clear the error word. After an abandoned launch the query
-// kernel's tile counters may be left mid-count, so they are cleared too.
-static arl2_status read_status(unsigned int* err, int* cnt, size_t ncnt) {
+// Synchronise, read and clear the error word. An abandoned query launch may leave record
+// flags set to its own epoch; later launches use other epochs, so they need no clearing.
+static arl2_status read_status(unsigned int* err) {
   if (cudaDeviceSynchronize() != cudaSuccess) return ARL2_ERR_CUDA;
   unsigned int h = 0;
   if (cudaMemcpy(&h, err, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return ARL2_ERR_CUDA;
-  if (h != 0) {
-    if (cudaMemset(err, 0, sizeof(h)) != cudaSuccess) return ARL2_ERR_CUDA;
-    if (cnt && cudaMemset(cnt, 0, ncnt * sizeof(int)) != cudaSuccess) return ARL2_ERR_CUDA;
-  }
+  if (h != 0 && cudaMemset(err, 0, sizeof(h)) != cudaSuccess) return ARL2_ERR_CUDA;
   if (cudaDeviceSynchronize() != cudaSuccess) return ARL2_ERR_CUDA;
   if (h & arl2::kErrLayoutBit) return ARL2_ERR_CUDA;
   return (h & arl2::kErrTimeoutBit) ? ARL2_ERR_TIMEOUT : ARL2_OK;
@@ -434,7 +439,7 @@ static arl2_status read_status(unsigned int* err, int* cnt, size_t ncnt) {
 
 arl2_status arl2_get_status(arl2_ctx* c) {
   if (!c) return ARL2_ERR_INVALID_ARG;
-  return read_status(c->err, c->qcnt, (size_t)c->qplan.qtiles);
+  return read_status(c->err);
 }
 
 arl2_status arl2_set_wait_timeout_ns(arl2_ctx* c, uint64_t timeout_ns) {
@@ -477,15 +482,15 @@ arl2_status arl2_kvcache_create(int H, int T, int d, int B, int max_frames, arl2
   for (int n = 1; n <= max_frames; ++n) {
     const arl2::QueryPlan p = arl2::plan_query(B, H, T, n * T, sms);
     c->qscratch_floats = std::max(c->qscratch_floats, arl2::query_scratch_floats(p));
-    c->qtiles = p.qtiles;
+    c->qflag_count = std::max(c->qflag_count, arl2::query_flag_count(p));
   }
   bool ok = dev_alloc(&c->K, elems, &c->bytes) && dev_alloc(&c->V, elems, &c->bytes) &&
             dev_alloc(&c->err, 1, &c->bytes) && dev_alloc(&c->qscratch, c->qscratch_floats, &c->bytes) &&
-            dev_alloc(&c->qcnt, (size_t)c->qtiles, &c->bytes);
+            dev_alloc(&c->qflags, c->qflag_count, &c->bytes);
   if (ok)
     ok = cudaMemset(c->K, 0, elems * 2) == cudaSuccess && cudaMemset(c->V, 0, elems * 2) == cudaSuccess &&
          cudaMemset(c->err, 0, 4) == cudaSuccess &&
-         cudaMemset(c->qcnt, 0, (size_t)c->qtiles * sizeof(int)) == cudaSuccess &&
+         cudaMemset(c->qflags, 0, c->qflag_count * sizeof(int)) == cudaSuccess &&
          make_act_map(&c->tm_k, c->K, B, max_frames * T, H, d) &&
          make_act_map(&c->tm_v, c->V, B, max_frames * T, H, d) && cudaDeviceSynchronize() == cudaSuccess;
   if (!ok) {
@@ -526,7 +531,8 @@ arl2_status arl2_kvcache_query(arl2_kvcache* c, const arl2_bf16* q, const arl2_b
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->d)));
   a.err = c->err;
   a.timeout_ns = c->timeout_ns;
-  set_plan(&a, arl2::plan_query(c->B, c->H, c->T, a.kv_len, c->num_sms), c->qscratch, c->qcnt);
+  set_plan(&a, arl2::plan_query(c->B, c->H, c->T, a.kv_len, c->num_sms), c->qscratch, c->qflags,
+           next_epoch(&c->qepoch));
   return arl2::launch_query(false, *mq, c->tm_k, c->tm_v, c->tm_k, c->tm_k, a, st) == cudaSuccess ? ARL2_OK
                                                                                                   : ARL2_ERR_CUDA;
 }
@@ -550,7 +556,7 @@ int arl2_kvcache_frames(const arl2_kvcache* c) { return c ? c->n : -1; }
 
 arl2_status arl2_kvcache_get_status(arl2_kvcache* c) {
   if (!c) return ARL2_ERR_INVALID_ARG;
-  return read_status(c->err, c->qcnt, (size_t)c->qtiles);
+  return read_status(c->err);
 }
 
 size_t arl2_kvcache_memory_bytes(const arl2_kvcache* c) { return c ? c->bytes : 0; }
@@ -561,7 +567,7 @@ void arl2_kvcache_destroy(arl2_kvcache* c) {
   cudaFree(c->V);
   cudaFree(c->err);
   cudaFree(c->qscratch);
-  cudaFree(c->qcnt);
+  cudaFree(c->qflags);
   delete c;
 }
 

@@ -29,8 +29,8 @@ struct QueryArgs {
   int max_segs;           // CTAs sharing one query tile, at most
   float* part_o;          // [qtiles * max_segs][32 column quads][128 rows] float4: partial O accumulators
   float* part_ml;         // [qtiles * max_segs, 2, 128] running max (log2 units) and sum
-  float* part_oi;         // [qtiles][32 column quads][128 rows] float4: O_inter of each query tile
-  int* cnt;               // [qtiles] arrival counters, zero between launches
+  int* flags;             // [qtiles * max_segs] record-published flags, set to the launch's epoch
+  int epoch;              // nonzero, different from the previous launch on the same flags
 };
 
 // The stream-K split of one query launch: CTA c takes units [c*U/P, (c+1)*U/P).
@@ -39,7 +39,8 @@ struct QueryPlan {
   long long units, qtiles;
 };
 QueryPlan plan_query(int B, int H, int T, int kv_len, int num_sms);
-size_t query_scratch_floats(const QueryPlan& p);   // part_o + part_ml + part_oi
+size_t query_scratch_floats(const QueryPlan& p);   // part_o + part_ml
+size_t query_flag_count(const QueryPlan& p);       // flags
 
 // One commit, first kernel: per (group of 128-token chunks, head, batch) partial U and
 // partial sum of alpha.

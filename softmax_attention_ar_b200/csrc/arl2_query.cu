@@ -13,13 +13,16 @@
 // [c*U/P, (c+1)*U/P), so every SM gets the same number of tile pairs. A CTA's range falls
 // into segments, each a key range of one query tile:
 //   - A segment that covers a whole query tile writes O directly.
-//   - Otherwise the CTA writes a partial record (O_acc, running max m, sum l) to scratch
-//     and bumps the tile's counter.
-//   - The CTA that brings the counter to the segment count merges every record of that
-//     tile in key order and writes O. It then resets the counter. The merge order is
-//     fixed, so the result does not depend on which CTA merges it.
-//   - The segment holding key tile 0 computes the readout O_inter first and stores it
-//     (fp32) in the tile's scratch record; whoever finishes the tile adds it.
+//   - The segment holding key tile 0 of a query tile (its head) finishes the tile. With
+//     contiguous ranges it is the last segment of its CTA, and the tile's other segments
+//     open the ranges of the following CTAs, so they are normally done by then.
+//   - Every other segment writes a partial record (O_acc, running max m, sum l) to
+//     scratch; warp 3 then sets the record's flag to the launch's epoch (fence first).
+//   - The head waits for those flags (bounded), merges the records with its own O in
+//     TMEM in a fixed order and writes O. Epochs differ between launches, so no flag
+//     is ever reset.
+//   - The head segment also computes the readout O_inter, after its last P.V MMA, into a
+//     free S tile in TMEM, and adds it when it writes O.
 // Scratch records are column-quad-major, so every scratch access of a warp is coalesced.
 //
 // Roles (384 threads, one CTA per SM):
@@ -28,12 +31,13 @@
 //   warp 1      TMEM owner; lane 0 issues every tcgen05.mma and commit.
 //   warp 2      V producer: V tiles into a three-stage ring. When a segment starts a tile,
 //               the bf16 state copy S_h goes first, through the ring.
+//   warp 3      publisher: raises the flag of each partial record the CTA stores.
 //   warps 4-11  two softmax warpgroups. Thread = query row = TMEM lane; warps 4-7 own
 //               score and output columns 0-63, warps 8-11 columns 64-127. A thread reads
 //               and writes only its own half-row; warps w and w+4 (same rows, same SM
 //               sub-partition) swap half-row maxima through shared memory each tile.
 //               These threads also pack Q' for the readout MMA and write outputs and
-//               partial records.
+//               partial records. Warp 3 stages the records a merge reads.
 // TMEM (512 columns):
 //   - cols 0, 128, 256: three S tiles. The score MMA of tile t+2 is queued right behind
 //     the P.V MMA of tile t and writes the buffer last read two MMA groups earlier, so no
@@ -41,10 +45,14 @@
 //     stalls the tensor pipe). P (bf16) overwrites its own S tile, scores 0-63 packed into
 //     columns 0-31 and scores 64-127 into columns 64-95, and feeds the P.V MMA straight
 //     from TMEM.
-//   - col 384: O. At the start of a segment that starts a tile, it first holds Q' (fp32,
-//     then packed to bf16 for the readout MMA, whose result goes to a free S tile).
+//   - col 384: O.
+//   - Readout, after the last P.V MMA of a segment holding key tile 0: Q' = Q Wq_h goes to
+//     the S tile of tile t0 + n (fp32, then packed in place to bf16 like P), and
+//     O_inter = Q' S_h to the S tile of the segment's last tile. The next segment issues
+//     its first two score tiles into neither of them before its O wait, and its third
+//     (into O_inter's tile) only after that wait.
 // Shared memory: Q | K0 K1 K2 | V0 V1 V2 (32 KiB tiles) from its 1 KiB-aligned base, then a
-// small control block (mbarriers, flags, the row-sum exchange).
+// small control block (mbarriers, flags, the half-row exchange slots).
 //
 // Online softmax: scores are kept in log2 units. The running max m is raised only when a
 // tile's max exceeds it by more than 8 (a factor of 256), so O in TMEM is rescaled rarely.
@@ -62,7 +70,7 @@ namespace {
 constexpr int kStages = 3;      // K and V ring depth
 constexpr int kSBufs = 3;       // score tiles in TMEM
 constexpr int kThreads = 384;
-constexpr int kSoftmaxThreads = 256;
+constexpr int kSoftmaxWarps = 8;   // barriers the softmax threads signal take one arrival per warp
 enum : int {
   kBarQFull = 0,      // Q of a segment landed
   kBarQEmpty = 1,     // the segment's MMAs are done with Q
@@ -71,19 +79,20 @@ enum : int {
   kBarVFull = 8,
   kBarVEmpty = 11,
   kBarSFull = 14,     // +S buffer (3): scores of a tile are in TMEM
-  kBarPFull = 17,     // +S buffer: P written over them (256 arrivals)
+  kBarPFull = 17,     // +S buffer: P written over them (one arrival per softmax warp)
   kBarPVDone = 20,    // +S buffer: the P.V MMA that read P is done
-  kBarQp = 23,        // Q' = Q Wq is in TMEM (O columns)
-  kBarQpReady = 24,   // Q' is packed to bf16 (256 arrivals)
-  kBarOIReady = 25,   // O_inter is in TMEM (a free S buffer)
-  kBarOIFree = 26,    // O_inter was read out (256 arrivals)
-  kBarOFull = 27,     // the segment's MMAs are all done
-  kBarOEmpty = 28,    // the segment's O was read (256 arrivals)
-  kBarFinal = 29,
-  kBarGroup = 30,     // bounded rendezvous of the softmax threads (256 arrivals)
-  kBarPair = 31,      // +row quarter (4): the two warps of those rows swapped half-row maxima
-  kBarNever = 35,     // never signalled: target of the failure-detection test hook
-  kNumBars = 36
+  kBarQp = 23,        // Q' = Q Wq is in TMEM (a free S buffer), at the end of a head segment
+  kBarQpReady = 24,   // Q' is packed to bf16 (per-warp arrivals)
+  kBarOFull = 25,     // the segment's MMAs (its readout included) are all done
+  kBarOEmpty = 26,    // the segment's O and O_inter were read (per-warp arrivals)
+  kBarFinal = 27,
+  kBarGroup = 28,     // bounded rendezvous of the softmax threads (per-warp arrivals)
+  kBarPair = 29,      // +row quarter (4): the two warps of those rows swapped half-row values
+  kBarNever = 33,     // never signalled: target of the failure-detection test hook
+  kBarRec = 34,       // a partial record is stored (per-warp arrivals); warp 3 publishes it
+  kBarRecLoad = 35,   // the merge inputs of the CTA's last segment are staged in shared memory
+  kBarStageGo = 36,   // that segment's MMAs are done: staging may start (per-warp arrivals)
+  kNumBars = 37
 };
 // Tiles at the (1 KiB-aligned) base of dynamic shared memory, then the control block.
 constexpr uint32_t kQOff = 0;
@@ -103,6 +112,14 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 384;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kMaxSegs = 8;                // the host plan keeps segments per query tile at or below this
+// Staging of a merge in the (then idle) tile region: up to three 64 KiB records (partial O
+// of the tile's other segments), then their (m, l) rows, 1 KiB each.
+constexpr uint32_t kStageRecBytes = kRows * kDP * 4;
+constexpr uint32_t kStageMlOff = 3 * kStageRecBytes;
+static_assert(kStageMlOff + (kMaxSegs - 1) * 1024 <= kTileRegion, "merge staging must fit the tile region");
+
+// Whether the head segment of a tile with nsegs segments merges from staged copies.
+__device__ __forceinline__ bool staged_merge(int nsegs) { return nsegs > 1 && nsegs - 1 <= 3; }
 
 struct Smem {
   uint32_t ctl, tiles;
@@ -112,12 +129,53 @@ struct Smem {
   __device__ uint32_t v(int s) const { return tiles + kVOff + s * kTileBytes; }
 };
 
-// Rendezvous of the 256 softmax threads with a bounded wait (no hang if a warp aborted).
+// One arrival for the calling warp, after all of its lanes got here (their earlier
+// memory operations are ordered before it).
+__device__ __forceinline__ void warp_arrive(uint32_t bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
+// Rendezvous of the 8 softmax warps with a bounded wait (no hang if a warp aborted).
 __device__ __forceinline__ bool group_sync(uint32_t bar, uint32_t& phase, const Guard& g) {
-  mbar_arrive(bar);
-  const bool ok = mbar_wait(bar, phase & 1, g);
+  warp_arrive(bar);
+  const bool ok = mbar_wait_warp(bar, phase & 1, g);
   ++phase;
-  return __all_sync(0xffffffffu, ok);
+  return ok;
+}
+
+// The two warps holding the same rows (one per column half) swap one value per row through
+// the exchange slots (double-buffered by exchange count). Returns the half-0 and half-1
+// values in that order, so both warps see identical operands.
+__device__ __forceinline__ bool pair_swap(uint32_t bar, float* xch, uint32_t& nx, int half, uint32_t r, float mine,
+                                          float& v0, float& v1, const Guard& g) {
+  float* xs = xch + (nx & 1) * 256;
+  xs[half * 128 + r] = mine;
+  warp_arrive(bar);
+  const bool ok = mbar_wait_warp(bar, nx & 1, g);
+  ++nx;
+  v0 = xs[r];
+  v1 = xs[128 + r];
+  return ok;
+}
+
+// Acquire load of a flag another CTA publishes, and a bounded wait for a given value.
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ bool wait_flag(const int* f, int value, const Guard& g) {
+  if (ld_acquire_gpu(f) == value) return true;
+  const uint64_t t0 = globaltimer();
+  while (ld_acquire_gpu(f) != value) {
+    if (*g.abort) return false;
+    if (globaltimer() - t0 > g.timeout_ns) {
+      raise_timeout(g);
+      return false;
+    }
+  }
+  return true;
 }
 
 // One segment of a CTA's unit range: key tiles [kb, ke) of query tile Q.
@@ -161,9 +219,9 @@ __device__ __forceinline__ uint32_t ring_phase(uint32_t g) { return (g / kStages
 __device__ __forceinline__ int sbuf(uint32_t t) { return static_cast<int>(t % kSBufs); }
 __device__ __forceinline__ uint32_t sphase(uint32_t t) { return (t / kSBufs) & 1; }
 
-// K producer (kIsK) or V producer. Per segment: [the readout operand (Wq or S) when the
-// segment starts a tile], then its key tiles, all through this producer's ring. The K
-// producer also loads each segment's Q tile.
+// K producer (kIsK) or V producer. Per segment: its key tiles, then, when the segment
+// holds key tile 0 of its query tile, the readout operand (Wq or S), all through this
+// producer's ring. The K producer also loads each segment's Q tile.
 template <bool kHybrid, bool kIsK>
 __device__ void producer(const Smem& sm, const CUtensorMap* tm_q, const CUtensorMap* tm_kv, const CUtensorMap* tm_rd,
                          const QueryArgs& a, const Guard& g, bool lead) {
@@ -187,17 +245,6 @@ __device__ void producer(const Smem& sm, const CUtensorMap* tm_q, const CUtensor
       }
     }
     ++nseg;
-    if (kHybrid && sg.head) {
-      if (!slot_wait(ring)) break;
-      const int s = ring_stage(ring);
-      const int c2 = kIsK ? sg.h : a.state_slot * a.B * a.H + sg.b * a.H + sg.h;
-      if (lead) {
-        mbar_expect_tx(sm.bar(full0 + s), kTileBytes);
-        for (int p = 0; p < 2; ++p) tma_load_3d(tile_addr(s) + p * kPanelBytes, tm_rd, sm.bar(full0 + s), 64 * p, 0, c2);
-      }
-      ++nissued[s];
-      ++ring;
-    }
     for (int j = sg.kb; j < sg.ke; ++j, ++ring) {
       if (!slot_wait(ring)) {
         ok = false;
@@ -210,6 +257,18 @@ __device__ void producer(const Smem& sm, const CUtensorMap* tm_q, const CUtensor
           tma_load_4d(tile_addr(s) + p * kPanelBytes, tm_kv, sm.bar(full0 + s), 64 * p, sg.h, j * kRows, sg.b);
       }
       ++nissued[s];
+    }
+    if (ok && kHybrid && sg.head) {
+      // The readout operand (Wq_h or the bf16 state copy S_h) follows the key tiles.
+      if (!slot_wait(ring)) break;
+      const int s = ring_stage(ring);
+      const int c2 = kIsK ? sg.h : a.state_slot * a.B * a.H + sg.b * a.H + sg.h;
+      if (lead) {
+        mbar_expect_tx(sm.bar(full0 + s), kTileBytes);
+        for (int p = 0; p < 2; ++p) tma_load_3d(tile_addr(s) + p * kPanelBytes, tm_rd, sm.bar(full0 + s), 64 * p, 0, c2);
+      }
+      ++nissued[s];
+      ++ring;
     }
   }
   // Every load issued must land before the CTA may exit (matters only after an abort).
@@ -246,7 +305,7 @@ __device__ void mma_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, co
   while (sch.next(sg)) {
     const bool rd = kHybrid && sg.head;
     const uint32_t t0 = tile, n = sg.ke - sg.kb;
-    const uint32_t r_rd = ring, r0 = ring + (rd ? 1 : 0);   // readout operands' slot, first key tile's slot
+    const uint32_t r0 = ring, r_rd = ring + n;   // first key tile's ring slot, the readout operands' slot
     // Score tiles issued before the P.V loop: two. Afterwards the scores of tile t + 2 are
     // issued right behind the P.V MMA of tile t: they go to the buffer whose P was read by
     // the P.V MMA before that one, so adjacent MMA groups never touch the same TMEM columns
@@ -256,41 +315,11 @@ __device__ void mma_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, co
     tc_fence_after();
     for (uint32_t i = 0; i < npre; ++i)
       if (!issue_qk(t0 + i, r0 + i)) return;
-    // O of the previous segment must have been read before it is rewritten.
+    // O (and the previous segment's O_inter, in the buffer of tile t0 + 2) must have been
+    // read before either is rewritten.
     if (nseg > 0 && !mbar_wait_warp(sm.bar(kBarOEmpty), (nseg - 1) & 1, g)) return;
     tc_fence_after();
-    if (rd) {
-      // Q' = Q Wq_h (phi_q) into the O columns; Wq_h sits in K slot r_rd.
-      const int ws = ring_stage(r_rd);
-      if (!mbar_wait_warp(sm.bar(kBarKFull + ws), ring_phase(r_rd), g)) return;
-      tc_fence_after();
-      if (lead) {
-        mma8_ss<false, true>(tO, desc_kmajor(sm.q(), 0), desc_mnmajor(sm.k(ws), 0), id_kmn, 0u);
-        mma_commit(sm.bar(kBarKEmpty + ws));
-        mma_commit(sm.bar(kBarQp));
-      }
-    }
-    if (lead && n <= npre) mma_commit(sm.bar(kBarQEmpty));
-    if (rd) {
-      // O_inter = Q' S_{N-1}: Q' packed to bf16 in the O columns, S_h in V slot r_rd, the
-      // result in the S buffer of tile t0 + 2 (free until that tile's scores are issued).
-      const int ss = ring_stage(r_rd);
-      if (!mbar_wait_warp(sm.bar(kBarQpReady), nhead & 1, g)) return;
-      if (!mbar_wait_warp(sm.bar(kBarVFull + ss), ring_phase(r_rd), g)) return;
-      tc_fence_after();
-      const uint32_t tX = tmem + 128u * sbuf(t0 + 2);
-      if (lead) {
-        mma8_ts(tX, tO, kPacked, desc_mnmajor(sm.v(ss), 0), id_kmn, 0u);
-        mma_commit(sm.bar(kBarVEmpty + ss));
-        mma_commit(sm.bar(kBarOIReady));
-      }
-      // Whatever tile next scores into that buffer (this segment's or a later one's) must
-      // wait for the read-out. It costs nothing here: the first P.V of the segment needs
-      // the softmax threads, which read O_inter out first.
-      if (!mbar_wait_warp(sm.bar(kBarOIFree), nhead & 1, g)) return;
-      tc_fence_after();
-      ++nhead;
-    }
+    if (lead && !rd && n <= npre) mma_commit(sm.bar(kBarQEmpty));
     const uint32_t nissued = npre;   // score tiles issued ahead of the P.V loop
     for (uint32_t i = 0; i < n; ++i) {
       const uint32_t t = t0 + i, r = r0 + i;
@@ -306,12 +335,36 @@ __device__ void mma_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, co
       }
       if (i + nissued < n) {
         if (!issue_qk(t + nissued, r + nissued)) return;
-        if (lead && i + nissued + 1 == n) mma_commit(sm.bar(kBarQEmpty));
+        if (lead && !rd && i + nissued + 1 == n) mma_commit(sm.bar(kBarQEmpty));
       }
     }
-    if (lead) mma_commit(sm.bar(kBarOFull));
+    if (rd) {
+      // Readout O_inter = (Q Wq_h) S_{N-1}, after the last P.V. Every score buffer is
+      // free: Q' goes to the buffer of tile t0 + n (Y), O_inter to that of the last tile (X,
+      // read by the softmax threads before the next segment's third score tile is issued).
+      const uint32_t tY = tmem + 128u * sbuf(t0 + n), tX = tmem + 128u * sbuf(t0 + n - 1);
+      const int rs = ring_stage(r_rd);
+      if (!mbar_wait_warp(sm.bar(kBarKFull + rs), ring_phase(r_rd), g)) return;
+      tc_fence_after();
+      if (lead) {
+        mma8_ss<false, true>(tY, desc_kmajor(sm.q(), 0), desc_mnmajor(sm.k(rs), 0), id_kmn, 0u);
+        mma_commit(sm.bar(kBarKEmpty + rs));
+        mma_commit(sm.bar(kBarQEmpty));
+        mma_commit(sm.bar(kBarQp));
+      }
+      // Q' packed to bf16 in place by the softmax threads, then O_inter = Q' S_h.
+      if (!mbar_wait_warp(sm.bar(kBarQpReady), nhead & 1, g)) return;
+      if (!mbar_wait_warp(sm.bar(kBarVFull + rs), ring_phase(r_rd), g)) return;
+      tc_fence_after();
+      if (lead) {
+        mma8_ts(tX, tY, kPacked, desc_mnmajor(sm.v(rs), 0), id_kmn, 0u);
+        mma_commit(sm.bar(kBarVEmpty + rs));
+      }
+      ++nhead;
+    }
+    if (lead) mma_commit(sm.bar(kBarOFull));   // every MMA of the segment, the readout included
     tile += n;
-    ring = r0 + n;
+    ring = r0 + n + (rd ? 1u : 0u);
     ++nseg;
   }
 }
@@ -369,155 +422,209 @@ __device__ __forceinline__ float4* quad_ptr(float* base, size_t record, int q, u
   return reinterpret_cast<float4*>(base) + ((record * 32 + q) * kRows + r);
 }
 
-__device__ __forceinline__ uint4 pack8(const float (&y)[8]) {
-  return make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
-                    pack_bf16x2(y[6], y[7]));
-}
-
-// End of a segment: write O (whole query tile), or this segment's partial record and,
-// for the CTA completing the tile, the merge of all its records. O_inter (fp32 scratch,
-// written by the segment that started the tile) is added by whoever finishes the tile.
-// Loads are issued in batches of 16 quads so their latencies overlap. Kept out of line so
-// its registers do not compete with the softmax loop. Returns false if a wait gave up.
+// End of a segment. The segment holding key tile 0 of a query tile (its head) finishes
+// the tile: it combines its own O (TMEM) with the partial records of the tile's other
+// segments, adds O_inter and writes O. With contiguous unit ranges the head segment is
+// the last segment of its CTA and every other segment of the tile starts another CTA's
+// range, so those records are normally published long before. Any other segment stores
+// its partial record (O_acc, running max m, sum l) and the publisher warp raises the
+// record's flag. Loads are issued in batches so their latencies overlap. Kept out of line
+// so its registers do not compete with the softmax loop. Returns false if a wait gave up.
 template <bool kHybrid>
 __device__ __noinline__ bool segment_epilogue(const Smem& sm, const QueryArgs& a, const Seg& sg, uint32_t r, int half,
-                                              int c0, int ncols, uint32_t tO, float m, float l_row,
-                                              uint32_t& gphase, volatile int* merge_flag, const Guard& g) {
-  const int d = a.d;
-  const int q0 = c0 / 4, nquads = ncols / 4;   // this half's column quads
-  const int t_row = sg.qt * kRows + static_cast<int>(r);
-  const bool row_ok = t_row < a.T;
-  uint16_t* out_row = a.o + ((static_cast<size_t>(sg.b) * a.T + t_row) * a.H + sg.h) * d + c0;
-  if (sg.head && sg.tail) {
-    const float inv_l = 1.f / l_row;
-    // Two passes of 8 column quads (32 columns): O_inter loads first, then O from TMEM.
-#pragma unroll
-    for (int hp = 0; hp < 2; ++hp) {
-      if (32 * hp >= ncols) break;
-      float4 oi[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        oi[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (kHybrid && 8 * hp + q < nquads) oi[q] = __ldcg(quad_ptr(a.part_oi, sg.Q, q0 + 8 * hp + q, r));
-      }
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c = 2 * hp + cc;
-        if (16 * c >= ncols) break;
-        uint32_t ov[16];
-        tmem_ld16(tO + c0 + 16u * c, ov);
-        tmem_wait_ld();
-        reg_fence16(ov);
-        if (row_ok) {
-#pragma unroll
-          for (int h8 = 0; h8 < 2; ++h8) {
-            const float4 i0 = oi[4 * cc + 2 * h8], i1 = oi[4 * cc + 2 * h8 + 1];
-            const float y[8] = {__uint_as_float(ov[8 * h8]) * inv_l + i0.x,     __uint_as_float(ov[8 * h8 + 1]) * inv_l + i0.y,
-                                __uint_as_float(ov[8 * h8 + 2]) * inv_l + i0.z, __uint_as_float(ov[8 * h8 + 3]) * inv_l + i0.w,
-                                __uint_as_float(ov[8 * h8 + 4]) * inv_l + i1.x, __uint_as_float(ov[8 * h8 + 5]) * inv_l + i1.y,
-                                __uint_as_float(ov[8 * h8 + 6]) * inv_l + i1.z, __uint_as_float(ov[8 * h8 + 7]) * inv_l + i1.w};
-            reinterpret_cast<uint4*>(out_row + 16 * c)[h8] = pack8(y);
-          }
-        }
-      }
-    }
-    tc_fence_before();
-    mbar_arrive(sm.bar(kBarOEmpty));
-    return true;
-  }
-  // Partial record of this segment: O_acc (coalesced quads), m, l.
+                                              int c0, int ncols, uint32_t tO, uint32_t tX, float m, float l_row,
+                                              uint32_t& gphase, volatile int* merge_ok, const float* stage,
+                                              const Guard& g) {
+  const int q0 = c0 / 4;   // this half's first column quad
   const long long first = static_cast<long long>(sg.Q) * a.nkv;
   const int c_first = owner(first, a);
-  const int nsegs = owner(first + a.nkv - 1, a) - c_first + 1;
   const size_t slot0 = static_cast<size_t>(sg.Q) * a.max_segs;
-  const size_t slot = slot0 + (static_cast<int>(blockIdx.x) - c_first);
+  if (!sg.head) {
+    const size_t slot = slot0 + (static_cast<int>(blockIdx.x) - c_first);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (16 * c >= ncols) break;
+      uint32_t ov[16];
+      tmem_ld16(tO + c0 + 16u * c, ov);
+      tmem_wait_ld();
+      reg_fence16(ov);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        *quad_ptr(a.part_o, slot, q0 + 4 * c + q, r) =
+            make_float4(__uint_as_float(ov[4 * q]), __uint_as_float(ov[4 * q + 1]), __uint_as_float(ov[4 * q + 2]),
+                        __uint_as_float(ov[4 * q + 3]));
+    }
+    if (half == 0) {
+      a.part_ml[(slot * 2) * kRows + r] = m;
+      a.part_ml[(slot * 2 + 1) * kRows + r] = l_row;
+    }
+    tc_fence_before();
+    warp_arrive(sm.bar(kBarOEmpty));   // TMEM read: the next segment may reuse O
+    warp_arrive(sm.bar(kBarRec));      // record stored: the publisher may raise its flag
+    return true;
+  }
+  // Head segment: the tile's other records (if any), then the merge. Warp 3 stages them
+  // in shared memory when they fit; otherwise they are read from scratch here.
+  const int nsegs = sg.tail ? 1 : owner(first + a.nkv - 1, a) - c_first + 1;
+  const bool staged = staged_merge(nsegs);
+  const float4* st4 = reinterpret_cast<const float4*>(stage);
+  if (staged) {
+    // Every MMA of the segment is done (OFull): warp 3 may overwrite the tile region. At
+    // most one staged merge per CTA and launch, so both barriers complete once (phase 0).
+    warp_arrive(sm.bar(kBarStageGo));
+    if (!mbar_wait_warp(sm.bar(kBarRecLoad), 0, g)) return false;
+  } else if (nsegs > 1) {
+    if (half == 0 && r == 0) {
+      bool ok = true;
+      for (int s = 1; s < nsegs && ok; ++s) ok = wait_flag(a.flags + slot0 + s, a.epoch, g);
+      *merge_ok = ok ? 1 : 0;
+    }
+    if (!group_sync(sm.bar(kBarGroup), gphase, g)) return false;
+    if (!*merge_ok) return false;
+  }
+  auto rec_m = [&](int s) {
+    return staged ? stage[kStageMlOff / 4 + (s - 1) * 256 + r] : __ldcg(a.part_ml + ((slot0 + s) * 2) * kRows + r);
+  };
+  auto rec_l = [&](int s) {
+    return staged ? stage[kStageMlOff / 4 + (s - 1) * 256 + 128 + r]
+                  : __ldcg(a.part_ml + ((slot0 + s) * 2 + 1) * kRows + r);
+  };
+  auto rec_o = [&](int s, int q) {
+    return staged ? st4[(s - 1) * (kStageRecBytes / 16) + q * kRows + r] : __ldcg(quad_ptr(a.part_o, slot0 + s, q, r));
+  };
+  float ws[kMaxSegs];
+  float M = m;
+#pragma unroll
+  for (int s = 1; s < kMaxSegs; ++s) {
+    if (s < nsegs) {
+      ws[s] = rec_m(s);
+      M = fmaxf(M, ws[s]);
+    }
+  }
+  const float w_own = ex2_approx(m - M);
+  float L = w_own * l_row;
+#pragma unroll
+  for (int s = 1; s < kMaxSegs; ++s) {
+    if (s < nsegs) {
+      ws[s] = ex2_approx(ws[s] - M);
+      L += ws[s] * rec_l(s);
+    }
+  }
+  const float inv_L = 1.f / L;
+  const int t_row = sg.qt * kRows + static_cast<int>(r);
+  const bool row_ok = t_row < a.T;
+  uint16_t* out_row = a.o + ((static_cast<size_t>(sg.b) * a.T + t_row) * a.H + sg.h) * a.d + c0;
+  // Four passes of 16 columns: the TMEM loads (O, and O_inter for the layer) are issued
+  // first, the other records are read while they are in flight.
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     if (16 * c >= ncols) break;
-    uint32_t ov[16];
+    uint32_t ov[16], xv[16];
     tmem_ld16(tO + c0 + 16u * c, ov);
-    tmem_wait_ld();
-    reg_fence16(ov);
+    if (kHybrid) tmem_ld16(tX + c0 + 16u * c, xv);
+    float4 acc[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      *quad_ptr(a.part_o, slot, q0 + 4 * c + q, r) =
-          make_float4(__uint_as_float(ov[4 * q]), __uint_as_float(ov[4 * q + 1]), __uint_as_float(ov[4 * q + 2]),
-                      __uint_as_float(ov[4 * q + 3]));
-  }
-  if (half == 0) {
-    a.part_ml[(slot * 2) * kRows + r] = m;
-    a.part_ml[(slot * 2 + 1) * kRows + r] = l_row;
-  }
-  // TMEM is read: the next segment's MMAs may reuse O.
-  tc_fence_before();
-  mbar_arrive(sm.bar(kBarOEmpty));
-  // Publish, then count this segment in; the CTA completing the count merges.
-  __threadfence();
-  if (!group_sync(sm.bar(kBarGroup), gphase, g)) return false;
-  if (half == 0 && r == 0) {
-    const int prev = atomicAdd(a.cnt + sg.Q, 1);
-    *merge_flag = (prev == nsegs - 1) ? 1 : 0;
-  }
-  if (!group_sync(sm.bar(kBarGroup), gphase, g)) return false;
-  if (!*merge_flag) return true;
-  __threadfence();
-  float ms[kMaxSegs], ls[kMaxSegs];
-  float M = -INFINITY;
+    for (int q = 0; q < 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-  for (int s = 0; s < kMaxSegs; ++s) {
-    if (s < nsegs) {
-      ms[s] = __ldcg(a.part_ml + ((slot0 + s) * 2) * kRows + r);
-      ls[s] = __ldcg(a.part_ml + ((slot0 + s) * 2 + 1) * kRows + r);
-      M = fmaxf(M, ms[s]);
-    }
-  }
-  float L = 0.f;
-#pragma unroll
-  for (int s = 0; s < kMaxSegs; ++s)
-    if (s < nsegs) L += ex2_approx(ms[s] - M) * ls[s];
-  const float inv_L = 1.f / L;
-  // Two passes of 8 column quads; each pass issues one segment's 8 loads at a time.
-#pragma unroll
-  for (int hp = 0; hp < 2; ++hp) {
-    if (32 * hp >= ncols) break;
-    float4 acc[8], oi[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-      oi[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (kHybrid && 8 * hp + q < nquads) oi[q] = __ldcg(quad_ptr(a.part_oi, sg.Q, q0 + 8 * hp + q, r));
-    }
-#pragma unroll
-    for (int s = 0; s < kMaxSegs; ++s) {
+    for (int s = 1; s < kMaxSegs; ++s) {
       if (s < nsegs) {
-        const float w = ex2_approx(ms[s] - M);
-        float4 v[8];
+        float4 v[4];
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          v[q] = (8 * hp + q < nquads) ? __ldcg(quad_ptr(a.part_o, slot0 + s, q0 + 8 * hp + q, r))
-                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int q = 0; q < 4; ++q) v[q] = rec_o(s, q0 + 4 * c + q);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          acc[q].x += w * v[q].x;
-          acc[q].y += w * v[q].y;
-          acc[q].z += w * v[q].z;
-          acc[q].w += w * v[q].w;
+        for (int q = 0; q < 4; ++q) {
+          acc[q].x += ws[s] * v[q].x;
+          acc[q].y += ws[s] * v[q].y;
+          acc[q].z += ws[s] * v[q].z;
+          acc[q].w += ws[s] * v[q].w;
         }
       }
     }
-    if (row_ok) {
+    tmem_wait_ld();
+    reg_fence16(ov);
+    if (kHybrid) reg_fence16(xv);
+    float y[16];
 #pragma unroll
-      for (int h8 = 0; h8 < 4; ++h8) {
-        if (32 * hp + 8 * h8 >= ncols) break;
-        const float4 a0 = acc[2 * h8], a1 = acc[2 * h8 + 1], i0 = oi[2 * h8], i1 = oi[2 * h8 + 1];
-        const float y[8] = {a0.x * inv_L + i0.x, a0.y * inv_L + i0.y, a0.z * inv_L + i0.z, a0.w * inv_L + i0.w,
-                            a1.x * inv_L + i1.x, a1.y * inv_L + i1.y, a1.z * inv_L + i1.z, a1.w * inv_L + i1.w};
-        reinterpret_cast<uint4*>(out_row + 32 * hp)[h8] = pack8(y);
+    for (int q = 0; q < 4; ++q) {
+      y[4 * q] = (acc[q].x + w_own * __uint_as_float(ov[4 * q])) * inv_L;
+      y[4 * q + 1] = (acc[q].y + w_own * __uint_as_float(ov[4 * q + 1])) * inv_L;
+      y[4 * q + 2] = (acc[q].z + w_own * __uint_as_float(ov[4 * q + 2])) * inv_L;
+      y[4 * q + 3] = (acc[q].w + w_own * __uint_as_float(ov[4 * q + 3])) * inv_L;
+    }
+    if (kHybrid) {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) y[e] += __uint_as_float(xv[e]);
+    }
+    if (row_ok) {
+      uint4* dst = reinterpret_cast<uint4*>(out_row + 16 * c);
+      dst[0] = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                          pack_bf16x2(y[6], y[7]));
+      dst[1] = make_uint4(pack_bf16x2(y[8], y[9]), pack_bf16x2(y[10], y[11]), pack_bf16x2(y[12], y[13]),
+                          pack_bf16x2(y[14], y[15]));
+    }
+  }
+  tc_fence_before();
+  warp_arrive(sm.bar(kBarOEmpty));
+  return true;
+}
+
+// Warp 3. (1) Raises the flag of each partial record this CTA stores, once the softmax
+// warps have stored it: their CTA-scope arrival orders those stores before this warp's
+// device-scope fence, so a CTA that reads the flag (acquire) sees the whole record.
+// (2) For a head segment that merges from staged copies (always the CTA's last segment):
+// waits for the other records' flags while the segment runs, then, once the softmax warps
+// report its MMAs done (the tile region idle), bulk-copies those records, their (m, l)
+// rows and O_inter into shared memory. Every barrier this warp waits on completes at most
+// once per launch, so a parity wait can never alias an earlier phase.
+template <bool kHybrid>
+__device__ void publisher(const Smem& sm, const QueryArgs& a, const Guard& g) {
+  const bool lead = (threadIdx.x & 31) == 0;
+  uint32_t nrec = 0;   // a CTA stores at most one record (only its first segment can lack key tile 0)
+  bool staged_issued = false;
+  Sched sch(a, blockIdx.x);
+  Seg sg;
+  while (sch.next(sg)) {
+    const long long first = static_cast<long long>(sg.Q) * a.nkv;
+    const int c_first = owner(first, a);
+    const size_t slot0 = static_cast<size_t>(sg.Q) * a.max_segs;
+    if (!sg.head) {
+      if (!mbar_wait_warp(sm.bar(kBarRec), nrec & 1, g)) break;
+      ++nrec;
+      if (lead) {
+        __threadfence();
+        atomicExch(a.flags + slot0 + (static_cast<int>(blockIdx.x) - c_first), a.epoch);
+      }
+      __syncwarp();
+    } else {
+      const int nsegs = sg.tail ? 1 : owner(first + a.nkv - 1, a) - c_first + 1;
+      if (staged_merge(nsegs)) {
+        bool ok = true;
+        if (lead)
+          for (int s = 1; s < nsegs && ok; ++s) ok = wait_flag(a.flags + slot0 + s, a.epoch, g);
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        // The softmax warps signal that the segment's MMAs are done (nothing reads the tile
+        // region any more) and that O_inter, stored at the segment's start, is ordered
+        // before this point. This is the CTA's last segment: one phase per launch.
+        if (!mbar_wait_warp(sm.bar(kBarStageGo), 0, g)) break;
+        if (lead) {
+          const uint32_t rec_bytes = static_cast<uint32_t>(a.d) * kRows * 4;   // d/4 column quads
+          const uint32_t nrecs = static_cast<uint32_t>(nsegs - 1);
+          fence_proxy_async_global();
+          mbar_expect_tx(sm.bar(kBarRecLoad), nrecs * (rec_bytes + 1024u));
+          for (int s = 1; s < nsegs; ++s) {
+            bulk_load(sm.tiles + (s - 1) * kStageRecBytes, a.part_o + (slot0 + s) * kRows * kDP, rec_bytes,
+                      sm.bar(kBarRecLoad));
+            bulk_load(sm.tiles + kStageMlOff + (s - 1) * 1024u, a.part_ml + (slot0 + s) * 2 * kRows, 1024u,
+                      sm.bar(kBarRecLoad));
+          }
+          }
+        staged_issued = true;
+        __syncwarp();
       }
     }
   }
-  if (half == 0 && r == 0) a.cnt[sg.Q] = 0;   // ready for the next launch
-  return true;
+  // Copies into shared memory must land before the CTA exits (matters only after an abort).
+  if (staged_issued) mbar_wait_drain(sm.bar(kBarRecLoad), 0);
 }
 
 template <bool kHybrid>
@@ -529,65 +636,18 @@ __device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const 
   const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
   const uint32_t tO = tmem + lane_off + kColO;
   float* xch = reinterpret_cast<float*>(ctl + kCtlX);      // [2 slots][2 halves][128]
-  volatile int* merge_flag = reinterpret_cast<volatile int*>(ctl + kCtlMisc + 8);
+  volatile int* merge_ok = reinterpret_cast<volatile int*>(ctl + kCtlMisc + 8);
+  const uint32_t pair_bar = sm.bar(kBarPair + quarter);
   const int d = a.d;
   const int c0 = 64 * half;                                 // first column of this thread's half
-  const int oc = 64 - c0;                                   // first column of the other half
   const int ncols = max(0, min(64, d - c0));                // output columns of this half
-  uint32_t nseg = 0, nhead = 0, tile = 0, gphase = 0;
+  uint32_t nseg = 0, nhead = 0, tile = 0, gphase = 0, nx = 0;
   // Test hook: a wait that can only run out (the bounded-wait path, without a fault).
   if (a.stall && !mbar_wait_warp(sm.bar(kBarNever), 0, g)) return;
   Sched sch(a, blockIdx.x);
   Seg sg;
   while (sch.next(sg)) {
     const uint32_t t0 = tile, n = sg.ke - sg.kb;
-    if (kHybrid && sg.head) {
-      // Q' (fp32, O columns) -> bf16 pairs over this half's own O columns: the readout
-      // MMA's A operand.
-      if (!mbar_wait_warp(sm.bar(kBarQp), nhead & 1, g)) return;
-      tc_fence_after();
-      {
-        uint32_t x0[32], x1[32], pk[32];
-        tmem_ld32(tO + c0, x0);
-        tmem_ld32(tO + c0 + 32, x1);
-        tmem_wait_ld();
-        reg_fence(x0);
-        reg_fence(x1);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          pk[i] = pack_bf16x2(__uint_as_float(x0[2 * i]), __uint_as_float(x0[2 * i + 1]));
-          pk[16 + i] = pack_bf16x2(__uint_as_float(x1[2 * i]), __uint_as_float(x1[2 * i + 1]));
-        }
-        tmem_st32(tO + c0, pk);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(sm.bar(kBarQpReady));
-      // O_inter (fp32, the S buffer of tile t0 + 2) -> this half's quads of the tile's
-      // O_inter record in scratch.
-      if (!mbar_wait_warp(sm.bar(kBarOIReady), nhead & 1, g)) return;
-      tc_fence_after();
-      {
-        const uint32_t tX = tmem + lane_off + 128u * sbuf(t0 + 2);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (16 * c >= ncols) break;
-          uint32_t x[16];
-          tmem_ld16(tX + c0 + 16u * c, x);
-          tmem_wait_ld();
-          reg_fence16(x);
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            *quad_ptr(a.part_oi, sg.Q, c0 / 4 + 4 * c + q, r) =
-                make_float4(__uint_as_float(x[4 * q]), __uint_as_float(x[4 * q + 1]), __uint_as_float(x[4 * q + 2]),
-                            __uint_as_float(x[4 * q + 3]));
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(sm.bar(kBarOIFree));
-      ++nhead;
-    }
-
     float m = -INFINITY, l = 0.f;
     for (uint32_t i = 0; i < n; ++i) {
       const uint32_t t = t0 + i;
@@ -597,20 +657,16 @@ __device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const 
       const uint32_t tS = tmem + lane_off + 128u * sb;
       const int valid = a.kv_len - (sg.kb + static_cast<int>(i)) * kRows;   // >= 1
       // This half's scores, then the row max: the two warps holding these rows (one per
-      // half) swap their half-row maxima through shared memory, double-buffered by tile
-      // parity. Each half reads and writes only its own columns.
+      // half) swap their half-row maxima. Each half reads and writes only its own columns.
       uint32_t sv[2][32];
       tmem_ld32(tS + c0, sv[0]);
       tmem_ld32(tS + c0 + 32, sv[1]);
       tmem_wait_ld();
       reg_fence(sv[0]);
       reg_fence(sv[1]);
-      float* xm = xch + (t & 1) * 256;
-      xm[half * 128 + r] = half_max(sv, c0, valid);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(sm.bar(kBarPair + quarter));
-      if (!mbar_wait_warp(sm.bar(kBarPair + quarter), t & 1, g)) return;
-      const float mt = fmaxf(xm[r], xm[128 + r]) * a.scale_log2;
+      float h0, h1;
+      if (!pair_swap(pair_bar, xch, nx, half, r, half_max(sv, c0, valid), h0, h1, g)) return;
+      const float mt = fmaxf(h0, h1) * a.scale_log2;
       float m_new = m;
       bool rescale = false;
       if (i == 0) {
@@ -625,14 +681,14 @@ __device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const 
         tc_fence_after();
         const float corr = rescale ? ex2_approx(m - m_new) : 1.f;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t ov[32];
-          tmem_ld32(tO + c0 + 32u * c, ov);
+        for (int c = 0; c < 4; ++c) {
+          uint32_t ov[16];
+          tmem_ld16(tO + c0 + 16u * c, ov);
           tmem_wait_ld();
-          reg_fence(ov);
+          reg_fence16(ov);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
-          tmem_st32(tO + c0 + 32u * c, ov);
+          for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
+          tmem_st16(tO + c0 + 16u * c, ov);
         }
         l *= corr;
       }
@@ -643,18 +699,48 @@ __device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const 
       tmem_st32(tS + c0, pk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(sm.bar(kBarPFull + sb));
+      warp_arrive(sm.bar(kBarPFull + sb));
     }
     tile += n;
 
-    // ---- end of segment: every MMA of it is done; combine the two half-row sums.
+    // ---- end of segment. A segment holding key tile 0 computes the readout here: Q' =
+    // Q Wq_h arrives (fp32) in the S buffer of tile t0 + n; each half packs its own 64
+    // columns to bf16 pairs in place (the readout MMA's A operand, same layout as P).
+    const uint32_t tX = tmem + lane_off + 128u * sbuf(t0 + n - 1);   // O_inter, when computed
+    if (kHybrid && sg.head) {
+      const uint32_t tY = tmem + lane_off + 128u * sbuf(t0 + n);
+      if (!mbar_wait_warp(sm.bar(kBarQp), nhead & 1, g)) return;
+      tc_fence_after();
+      // Two rounds of 32 columns; round h packs into columns c0 + 16h .. c0 + 16h + 15,
+      // which round h has already read (round 1 writes only what round 0 read).
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t x0[16], x1[16], pk[16];
+        tmem_ld16(tY + c0 + 32u * h, x0);
+        tmem_ld16(tY + c0 + 32u * h + 16u, x1);
+        tmem_wait_ld();
+        reg_fence16(x0);
+        reg_fence16(x1);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          pk[i] = pack_bf16x2(__uint_as_float(x0[2 * i]), __uint_as_float(x0[2 * i + 1]));
+          pk[8 + i] = pack_bf16x2(__uint_as_float(x1[2 * i]), __uint_as_float(x1[2 * i + 1]));
+        }
+        tmem_st16(tY + c0 + 16u * h, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      warp_arrive(sm.bar(kBarQpReady));
+      ++nhead;
+    }
+    // Every MMA of the segment (the readout included) is done; combine the half-row sums.
     if (!mbar_wait_warp(sm.bar(kBarOFull), nseg & 1, g)) return;
     tc_fence_after();
-    xch[half * 128 + r] = l;
-    if (!group_sync(sm.bar(kBarGroup), gphase, g)) return;
-    const float l_row = xch[r] + xch[128 + r];
-    if (!group_sync(sm.bar(kBarGroup), gphase, g)) return;   // before anyone rewrites xch
-    if (!segment_epilogue<kHybrid>(sm, a, sg, r, half, c0, ncols, tO, m, l_row, gphase, merge_flag, g)) return;
+    float l0, l1;
+    if (!pair_swap(pair_bar, xch, nx, half, r, l, l0, l1, g)) return;
+    if (!segment_epilogue<kHybrid>(sm, a, sg, r, half, c0, ncols, tO, tX, m, l0 + l1, gphase, merge_ok,
+                                   reinterpret_cast<const float*>(ctl - kTileRegion), g))
+      return;
     ++nseg;
   }
 }
@@ -689,19 +775,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < kSBufs; ++s) {
       mbar_init(sm.bar(kBarSFull + s), 1);
-      mbar_init(sm.bar(kBarPFull + s), kSoftmaxThreads);
+      mbar_init(sm.bar(kBarPFull + s), kSoftmaxWarps);
       mbar_init(sm.bar(kBarPVDone + s), 1);
     }
     mbar_init(sm.bar(kBarQp), 1);
-    mbar_init(sm.bar(kBarQpReady), kSoftmaxThreads);
-    mbar_init(sm.bar(kBarOIReady), 1);
-    mbar_init(sm.bar(kBarOIFree), kSoftmaxThreads);
+    mbar_init(sm.bar(kBarQpReady), kSoftmaxWarps);
     mbar_init(sm.bar(kBarOFull), 1);
-    mbar_init(sm.bar(kBarOEmpty), kSoftmaxThreads);
+    mbar_init(sm.bar(kBarOEmpty), kSoftmaxWarps);
     mbar_init(sm.bar(kBarFinal), 1);
-    mbar_init(sm.bar(kBarGroup), kSoftmaxThreads);
+    mbar_init(sm.bar(kBarGroup), kSoftmaxWarps);
     for (int q = 0; q < 4; ++q) mbar_init(sm.bar(kBarPair + q), 2);   // one arrival per warp
     mbar_init(sm.bar(kBarNever), 1);
+    mbar_init(sm.bar(kBarRec), kSoftmaxWarps);
+    mbar_init(sm.bar(kBarRecLoad), 1);
+    mbar_init(sm.bar(kBarStageGo), kSoftmaxWarps);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -731,6 +818,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 2) {
     producer<kHybrid, false>(sm, &tm_q, &tm_v, &tm_s, a, g, elect_one());
+  } else if (warp == 3) {
+    publisher<kHybrid>(sm, a, g);
   } else if (warp >= 4) {
     softmax_role<kHybrid>(sm, ctl_ptr, tmem, a, warp, lane, g);
   }
@@ -783,9 +872,11 @@ QueryPlan plan_query(int B, int H, int T, int kv_len, int num_sms) {
   return p;
 }
 
+size_t query_flag_count(const QueryPlan& p) { return static_cast<size_t>(p.qtiles) * p.max_segs; }
+
 size_t query_scratch_floats(const QueryPlan& p) {
   const size_t slots = static_cast<size_t>(p.qtiles) * p.max_segs;
-  return slots * kRows * kDP + slots * 2 * kRows + static_cast<size_t>(p.qtiles) * kRows * kDP;
+  return slots * kRows * kDP + slots * 2 * kRows;
 }
 
 cudaError_t launch_query(bool hybrid, const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
