@@ -44,11 +44,12 @@ bool make_map(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims,
   return r == CUDA_SUCCESS;
 }
 
-// [B, L, H, d] token-major activations: dims (d, H, L, B), box (64, 1, 128, 1).
-bool make_act_map(CUtensorMap* m, const void* ptr, int B, int L, int H, int d) {
+// [B, L, H, d] token-major activations: dims (d, H, L, B), box (64, 1, rows, 1); loads use
+// 128-row boxes, the query's output stores 32-row boxes (one per warp).
+bool make_act_map(CUtensorMap* m, const void* ptr, int B, int L, int H, int d, int rows = 128) {
   const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)B};
   const cuuint64_t str[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)L * H * d * 2};
-  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
   return make_map(m, ptr, 4, dims, str, box);
 }
 
@@ -65,7 +66,8 @@ bool aligned4(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 3u)
 
 // Small cache of activation maps keyed by base pointer: callers usually reuse buffers.
 struct MapCache {
-  static constexpr int kSlots = 16;
+  static constexpr int kSlots = 64;
+  int rows = 128;                 // box rows of the maps this cache makes
   const void* ptr[kSlots] = {};
   CUtensorMap map[kSlots];
   int next = 0;
@@ -75,7 +77,7 @@ struct MapCache {
     const int i = next;
     next = (next + 1) % kSlots;
     ptr[i] = nullptr;
-    if (!make_act_map(&map[i], p, B, L, H, d)) return nullptr;
+    if (!make_act_map(&map[i], p, B, L, H, d, rows)) return nullptr;
     ptr[i] = p;
     return &map[i];
   }
@@ -143,6 +145,7 @@ struct arl2_ctx {
   CUtensorMap tm_w[3];
   CUtensorMap tm_s;
   MapCache acts;
+  MapCache outs{32};              // output maps (32-row store boxes)
   size_t bytes = 0;
 
   size_t act_elems() const { return (size_t)B * T * H * d; }
@@ -158,6 +161,7 @@ struct arl2_kvcache {
   unsigned int* err = nullptr;
   CUtensorMap tm_k, tm_v;
   MapCache acts;
+  MapCache outs{32};
   size_t bytes = 0;
   unsigned long long timeout_ns = kDefaultTimeoutNs;
   int num_sms = 0;
@@ -219,7 +223,8 @@ arl2_status query_impl(arl2_ctx* c, const void* q, const void* k, const void* v,
   const CUtensorMap* mq = c->acts.get(q, c->B, c->T, c->H, c->d);
   const CUtensorMap* mk = c->acts.get(k, c->B, c->T, c->H, c->d);
   const CUtensorMap* mv = c->acts.get(v, c->B, c->T, c->H, c->d);
-  if (!mq || !mk || !mv) return ARL2_ERR_CUDA;
+  const CUtensorMap* mo = c->outs.get(o, c->B, c->T, c->H, c->d);
+  if (!mq || !mk || !mv || !mo) return ARL2_ERR_CUDA;
   arl2::QueryArgs a{};
   a.o = static_cast<uint16_t*>(o);
   a.T = c->T;
@@ -234,8 +239,8 @@ arl2_status query_impl(arl2_ctx* c, const void* q, const void* k, const void* v,
   a.stall = c->stall_next ? 1 : 0;
   c->stall_next = false;
   set_plan(&a, c->qplan, c->qscratch, c->qflags, next_epoch(&c->qepoch));
-  return arl2::launch_query(true, *mq, *mk, *mv, c->tm_w[0], c->tm_s, a, st) == cudaSuccess ? ARL2_OK
-                                                                                           : ARL2_ERR_CUDA;
+  return arl2::launch_query(true, *mq, *mk, *mv, c->tm_w[0], c->tm_s, *mo, a, st) == cudaSuccess ? ARL2_OK
+                                                                                                : ARL2_ERR_CUDA;
 }
 
 arl2_status commit_impl(arl2_ctx* c, const void* k, const void* v, const float* alpha, const float* beta,
@@ -519,7 +524,8 @@ arl2_status arl2_kvcache_query(arl2_kvcache* c, const arl2_bf16* q, const arl2_b
   arl2_status s = kv_write_slot(c, k, v, st);
   if (s != ARL2_OK) return s;
   const CUtensorMap* mq = c->acts.get(q, c->B, c->T, c->H, c->d);
-  if (!mq) return ARL2_ERR_CUDA;
+  const CUtensorMap* mo = c->outs.get(o, c->B, c->T, c->H, c->d);
+  if (!mq || !mo) return ARL2_ERR_CUDA;
   arl2::QueryArgs a{};
   a.o = o;
   a.T = c->T;
@@ -533,8 +539,9 @@ arl2_status arl2_kvcache_query(arl2_kvcache* c, const arl2_bf16* q, const arl2_b
   a.timeout_ns = c->timeout_ns;
   set_plan(&a, arl2::plan_query(c->B, c->H, c->T, a.kv_len, c->num_sms), c->qscratch, c->qflags,
            next_epoch(&c->qepoch));
-  return arl2::launch_query(false, *mq, c->tm_k, c->tm_v, c->tm_k, c->tm_k, a, st) == cudaSuccess ? ARL2_OK
-                                                                                                  : ARL2_ERR_CUDA;
+  return arl2::launch_query(false, *mq, c->tm_k, c->tm_v, c->tm_k, c->tm_k, *mo, a, st) == cudaSuccess
+             ? ARL2_OK
+             : ARL2_ERR_CUDA;
 }
 
 arl2_status arl2_kvcache_commit(arl2_kvcache* c, const arl2_bf16* k, const arl2_bf16* v, arl2_stream stream) {

@@ -80,7 +80,8 @@ cudaError_t query_setup();   // per-device function attributes
 cudaError_t commit_setup();
 
 cudaError_t launch_query(bool hybrid, const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                         const CUtensorMap& tm_w, const CUtensorMap& tm_s, const QueryArgs& a, cudaStream_t stream);
+                         const CUtensorMap& tm_w, const CUtensorMap& tm_s, const CUtensorMap& tm_o, const QueryArgs& a,
+                         cudaStream_t stream);
 cudaError_t launch_commit(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const CUtensorMap& tm_wk,
                           const CUtensorMap& tm_wv, const CUtensorMap& tm_s, const CommitArgs& a,
                           const ReduceArgs& r, cudaStream_t stream);

@@ -91,8 +91,9 @@ enum : int {
   kBarNever = 33,     // never signalled: target of the failure-detection test hook
   kBarRec = 34,       // a partial record is stored (per-warp arrivals); warp 3 publishes it
   kBarRecLoad = 35,   // the merge inputs of the CTA's last segment are staged in shared memory
-  kBarStageGo = 36,   // that segment's MMAs are done: staging may start (per-warp arrivals)
-  kNumBars = 37
+  kBarLastPV = 36,    // the last P.V MMA of a staged merge's segment is done (V stages idle)
+  kBarLastQK = 37,    // its last score MMA is done (K stages idle): staging may start
+  kNumBars = 38
 };
 // Tiles at the (1 KiB-aligned) base of dynamic shared memory, then the control block.
 constexpr uint32_t kQOff = 0;
@@ -112,14 +113,14 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 384;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kMaxSegs = 8;                // the host plan keeps segments per query tile at or below this
-// Staging of a merge in the (then idle) tile region: up to three 64 KiB records (partial O
-// of the tile's other segments), then their (m, l) rows, 1 KiB each.
-constexpr uint32_t kStageRecBytes = kRows * kDP * 4;
-constexpr uint32_t kStageMlOff = 3 * kStageRecBytes;
-static_assert(kStageMlOff + (kMaxSegs - 1) * 1024 <= kTileRegion, "merge staging must fit the tile region");
-
-// Whether the head segment of a tile with nsegs segments merges from staged copies.
-__device__ __forceinline__ bool staged_merge(int nsegs) { return nsegs > 1 && nsegs - 1 <= 3; }
+// Staged merge: a query tile split in two segments is finished by its head segment (the
+// CTA's last) from a shared-memory copy of the other record, taken while the head's last
+// tiles are still in flight. The readout still reads Q, and Wq_h and S_h in ring stage ws of
+// the K and V rings; the other stages are idle:
+//   K stage ws+1: record column quads 0-15 (32 KiB)   K stage ws+2: quads 16-31
+//   V stage ws+1: the record's m and l rows (1 KiB)   V stage ws+2: the bf16 output tile,
+//                                                     stored by TMA (two swizzled panels)
+__device__ __forceinline__ bool staged_merge(int nsegs) { return nsegs == 2; }
 
 struct Smem {
   uint32_t ctl, tiles;
@@ -183,6 +184,7 @@ struct Seg {
   int Q, kb, ke;
   int b, h, qt;
   bool head, tail;
+  bool last;   // the CTA's last segment
 };
 
 struct Sched {
@@ -204,6 +206,7 @@ struct Sched {
     s.h = bh % H;
     s.head = s.kb == 0;
     s.tail = s.ke == nkv;
+    s.last = u >= u1;
     return true;
   }
 };
@@ -217,6 +220,13 @@ __device__ __forceinline__ int owner(long long u, const QueryArgs& a) {
 __device__ __forceinline__ int ring_stage(uint32_t g) { return static_cast<int>(g % kStages); }
 __device__ __forceinline__ uint32_t ring_phase(uint32_t g) { return (g / kStages) & 1; }
 __device__ __forceinline__ int sbuf(uint32_t t) { return static_cast<int>(t % kSBufs); }
+// S buffer that receives O_inter of a head segment (tiles t0 .. t0+n-1). In the CTA's last
+// segment: that of tile t0+n-2, whose P.V MMA is not the one just ahead, so the readout
+// does not wait for the last P.V to finish reading. Otherwise that of the last tile, which
+// the next segment rewrites only with its third score tile, after its O wait.
+__device__ __forceinline__ int o_inter_tile(uint32_t t0, uint32_t n, bool last) {
+  return sbuf(last ? t0 + n + 1 : t0 + n - 1);
+}
 __device__ __forceinline__ uint32_t sphase(uint32_t t) { return (t / kSBufs) & 1; }
 
 // K producer (kIsK) or V producer. Per segment: its key tiles, then, when the segment
@@ -246,6 +256,13 @@ __device__ void producer(const Smem& sm, const CUtensorMap* tm_q, const CUtensor
     }
     ++nseg;
     for (int j = sg.kb; j < sg.ke; ++j, ++ring) {
+      // Start-up order: the first Q tile and first K tile go out alone (they gate the
+      // first score MMA); the rest of both rings fills once that K tile has landed. The
+      // first fill of K stage 0 is phase 0 of its barrier, waited on from the start.
+      if (ring == (kIsK ? 1u : 0u) && !mbar_wait_warp(sm.bar(kBarKFull), 0, g)) {
+        ok = false;
+        break;
+      }
       if (!slot_wait(ring)) {
         ok = false;
         break;
@@ -302,9 +319,31 @@ __device__ void mma_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, co
     }
     return true;
   };
+  // First readout MMA, Q' = Q Wq_h into the S buffer of tile t0 + n (Y). Issued right
+  // after the segment's last score MMA (never before the O wait, as Y may be the buffer
+  // of the previous segment's O_inter): Y last held tile t0 + n - 3, whose P.V MMA is
+  // already queued, and Q is free once this MMA is done.
+  auto issue_qwq = [&](uint32_t t0, uint32_t n, uint32_t r_rd) -> bool {
+    const int rs = ring_stage(r_rd);
+    if (!mbar_wait_warp(sm.bar(kBarKFull + rs), ring_phase(r_rd), g)) return false;
+    tc_fence_after();
+    if (lead) {
+      mma8_ss<false, true>(tmem + 128u * sbuf(t0 + n), desc_kmajor(sm.q(), 0), desc_mnmajor(sm.k(rs), 0), id_kmn,
+                           0u);
+      mma_commit(sm.bar(kBarKEmpty + rs));
+      mma_commit(sm.bar(kBarQEmpty));
+      mma_commit(sm.bar(kBarQp));
+    }
+    return true;
+  };
   while (sch.next(sg)) {
     const bool rd = kHybrid && sg.head;
     const uint32_t t0 = tile, n = sg.ke - sg.kb;
+    bool staged = false;   // a staged merge: the K, then V, stages it uses are signalled idle
+    if (sg.head && !sg.tail) {
+      const long long first = static_cast<long long>(sg.Q) * a.nkv;
+      staged = staged_merge(owner(first + a.nkv - 1, a) - owner(first, a) + 1);
+    }
     const uint32_t r0 = ring, r_rd = ring + n;   // first key tile's ring slot, the readout operands' slot
     // Score tiles issued before the P.V loop: two. Afterwards the scores of tile t + 2 are
     // issued right behind the P.V MMA of tile t: they go to the buffer whose P was read by
@@ -319,7 +358,11 @@ __device__ void mma_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, co
     // read before either is rewritten.
     if (nseg > 0 && !mbar_wait_warp(sm.bar(kBarOEmpty), (nseg - 1) & 1, g)) return;
     tc_fence_after();
-    if (lead && !rd && n <= npre) mma_commit(sm.bar(kBarQEmpty));
+    if (n <= npre) {   // every score tile is issued
+      if (lead && staged) mma_commit(sm.bar(kBarLastQK));
+      if (rd && !issue_qwq(t0, n, r_rd)) return;
+      if (lead && !rd) mma_commit(sm.bar(kBarQEmpty));
+    }
     const uint32_t nissued = npre;   // score tiles issued ahead of the P.V loop
     for (uint32_t i = 0; i < n; ++i) {
       const uint32_t t = t0 + i, r = r0 + i;
@@ -335,24 +378,19 @@ __device__ void mma_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, co
       }
       if (i + nissued < n) {
         if (!issue_qk(t + nissued, r + nissued)) return;
-        if (lead && !rd && i + nissued + 1 == n) mma_commit(sm.bar(kBarQEmpty));
+        if (i + nissued + 1 == n) {   // that was the last score tile
+          if (lead && staged) mma_commit(sm.bar(kBarLastQK));
+          if (rd && !issue_qwq(t0, n, r_rd)) return;
+          if (lead && !rd) mma_commit(sm.bar(kBarQEmpty));
+        }
       }
     }
+    if (lead && staged) mma_commit(sm.bar(kBarLastPV));
     if (rd) {
-      // Readout O_inter = (Q Wq_h) S_{N-1}, after the last P.V. Every score buffer is
-      // free: Q' goes to the buffer of tile t0 + n (Y), O_inter to that of the last tile (X,
-      // read by the softmax threads before the next segment's third score tile is issued).
-      const uint32_t tY = tmem + 128u * sbuf(t0 + n), tX = tmem + 128u * sbuf(t0 + n - 1);
+      // Second readout MMA, after the last P.V: O_inter = Q' S_{N-1}, with Q' packed to
+      // bf16 in place by the softmax threads, into X (see o_inter_tile).
+      const uint32_t tY = tmem + 128u * sbuf(t0 + n), tX = tmem + 128u * o_inter_tile(t0, n, sg.last);
       const int rs = ring_stage(r_rd);
-      if (!mbar_wait_warp(sm.bar(kBarKFull + rs), ring_phase(r_rd), g)) return;
-      tc_fence_after();
-      if (lead) {
-        mma8_ss<false, true>(tY, desc_kmajor(sm.q(), 0), desc_mnmajor(sm.k(rs), 0), id_kmn, 0u);
-        mma_commit(sm.bar(kBarKEmpty + rs));
-        mma_commit(sm.bar(kBarQEmpty));
-        mma_commit(sm.bar(kBarQp));
-      }
-      // Q' packed to bf16 in place by the softmax threads, then O_inter = Q' S_h.
       if (!mbar_wait_warp(sm.bar(kBarQpReady), nhead & 1, g)) return;
       if (!mbar_wait_warp(sm.bar(kBarVFull + rs), ring_phase(r_rd), g)) return;
       tc_fence_after();
@@ -422,75 +460,31 @@ __device__ __forceinline__ float4* quad_ptr(float* base, size_t record, int q, u
   return reinterpret_cast<float4*>(base) + ((record * 32 + q) * kRows + r);
 }
 
-// End of a segment. The segment holding key tile 0 of a query tile (its head) finishes
-// the tile: it combines its own O (TMEM) with the partial records of the tile's other
-// segments, adds O_inter and writes O. With contiguous unit ranges the head segment is
-// the last segment of its CTA and every other segment of the tile starts another CTA's
-// range, so those records are normally published long before. Any other segment stores
-// its partial record (O_acc, running max m, sum l) and the publisher warp raises the
-// record's flag. Loads are issued in batches so their latencies overlap. Kept out of line
-// so its registers do not compete with the softmax loop. Returns false if a wait gave up.
-template <bool kHybrid>
-__device__ __noinline__ bool segment_epilogue(const Smem& sm, const QueryArgs& a, const Seg& sg, uint32_t r, int half,
-                                              int c0, int ncols, uint32_t tO, uint32_t tX, float m, float l_row,
-                                              uint32_t& gphase, volatile int* merge_ok, const float* stage,
-                                              const Guard& g) {
-  const int q0 = c0 / 4;   // this half's first column quad
-  const long long first = static_cast<long long>(sg.Q) * a.nkv;
-  const int c_first = owner(first, a);
-  const size_t slot0 = static_cast<size_t>(sg.Q) * a.max_segs;
-  if (!sg.head) {
-    const size_t slot = slot0 + (static_cast<int>(blockIdx.x) - c_first);
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      if (16 * c >= ncols) break;
-      uint32_t ov[16];
-      tmem_ld16(tO + c0 + 16u * c, ov);
-      tmem_wait_ld();
-      reg_fence16(ov);
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        *quad_ptr(a.part_o, slot, q0 + 4 * c + q, r) =
-            make_float4(__uint_as_float(ov[4 * q]), __uint_as_float(ov[4 * q + 1]), __uint_as_float(ov[4 * q + 2]),
-                        __uint_as_float(ov[4 * q + 3]));
-    }
-    if (half == 0) {
-      a.part_ml[(slot * 2) * kRows + r] = m;
-      a.part_ml[(slot * 2 + 1) * kRows + r] = l_row;
-    }
-    tc_fence_before();
-    warp_arrive(sm.bar(kBarOEmpty));   // TMEM read: the next segment may reuse O
-    warp_arrive(sm.bar(kBarRec));      // record stored: the publisher may raise its flag
-    return true;
-  }
-  // Head segment: the tile's other records (if any), then the merge. Warp 3 stages them
-  // in shared memory when they fit; otherwise they are read from scratch here.
-  const int nsegs = sg.tail ? 1 : owner(first + a.nkv - 1, a) - c_first + 1;
-  const bool staged = staged_merge(nsegs);
+// The merge of a head segment: its own O (TMEM, max m, sum l_row) with the tile's other
+// nsegs - 1 records, plus O_inter (TMEM, the layer only), normalised and rounded to bf16.
+// kStaged: the single other record is in shared memory (see staged_merge) and the output
+// goes to the shared-memory tile otile for a TMA store; otherwise records come from
+// scratch and rows go straight to global memory. Two instantiations, so neither path
+// carries the other's loads.
+template <bool kHybrid, bool kStaged>
+__device__ __forceinline__ void merge_rows(const QueryArgs& a, const Seg& sg, uint32_t r, int half, int c0, int ncols,
+                                           uint32_t tO, uint32_t tX, float m, float l_row, int nsegs_rt,
+                                           size_t slot0, const float* stage, int k1, int k2, uint32_t otile) {
+  const int nsegs = kStaged ? 2 : nsegs_rt;
+  const int q0 = c0 / 4;
   const float4* st4 = reinterpret_cast<const float4*>(stage);
-  if (staged) {
-    // Every MMA of the segment is done (OFull): warp 3 may overwrite the tile region. At
-    // most one staged merge per CTA and launch, so both barriers complete once (phase 0).
-    warp_arrive(sm.bar(kBarStageGo));
-    if (!mbar_wait_warp(sm.bar(kBarRecLoad), 0, g)) return false;
-  } else if (nsegs > 1) {
-    if (half == 0 && r == 0) {
-      bool ok = true;
-      for (int s = 1; s < nsegs && ok; ++s) ok = wait_flag(a.flags + slot0 + s, a.epoch, g);
-      *merge_ok = ok ? 1 : 0;
-    }
-    if (!group_sync(sm.bar(kBarGroup), gphase, g)) return false;
-    if (!*merge_ok) return false;
-  }
+  // Record s of the tile's other segments: the staged copy (shared memory) or scratch.
   auto rec_m = [&](int s) {
-    return staged ? stage[kStageMlOff / 4 + (s - 1) * 256 + r] : __ldcg(a.part_ml + ((slot0 + s) * 2) * kRows + r);
+    if constexpr (kStaged) return stage[(kVOff + k1 * kTileBytes) / 4 + r];
+    else return __ldcg(a.part_ml + ((slot0 + s) * 2) * kRows + r);
   };
   auto rec_l = [&](int s) {
-    return staged ? stage[kStageMlOff / 4 + (s - 1) * 256 + 128 + r]
-                  : __ldcg(a.part_ml + ((slot0 + s) * 2 + 1) * kRows + r);
+    if constexpr (kStaged) return stage[(kVOff + k1 * kTileBytes) / 4 + kRows + r];
+    else return __ldcg(a.part_ml + ((slot0 + s) * 2 + 1) * kRows + r);
   };
   auto rec_o = [&](int s, int q) {
-    return staged ? st4[(s - 1) * (kStageRecBytes / 16) + q * kRows + r] : __ldcg(quad_ptr(a.part_o, slot0 + s, q, r));
+    if constexpr (kStaged) return st4[(kKOff + (q < 16 ? k1 : k2) * kTileBytes) / 16 + (q & 15) * kRows + r];
+    else return __ldcg(quad_ptr(a.part_o, slot0 + s, q, r));
   };
   float ws[kMaxSegs];
   float M = m;
@@ -555,13 +549,99 @@ __device__ __noinline__ bool segment_epilogue(const Smem& sm, const QueryArgs& a
 #pragma unroll
       for (int e = 0; e < 16; ++e) y[e] += __uint_as_float(xv[e]);
     }
-    if (row_ok) {
+    const uint4 w0 = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                                pack_bf16x2(y[6], y[7]));
+    const uint4 w1 = make_uint4(pack_bf16x2(y[8], y[9]), pack_bf16x2(y[10], y[11]), pack_bf16x2(y[12], y[13]),
+                                pack_bf16x2(y[14], y[15]));
+    if constexpr (kStaged) {
+      // Columns 16c .. 16c+15 of this half = 16-byte chunks 2c and 2c+1 of panel `half`.
+      const uint32_t row = otile + half * kPanelBytes + r * 128u;
+      st_shared_v4(row + (((2u * c) ^ (r & 7u)) << 4), w0.x, w0.y, w0.z, w0.w);
+      st_shared_v4(row + (((2u * c + 1u) ^ (r & 7u)) << 4), w1.x, w1.y, w1.z, w1.w);
+    } else if (row_ok) {
       uint4* dst = reinterpret_cast<uint4*>(out_row + 16 * c);
-      dst[0] = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
-                          pack_bf16x2(y[6], y[7]));
-      dst[1] = make_uint4(pack_bf16x2(y[8], y[9]), pack_bf16x2(y[10], y[11]), pack_bf16x2(y[12], y[13]),
-                          pack_bf16x2(y[14], y[15]));
+      dst[0] = w0;
+      dst[1] = w1;
     }
+  }
+}
+
+// End of a segment. The segment holding key tile 0 of a query tile (its head) finishes
+// the tile: it combines its own O (TMEM) with the partial records of the tile's other
+// segments, adds O_inter and writes O. With contiguous unit ranges the head segment is
+// the last segment of its CTA and every other segment of the tile starts another CTA's
+// range, so those records are normally published long before. Any other segment stores
+// its partial record (O_acc, running max m, sum l) and the publisher warp raises the
+// record's flag. Loads are issued in batches so their latencies overlap. Kept out of line
+// so its registers do not compete with the softmax loop. Returns false if a wait gave up.
+template <bool kHybrid>
+__device__ __noinline__ bool segment_epilogue(const Smem& sm, const QueryArgs& a, const Seg& sg, uint32_t r, int half,
+                                              int c0, int ncols, uint32_t tO, uint32_t tX, float m, float l_row,
+                                              uint32_t& gphase, volatile int* merge_ok, const float* stage, int rs,
+                                              const CUtensorMap* tm_o, const Guard& g) {
+  const int q0 = c0 / 4;   // this half's first column quad
+  const long long first = static_cast<long long>(sg.Q) * a.nkv;
+  const int c_first = owner(first, a);
+  const size_t slot0 = static_cast<size_t>(sg.Q) * a.max_segs;
+  if (!sg.head) {
+    const size_t slot = slot0 + (static_cast<int>(blockIdx.x) - c_first);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (16 * c >= ncols) break;
+      uint32_t ov[16];
+      tmem_ld16(tO + c0 + 16u * c, ov);
+      tmem_wait_ld();
+      reg_fence16(ov);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        *quad_ptr(a.part_o, slot, q0 + 4 * c + q, r) =
+            make_float4(__uint_as_float(ov[4 * q]), __uint_as_float(ov[4 * q + 1]), __uint_as_float(ov[4 * q + 2]),
+                        __uint_as_float(ov[4 * q + 3]));
+    }
+    if (half == 0) {
+      a.part_ml[(slot * 2) * kRows + r] = m;
+      a.part_ml[(slot * 2 + 1) * kRows + r] = l_row;
+    }
+    tc_fence_before();
+    warp_arrive(sm.bar(kBarOEmpty));   // TMEM read: the next segment may reuse O
+    warp_arrive(sm.bar(kBarRec));      // record stored: the publisher may raise its flag
+    return true;
+  }
+  // Head segment: the tile's other records (if any), then the merge. Warp 3 stages them
+  // in shared memory when they fit; otherwise they are read from scratch here.
+  const int nsegs = sg.tail ? 1 : owner(first + a.nkv - 1, a) - c_first + 1;
+  const bool staged = staged_merge(nsegs);
+  const int k1 = (rs + 1) % kStages, k2 = (rs + 2) % kStages;   // idle ring stages (see staged_merge)
+  if (staged) {
+    // At most one staged merge per CTA and launch: the barrier completes once (phase 0).
+    if (!mbar_wait_warp(sm.bar(kBarRecLoad), 0, g)) return false;
+  } else if (nsegs > 1) {
+    if (half == 0 && r == 0) {
+      bool ok = true;
+      for (int s = 1; s < nsegs && ok; ++s) ok = wait_flag(a.flags + slot0 + s, a.epoch, g);
+      *merge_ok = ok ? 1 : 0;
+    }
+    if (!group_sync(sm.bar(kBarGroup), gphase, g)) return false;
+    if (!*merge_ok) return false;
+  }
+  const uint32_t otile = sm.v(k2);   // staged: the output tile (two 128-byte-swizzled panels)
+  if (staged)
+    merge_rows<kHybrid, true>(a, sg, r, half, c0, ncols, tO, tX, m, l_row, nsegs, slot0, stage, k1, k2, otile);
+  else
+    merge_rows<kHybrid, false>(a, sg, r, half, c0, ncols, tO, tX, m, l_row, nsegs, slot0, stage, k1, k2, otile);
+  if (staged && 64 * half < a.d) {
+    // Each warp stores its own 32 rows x 64 columns by TMA (coalesced; rows past T and
+    // columns past d are clipped). A 32-row slice of a swizzled panel starts on a 1 KiB
+    // boundary, so it is a swizzled box of its own.
+    fence_proxy_async_smem();
+    __syncwarp();
+    if ((r & 31u) == 0) {
+      const uint32_t q32 = r & ~31u;
+      tma_store_4d(tm_o, otile + half * kPanelBytes + q32 * 128u, 64 * half, sg.h, sg.qt * kRows + q32, sg.b);
+      bulk_commit_group();
+      bulk_wait_group_read0();   // the source must stay intact until read (the CTA exits next)
+    }
+    __syncwarp();
   }
   tc_fence_before();
   warp_arrive(sm.bar(kBarOEmpty));
@@ -571,15 +651,15 @@ __device__ __noinline__ bool segment_epilogue(const Smem& sm, const QueryArgs& a
 // Warp 3. (1) Raises the flag of each partial record this CTA stores, once the softmax
 // warps have stored it: their CTA-scope arrival orders those stores before this warp's
 // device-scope fence, so a CTA that reads the flag (acquire) sees the whole record.
-// (2) For a head segment that merges from staged copies (always the CTA's last segment):
-// waits for the other records' flags while the segment runs, then, once the softmax warps
-// report its MMAs done (the tile region idle), bulk-copies those records, their (m, l)
-// rows and O_inter into shared memory. Every barrier this warp waits on completes at most
-// once per launch, so a parity wait can never alias an earlier phase.
+// (2) For a staged merge (the CTA's last segment): waits for the other record's flag while
+// the segment runs, then bulk-copies that record into the idle K stages once the last score
+// MMA is done, and its (m, l) rows into an idle V stage once the last P.V MMA is done. Every barrier this warp waits on completes at
+// most once per launch, so a parity wait can never alias an earlier phase.
 template <bool kHybrid>
 __device__ void publisher(const Smem& sm, const QueryArgs& a, const Guard& g) {
   const bool lead = (threadIdx.x & 31) == 0;
   uint32_t nrec = 0;   // a CTA stores at most one record (only its first segment can lack key tile 0)
+  uint32_t ring = 0;   // ring slots used so far (key tiles, plus one readout operand per head)
   bool staged_issued = false;
   Sched sch(a, blockIdx.x);
   Seg sg;
@@ -587,6 +667,9 @@ __device__ void publisher(const Smem& sm, const QueryArgs& a, const Guard& g) {
     const long long first = static_cast<long long>(sg.Q) * a.nkv;
     const int c_first = owner(first, a);
     const size_t slot0 = static_cast<size_t>(sg.Q) * a.max_segs;
+    const uint32_t n = sg.ke - sg.kb;
+    const int ws = ring_stage(ring + n);   // the readout operands' stage
+    ring += n + ((kHybrid && sg.head) ? 1u : 0u);
     if (!sg.head) {
       if (!mbar_wait_warp(sm.bar(kBarRec), nrec & 1, g)) break;
       ++nrec;
@@ -595,32 +678,29 @@ __device__ void publisher(const Smem& sm, const QueryArgs& a, const Guard& g) {
         atomicExch(a.flags + slot0 + (static_cast<int>(blockIdx.x) - c_first), a.epoch);
       }
       __syncwarp();
-    } else {
-      const int nsegs = sg.tail ? 1 : owner(first + a.nkv - 1, a) - c_first + 1;
-      if (staged_merge(nsegs)) {
-        bool ok = true;
-        if (lead)
-          for (int s = 1; s < nsegs && ok; ++s) ok = wait_flag(a.flags + slot0 + s, a.epoch, g);
-        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-        // The softmax warps signal that the segment's MMAs are done (nothing reads the tile
-        // region any more) and that O_inter, stored at the segment's start, is ordered
-        // before this point. This is the CTA's last segment: one phase per launch.
-        if (!mbar_wait_warp(sm.bar(kBarStageGo), 0, g)) break;
-        if (lead) {
-          const uint32_t rec_bytes = static_cast<uint32_t>(a.d) * kRows * 4;   // d/4 column quads
-          const uint32_t nrecs = static_cast<uint32_t>(nsegs - 1);
-          fence_proxy_async_global();
-          mbar_expect_tx(sm.bar(kBarRecLoad), nrecs * (rec_bytes + 1024u));
-          for (int s = 1; s < nsegs; ++s) {
-            bulk_load(sm.tiles + (s - 1) * kStageRecBytes, a.part_o + (slot0 + s) * kRows * kDP, rec_bytes,
-                      sm.bar(kBarRecLoad));
-            bulk_load(sm.tiles + kStageMlOff + (s - 1) * 1024u, a.part_ml + (slot0 + s) * 2 * kRows, 1024u,
-                      sm.bar(kBarRecLoad));
-          }
-          }
-        staged_issued = true;
-        __syncwarp();
+    } else if (!sg.tail && staged_merge(owner(first + a.nkv - 1, a) - c_first + 1)) {
+      bool ok = true;
+      if (lead) ok = wait_flag(a.flags + slot0 + 1, a.epoch, g);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      const int k1 = (ws + 1) % kStages, k2 = (ws + 2) % kStages;
+      // The record (d/4 column quads) into K stages k1, k2 once the last score MMA is done,
+      // in 4 KiB pieces so that several are in flight; its (m, l) rows into V stage k1
+      // once the last P.V MMA is done.
+      if (!mbar_wait_warp(sm.bar(kBarLastQK), 0, g)) break;
+      const uint32_t rec_bytes = static_cast<uint32_t>(a.d) * kRows * 4;
+      const char* rec = reinterpret_cast<const char*>(a.part_o + (slot0 + 1) * kRows * kDP);
+      if (lead) {
+        fence_proxy_async_global();
+        mbar_expect_tx(sm.bar(kBarRecLoad), rec_bytes + 1024u);
       }
+      for (uint32_t off = 4096u * (threadIdx.x & 31); off < rec_bytes; off += 4096u * 32) {
+        const uint32_t dst = (off < kTileBytes ? sm.k(k1) : sm.k(k2)) + off % kTileBytes;
+        bulk_load(dst, rec + off, 4096u, sm.bar(kBarRecLoad));
+      }
+      staged_issued = true;
+      if (!mbar_wait_warp(sm.bar(kBarLastPV), 0, g)) break;
+      if (lead) bulk_load(sm.v(k1), a.part_ml + (slot0 + 1) * 2 * kRows, 1024u, sm.bar(kBarRecLoad));
+      __syncwarp();
     }
   }
   // Copies into shared memory must land before the CTA exits (matters only after an abort).
@@ -628,11 +708,11 @@ __device__ void publisher(const Smem& sm, const QueryArgs& a, const Guard& g) {
 }
 
 template <bool kHybrid>
-__device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const QueryArgs& a, int warp, int lane,
-                             const Guard& g) {
+__device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const QueryArgs& a, int warp,
+                             const CUtensorMap* tm_o, const Guard& g) {
   const int quarter = warp & 3;
   const int half = (warp - 4) >> 2;                         // 0: columns 0-63, 1: columns 64-127
-  const uint32_t r = quarter * 32 + lane;                   // tile row == TMEM lane
+  const uint32_t r = quarter * 32 + (threadIdx.x & 31);     // tile row == TMEM lane
   const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
   const uint32_t tO = tmem + lane_off + kColO;
   float* xch = reinterpret_cast<float*>(ctl + kCtlX);      // [2 slots][2 halves][128]
@@ -641,13 +721,15 @@ __device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const 
   const int d = a.d;
   const int c0 = 64 * half;                                 // first column of this thread's half
   const int ncols = max(0, min(64, d - c0));                // output columns of this half
-  uint32_t nseg = 0, nhead = 0, tile = 0, gphase = 0, nx = 0;
+  uint32_t nseg = 0, nhead = 0, tile = 0, gphase = 0, nx = 0, ring = 0;
   // Test hook: a wait that can only run out (the bounded-wait path, without a fault).
   if (a.stall && !mbar_wait_warp(sm.bar(kBarNever), 0, g)) return;
   Sched sch(a, blockIdx.x);
   Seg sg;
   while (sch.next(sg)) {
     const uint32_t t0 = tile, n = sg.ke - sg.kb;
+    const int rs = ring_stage(ring + n);   // ring stage of the readout operands (staged merges)
+    ring += n + ((kHybrid && sg.head) ? 1u : 0u);
     float m = -INFINITY, l = 0.f;
     for (uint32_t i = 0; i < n; ++i) {
       const uint32_t t = t0 + i;
@@ -706,7 +788,7 @@ __device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const 
     // ---- end of segment. A segment holding key tile 0 computes the readout here: Q' =
     // Q Wq_h arrives (fp32) in the S buffer of tile t0 + n; each half packs its own 64
     // columns to bf16 pairs in place (the readout MMA's A operand, same layout as P).
-    const uint32_t tX = tmem + lane_off + 128u * sbuf(t0 + n - 1);   // O_inter, when computed
+    const uint32_t tX = tmem + lane_off + 128u * o_inter_tile(t0, n, sg.last);   // O_inter, when computed
     if (kHybrid && sg.head) {
       const uint32_t tY = tmem + lane_off + 128u * sbuf(t0 + n);
       if (!mbar_wait_warp(sm.bar(kBarQp), nhead & 1, g)) return;
@@ -739,7 +821,7 @@ __device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const 
     float l0, l1;
     if (!pair_swap(pair_bar, xch, nx, half, r, l, l0, l1, g)) return;
     if (!segment_epilogue<kHybrid>(sm, a, sg, r, half, c0, ncols, tO, tX, m, l0 + l1, gphase, merge_ok,
-                                   reinterpret_cast<const float*>(ctl - kTileRegion), g))
+                                   reinterpret_cast<const float*>(ctl - kTileRegion), rs, tm_o, g))
       return;
     ++nseg;
   }
@@ -749,7 +831,8 @@ template <bool kHybrid>
 __global__ void __launch_bounds__(kThreads, 1)
     arl2_query_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
-                      const __grid_constant__ CUtensorMap tm_s, const QueryArgs a) {
+                      const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_o,
+                      const QueryArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t tiles = smem_u32(smem_raw);
   if (tiles & 1023u) {   // the swizzled tiles need a 1 KiB-aligned base: report, do nothing
@@ -788,7 +871,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(sm.bar(kBarNever), 1);
     mbar_init(sm.bar(kBarRec), kSoftmaxWarps);
     mbar_init(sm.bar(kBarRecLoad), 1);
-    mbar_init(sm.bar(kBarStageGo), kSoftmaxWarps);
+    mbar_init(sm.bar(kBarLastPV), 1);
+    mbar_init(sm.bar(kBarLastQK), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -821,7 +905,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 3) {
     publisher<kHybrid>(sm, a, g);
   } else if (warp >= 4) {
-    softmax_role<kHybrid>(sm, ctl_ptr, tmem, a, warp, lane, g);
+    softmax_role<kHybrid>(sm, ctl_ptr, tmem, a, warp, &tm_o, g);
   }
 
   tc_fence_before();
@@ -880,12 +964,13 @@ size_t query_scratch_floats(const QueryPlan& p) {
 }
 
 cudaError_t launch_query(bool hybrid, const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                         const CUtensorMap& tm_w, const CUtensorMap& tm_s, const QueryArgs& a, cudaStream_t stream) {
+                         const CUtensorMap& tm_w, const CUtensorMap& tm_s, const CUtensorMap& tm_o, const QueryArgs& a,
+                         cudaStream_t stream) {
   const dim3 grid(a.num_ctas);
   if (hybrid)
-    arl2_query_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_k, tm_v, tm_w, tm_s, a);
+    arl2_query_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_k, tm_v, tm_w, tm_s, tm_o, a);
   else
-    arl2_query_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_k, tm_v, tm_w, tm_s, a);
+    arl2_query_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_k, tm_v, tm_w, tm_s, tm_o, a);
   return cudaGetLastError();
 }
 
