@@ -58,6 +58,27 @@ COMMIT_FLOPS = B * H * 4 * 2.0 * T * D * D                             # K Wk, V
 COMMIT_BYTES = B * T * H * D * 2 * 2 + 2 * B * H * T * 4 + B * H * D * D * 4 * 2 + 2 * H * D * D * 2
 
 
+def _query_traffic():
+    """DRAM bytes per query launch from the committed ncu capture, or None when the query
+    kernel's sources changed since that capture (the summary records their SHA-256)."""
+    import hashlib
+    import re
+    path = os.path.join(ROOT, "profiles", "arl2_query_kernel_480p.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    t = re.search(r"^traffic_bytes_per_launch: (\d+)$", text, re.M)
+    h = re.search(r"^kernel_sources_sha256: ([0-9a-f]{64})$", text, re.M)
+    if not t or not h:
+        return None
+    csrc = os.path.join(ROOT, "softmax_attention_ar_b200", "csrc")
+    digest = hashlib.sha256()
+    for f in ("arl2_query.cu", "arl2_device.cuh", "arl2_kernels.h"):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            digest.update(fh.read())
+    return int(t.group(1)) if digest.hexdigest() == h.group(1) else None
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -308,7 +329,7 @@ def run_ours(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": CONFIG,
         "roofline": {"bound": "tensor", "achieved": q_tflops, "peak": peak, "unit": "TFLOP/s",
-                     "frac": q_tflops / peak, "traffic": None,
+                     "frac": q_tflops / peak, "traffic": _query_traffic(), "traffic_unit": "DRAM bytes per launch",
                      "kernel": "arl2_query_kernel (one query pass)",
                      "peak_source": f"bf16_tflops_sustained ({peaks['source']})",
                      "frac_of_burst_peak": q_tflops / peaks["bf16_tflops"]},
