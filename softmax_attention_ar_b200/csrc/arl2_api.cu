@@ -83,6 +83,45 @@ struct MapCache {
   }
 };
 
+// Outputs of the most recent query launches, per stream, process-wide. A query may run as a
+// programmatic dependent of the previous kernel in its stream only if its inputs do not
+// overlap the output of the query launched last on that stream (chained layers).
+struct LastOut {
+  cudaStream_t stream = nullptr;
+  uintptr_t begin = 0, end = 0;
+  bool used = false;
+};
+std::mutex g_lastout_mu;
+LastOut g_lastout[16];
+
+// Record o as the last query output on stream st; return whether [q, k, v] (each `bytes`
+// long) are clear of the output recorded before it.
+bool note_query_output(cudaStream_t st, const void* q, const void* k, const void* v, const void* o, size_t bytes) {
+  std::lock_guard<std::mutex> lk(g_lastout_mu);
+  LastOut* slot = nullptr;
+  for (auto& e : g_lastout)
+    if (e.used && e.stream == st) slot = &e;
+  bool clear = true;
+  if (slot) {
+    for (const void* p : {q, k, v}) {
+      const uintptr_t b = reinterpret_cast<uintptr_t>(p), e = b + bytes;
+      if (b < slot->end && slot->begin < e) clear = false;
+    }
+  } else {
+    for (auto& e : g_lastout)
+      if (!e.used) {
+        slot = &e;
+        break;
+      }
+    if (!slot) slot = &g_lastout[reinterpret_cast<uintptr_t>(st) % 16];
+  }
+  slot->used = true;
+  slot->stream = st;
+  slot->begin = reinterpret_cast<uintptr_t>(o);
+  slot->end = slot->begin + bytes;
+  return clear;
+}
+
 std::mutex g_setup_mu;
 bool g_setup_done[64] = {};
 
@@ -141,6 +180,7 @@ struct arl2_ctx {
   int frame = 0;
   bool maps_set = false;
   bool stall_next = false;        // failure-detection test hook (next query only)
+  bool overlap = false;           // queries may start behind the previous kernel (see the header)
   unsigned long long timeout_ns = kDefaultTimeoutNs;
   CUtensorMap tm_w[3];
   CUtensorMap tm_s;
@@ -239,8 +279,10 @@ arl2_status query_impl(arl2_ctx* c, const void* q, const void* k, const void* v,
   a.stall = c->stall_next ? 1 : 0;
   c->stall_next = false;
   set_plan(&a, c->qplan, c->qscratch, c->qflags, next_epoch(&c->qepoch));
-  return arl2::launch_query(true, *mq, *mk, *mv, c->tm_w[0], c->tm_s, *mo, a, st) == cudaSuccess ? ARL2_OK
-                                                                                                : ARL2_ERR_CUDA;
+  const bool clear = note_query_output(st, q, k, v, o, c->act_elems() * 2);
+  return arl2::launch_query(true, *mq, *mk, *mv, c->tm_w[0], c->tm_s, *mo, a, st, c->overlap && clear) == cudaSuccess
+             ? ARL2_OK
+             : ARL2_ERR_CUDA;
 }
 
 arl2_status commit_impl(arl2_ctx* c, const void* k, const void* v, const float* alpha, const float* beta,
@@ -447,6 +489,12 @@ arl2_status arl2_get_status(arl2_ctx* c) {
   return read_status(c->err);
 }
 
+arl2_status arl2_set_query_overlap(arl2_ctx* c, int enable) {
+  if (!c) return ARL2_ERR_INVALID_ARG;
+  c->overlap = enable != 0;
+  return ARL2_OK;
+}
+
 arl2_status arl2_set_wait_timeout_ns(arl2_ctx* c, uint64_t timeout_ns) {
   if (!c || timeout_ns == 0) return ARL2_ERR_INVALID_ARG;
   c->timeout_ns = timeout_ns;
@@ -539,7 +587,7 @@ arl2_status arl2_kvcache_query(arl2_kvcache* c, const arl2_bf16* q, const arl2_b
   a.timeout_ns = c->timeout_ns;
   set_plan(&a, arl2::plan_query(c->B, c->H, c->T, a.kv_len, c->num_sms), c->qscratch, c->qflags,
            next_epoch(&c->qepoch));
-  return arl2::launch_query(false, *mq, c->tm_k, c->tm_v, c->tm_k, c->tm_k, *mo, a, st) == cudaSuccess
+  return arl2::launch_query(false, *mq, c->tm_k, c->tm_v, c->tm_k, c->tm_k, *mo, a, st, false) == cudaSuccess
              ? ARL2_OK
              : ARL2_ERR_CUDA;
 }

@@ -286,24 +286,44 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
-// S_new = abar * S_old + sum_g part_g, four consecutive elements per thread.
+// S_new = abar * S_old + sum_g part_g, four consecutive elements per thread. The partials
+// are loaded in batches of 8 (all in flight at once) and added in group order, so the sum
+// does not depend on the batching.
 __global__ void __launch_bounds__(256) arl2_commit_reduce_kernel(const ReduceArgs a) {
   const int bh = blockIdx.y;
   const int dd = a.d * a.d;
   const int e = (blockIdx.x * 256 + threadIdx.x) * 4;
   if (e >= dd) return;
+  const float* ap = a.alpha_part + static_cast<size_t>(bh) * a.ngroups;
   float asum = 0.f;
-  for (int g = 0; g < a.ngroups; ++g) asum += a.alpha_part[static_cast<size_t>(bh) * a.ngroups + g];
+  for (int g0 = 0; g0 < a.ngroups; g0 += 8) {
+    float x[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) x[j] = (g0 + j < a.ngroups) ? ap[g0 + j] : 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (g0 + j < a.ngroups) asum += x[j];
+  }
   const float abar = asum * a.inv_T;
   const size_t off = static_cast<size_t>(bh) * dd + e;
   const float4 s = *reinterpret_cast<const float4*>(a.S_old + off);
   float4 acc = make_float4(abar * s.x, abar * s.y, abar * s.z, abar * s.w);
-  for (int g = 0; g < a.ngroups; ++g) {
-    const float4 u = *reinterpret_cast<const float4*>(a.part + (static_cast<size_t>(bh) * a.ngroups + g) * dd + e);
-    acc.x += u.x;
-    acc.y += u.y;
-    acc.z += u.z;
-    acc.w += u.w;
+  const float* pp = a.part + static_cast<size_t>(bh) * a.ngroups * dd + e;
+  for (int g0 = 0; g0 < a.ngroups; g0 += 8) {
+    float4 u[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      u[j] = (g0 + j < a.ngroups) ? *reinterpret_cast<const float4*>(pp + static_cast<size_t>(g0 + j) * dd)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (g0 + j < a.ngroups) {
+        acc.x += u[j].x;
+        acc.y += u[j].y;
+        acc.z += u[j].z;
+        acc.w += u[j].w;
+      }
+    }
   }
   *reinterpret_cast<float4*>(a.S_new + off) = acc;
   *reinterpret_cast<uint2*>(a.S_new_bf16 + off) = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));

@@ -392,6 +392,15 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
+// Programmatic dependent launch. launch_dependents: the next kernel in the stream, if it was
+// launched as a programmatic dependent, may start once every CTA of this grid executed this
+// or exited. wait: block until the preceding grid (if this one was launched as its
+// dependent) has completed and its memory is visible; a no-op otherwise.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // One lane of a converged warp (the lowest active one) gets true.
 __device__ __forceinline__ bool elect_one() {
   uint32_t pred;

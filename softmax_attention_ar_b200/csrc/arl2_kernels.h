@@ -79,9 +79,12 @@ size_t commit_smem_bytes();
 cudaError_t query_setup();   // per-device function attributes
 cudaError_t commit_setup();
 
+// dependent: launch as a programmatic dependent of the preceding kernel in the stream. The
+// kernel reads its inputs before that kernel completes, so the caller must know that the
+// preceding kernel does not write them.
 cudaError_t launch_query(bool hybrid, const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                          const CUtensorMap& tm_w, const CUtensorMap& tm_s, const CUtensorMap& tm_o, const QueryArgs& a,
-                         cudaStream_t stream);
+                         cudaStream_t stream, bool dependent);
 cudaError_t launch_commit(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const CUtensorMap& tm_wk,
                           const CUtensorMap& tm_wv, const CUtensorMap& tm_s, const CommitArgs& a,
                           const ReduceArgs& r, cudaStream_t stream);

@@ -580,6 +580,9 @@ __device__ __noinline__ bool segment_epilogue(const Smem& sm, const QueryArgs& a
                                               uint32_t& gphase, volatile int* merge_ok, const float* stage, int rs,
                                               const CUtensorMap* tm_o, const Guard& g) {
   const int q0 = c0 / 4;   // this half's first column quad
+  // First global write of this thread in the launch: a query launched as the programmatic
+  // dependent of the previous one waits for it here (shared scratch, maybe the same output).
+  griddep_wait();
   const long long first = static_cast<long long>(sg.Q) * a.nkv;
   const int c_first = owner(first, a);
   const size_t slot0 = static_cast<size_t>(sg.Q) * a.max_segs;
@@ -673,6 +676,7 @@ __device__ void publisher(const Smem& sm, const QueryArgs& a, const Guard& g) {
     if (!sg.head) {
       if (!mbar_wait_warp(sm.bar(kBarRec), nrec & 1, g)) break;
       ++nrec;
+      griddep_wait();   // the previous launch may still poll this flag for its own epoch
       if (lead) {
         __threadfence();
         atomicExch(a.flags + slot0 + (static_cast<int>(blockIdx.x) - c_first), a.epoch);
@@ -890,6 +894,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // A query launched right behind this one may start its CTAs as SMs free up. It reads
+  // nothing this one writes; it waits for this grid before its first global write (its
+  // scratch and output may be this grid's).
+  griddep_launch_dependents();
 
   // Producers and the MMA issuer run warp-wide (uniform control flow and waits); one
   // elected lane issues each TMA copy, MMA and commit.
@@ -965,13 +973,20 @@ size_t query_scratch_floats(const QueryPlan& p) {
 
 cudaError_t launch_query(bool hybrid, const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                          const CUtensorMap& tm_w, const CUtensorMap& tm_s, const CUtensorMap& tm_o, const QueryArgs& a,
-                         cudaStream_t stream) {
-  const dim3 grid(a.num_ctas);
+                         cudaStream_t stream, bool dependent) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(a.num_ctas);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = dependent ? 1 : 0;
   if (hybrid)
-    arl2_query_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_k, tm_v, tm_w, tm_s, tm_o, a);
-  else
-    arl2_query_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_k, tm_v, tm_w, tm_s, tm_o, a);
-  return cudaGetLastError();
+    return cudaLaunchKernelEx(&cfg, arl2_query_kernel<true>, tm_q, tm_k, tm_v, tm_w, tm_s, tm_o, a);
+  return cudaLaunchKernelEx(&cfg, arl2_query_kernel<false>, tm_q, tm_k, tm_v, tm_w, tm_s, tm_o, a);
 }
 
 }  // namespace arl2

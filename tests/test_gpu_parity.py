@@ -239,6 +239,36 @@ def test_bounded_waits_report_a_timeout_and_leave_the_context_usable():
     assert max(o_errors(o_gpu, o_ref)) <= O_TOL
 
 
+def test_back_to_back_queries_overlapping_the_previous_kernel():
+    # With overlap on, each query is launched as a programmatic dependent of the one before
+    # it (its CTAs start while the previous query's last CTAs still run). Checked: four
+    # queries into one output buffer (the last one must win), four into separate buffers,
+    # and a query whose q is the previous query's output (the guard launches it normally).
+    B, T, H, d = 1, 1560, 4, 128
+    c = Case(B, T, H, d, config=116)
+    c.gpu.set_query_overlap(True)
+    host = [c.inputs(0, p) for p in range(4)]
+    dev = [tuple(dev_bf16(x) for x in qkv) for qkv in host]
+    rows = sample_rows(T, 32, seed=7)
+    refs = [c.ref.query(*(synth.bf16_to_f64(x) for x in qkv), rows=rows) for qkv in host]
+    shared = torch.empty_like(dev[0][0])
+    for p in range(4):
+        c.gpu.query(*dev[p], out=shared)
+    assert max(o_errors(host_f64(shared)[:, rows], refs[3])) <= O_TOL
+    outs = [torch.empty_like(dev[0][0]) for _ in range(4)]
+    for p in range(4):
+        c.gpu.query(*dev[p], out=outs[p])
+    for p in range(4):
+        assert max(o_errors(host_f64(outs[p])[:, rows], refs[p])) <= O_TOL, f"query {p}"
+    o1, o2 = torch.empty_like(dev[0][0]), torch.empty_like(dev[0][0])
+    c.gpu.query(*dev[0], out=o1)
+    c.gpu.query(o1, dev[1][1], dev[1][2], out=o2)
+    q2 = o1.view(torch.int16).cpu().numpy().view(np.uint16)
+    ref2 = c.ref.query(synth.bf16_to_f64(q2), synth.bf16_to_f64(host[1][1]), synth.bf16_to_f64(host[1][2]), rows=rows)
+    assert max(o_errors(host_f64(o2)[:, rows], ref2)) <= O_TOL
+    assert c.gpu.status() == arl2.ARL2_OK
+
+
 # ------------------------------------------------------------------ growing-KV baseline
 def test_kv_cache_baseline_parity():
     B, T, H, d, frames = 1, 200, 2, 128, 3
