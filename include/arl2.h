@@ -126,16 +126,18 @@ arl2_status arl2_get_status(arl2_ctx* ctx);
  * ARL2_ERR_TIMEOUT. Returns ARL2_ERR_INVALID_ARG for NULL or 0. */
 arl2_status arl2_set_wait_timeout_ns(arl2_ctx* ctx, uint64_t timeout_ns);
 
-/* Let this context's queries overlap the kernel before them in their stream (default off).
- * When on, a query is launched as a programmatic dependent: its CTAs may start, and read q,
- * k and v, while the preceding kernel in the stream is still running (on B200 this hides a
- * query's start-up behind the previous query's last CTAs). It waits for that kernel before
- * its first write, so back-to-back queries may share an output buffer. Turn it on only
- * when no kernel that writes q, k or v can run right before a query call in the same
- * stream without waiting for completion (kernels that do not use programmatic launch
- * always complete first, as do copies). As a guard, a query whose q, k or v overlaps the
+/* Let this context's queries and commits overlap the kernel before them in their stream
+ * (default off). When on, each is launched as a programmatic dependent: its CTAs may start,
+ * and read their inputs, while the preceding kernel in the stream is still running. On
+ * B200 this hides a call's start-up behind the previous query's last CTAs.
+ * - A query waits for that kernel before its first write, so back-to-back queries may
+ *   share an output buffer.
+ * - A commit writes only the other state buffer and its own scratch.
+ * Turn it on only when no kernel that writes a call's inputs can run right before it in
+ * the same stream without waiting for completion. Kernels that do not use programmatic
+ * launch always complete first, as do copies. As a guard, a call whose inputs overlap the
  * output of the last query launched in the same stream is launched normally. */
-arl2_status arl2_set_query_overlap(arl2_ctx* ctx, int enable);
+arl2_status arl2_set_launch_overlap(arl2_ctx* ctx, int enable);
 
 /* Failure-detection test hook. The next arl2_frame_query (or arl2_frame_query_host)
  * launch makes its softmax threads wait on an mbarrier that nothing signals. That wait

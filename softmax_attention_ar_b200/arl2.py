@@ -39,7 +39,7 @@ SIGNATURES = {
     "arl2_get_status": (_S, [_P]),
     "arl2_set_wait_timeout_ns": (_S, [_P, _U64]),
     "arl2_test_stall_next_query": (_S, [_P]),
-    "arl2_set_query_overlap": (_S, [_P, ctypes.c_int]),
+    "arl2_set_launch_overlap": (_S, [_P, ctypes.c_int]),
     "arl2_memory_bytes": (_SZ, [_P]),
     "arl2_destroy": (None, [_P]),
     "arl2_frame_commit_noalloc": (_S, [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
@@ -210,9 +210,9 @@ class ARL2Layer:
     def set_wait_timeout_ns(self, ns: int) -> None:
         _check(self._lib.arl2_set_wait_timeout_ns(self._ctx, int(ns)), "arl2_set_wait_timeout_ns")
 
-    def set_query_overlap(self, enable: bool) -> None:
-        """Queries may start behind the previous kernel in their stream (see arl2.h)."""
-        _check(self._lib.arl2_set_query_overlap(self._ctx, int(bool(enable))), "arl2_set_query_overlap")
+    def set_launch_overlap(self, enable: bool) -> None:
+        """Queries and commits may start behind the previous kernel in their stream (see arl2.h)."""
+        _check(self._lib.arl2_set_launch_overlap(self._ctx, int(bool(enable))), "arl2_set_launch_overlap")
 
     def test_stall_next_query(self) -> None:
         """Failure-detection hook: the next query's bounded wait runs out (no GPU fault)."""

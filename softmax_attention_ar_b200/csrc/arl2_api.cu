@@ -1,6 +1,8 @@
 // C-ABI layer of the ARL2 library: contexts, argument checks, TMA descriptors, state
 // ping-pong and launches. The computation itself lives in arl2_query.cu and arl2_commit.cu.
 #include <algorithm>
+#include <initializer_list>
+#include <utility>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -83,9 +85,9 @@ struct MapCache {
   }
 };
 
-// Outputs of the most recent query launches, per stream, process-wide. A query may run as a
-// programmatic dependent of the previous kernel in its stream only if its inputs do not
-// overlap the output of the query launched last on that stream (chained layers).
+// Outputs of the most recent query launches, per stream, process-wide. A query or commit may
+// run as a programmatic dependent of the previous kernel in its stream only if its inputs do
+// not overlap the output of the query launched last on that stream (chained layers).
 struct LastOut {
   cudaStream_t stream = nullptr;
   uintptr_t begin = 0, end = 0;
@@ -94,32 +96,33 @@ struct LastOut {
 std::mutex g_lastout_mu;
 LastOut g_lastout[16];
 
-// Record o as the last query output on stream st; return whether [q, k, v] (each `bytes`
-// long) are clear of the output recorded before it.
-bool note_query_output(cudaStream_t st, const void* q, const void* k, const void* v, const void* o, size_t bytes) {
+// Whether every (pointer, bytes) range is clear of the output of the last query launched on
+// stream st.
+bool clear_of_last_output(cudaStream_t st, std::initializer_list<std::pair<const void*, size_t>> ranges) {
+  std::lock_guard<std::mutex> lk(g_lastout_mu);
+  for (const auto& e : g_lastout) {
+    if (!e.used || e.stream != st) continue;
+    for (const auto& r : ranges) {
+      const uintptr_t b = reinterpret_cast<uintptr_t>(r.first), end = b + r.second;
+      if (b < e.end && e.begin < end) return false;
+    }
+  }
+  return true;
+}
+
+// Record o as the last query output on stream st.
+void record_query_output(cudaStream_t st, const void* o, size_t bytes) {
   std::lock_guard<std::mutex> lk(g_lastout_mu);
   LastOut* slot = nullptr;
   for (auto& e : g_lastout)
     if (e.used && e.stream == st) slot = &e;
-  bool clear = true;
-  if (slot) {
-    for (const void* p : {q, k, v}) {
-      const uintptr_t b = reinterpret_cast<uintptr_t>(p), e = b + bytes;
-      if (b < slot->end && slot->begin < e) clear = false;
-    }
-  } else {
-    for (auto& e : g_lastout)
-      if (!e.used) {
-        slot = &e;
-        break;
-      }
-    if (!slot) slot = &g_lastout[reinterpret_cast<uintptr_t>(st) % 16];
-  }
+  for (auto& e : g_lastout)
+    if (!slot && !e.used) slot = &e;
+  if (!slot) slot = &g_lastout[reinterpret_cast<uintptr_t>(st) % 16];
   slot->used = true;
   slot->stream = st;
   slot->begin = reinterpret_cast<uintptr_t>(o);
   slot->end = slot->begin + bytes;
-  return clear;
 }
 
 std::mutex g_setup_mu;
@@ -180,7 +183,7 @@ struct arl2_ctx {
   int frame = 0;
   bool maps_set = false;
   bool stall_next = false;        // failure-detection test hook (next query only)
-  bool overlap = false;           // queries may start behind the previous kernel (see the header)
+  bool overlap = false;           // calls may start behind the previous kernel (see the header)
   unsigned long long timeout_ns = kDefaultTimeoutNs;
   CUtensorMap tm_w[3];
   CUtensorMap tm_s;
@@ -279,8 +282,10 @@ arl2_status query_impl(arl2_ctx* c, const void* q, const void* k, const void* v,
   a.stall = c->stall_next ? 1 : 0;
   c->stall_next = false;
   set_plan(&a, c->qplan, c->qscratch, c->qflags, next_epoch(&c->qepoch));
-  const bool clear = note_query_output(st, q, k, v, o, c->act_elems() * 2);
-  return arl2::launch_query(true, *mq, *mk, *mv, c->tm_w[0], c->tm_s, *mo, a, st, c->overlap && clear) == cudaSuccess
+  const size_t act = c->act_elems() * 2;
+  const bool dependent = c->overlap && clear_of_last_output(st, {{q, act}, {k, act}, {v, act}});
+  record_query_output(st, o, act);
+  return arl2::launch_query(true, *mq, *mk, *mv, c->tm_w[0], c->tm_s, *mo, a, st, dependent) == cudaSuccess
              ? ARL2_OK
              : ARL2_ERR_CUDA;
 }
@@ -315,7 +320,11 @@ arl2_status commit_impl(arl2_ctx* c, const void* k, const void* v, const float* 
   r.ngroups = c->ngroups;
   r.BH = c->B * c->H;
   r.inv_T = a.inv_T;
-  if (arl2::launch_commit(*mk, *mv, c->tm_w[1], c->tm_w[2], c->tm_s, a, r, st) != cudaSuccess) return ARL2_ERR_CUDA;
+  const size_t act = c->act_elems() * 2, gate = (size_t)c->B * c->H * c->T * 4;
+  const bool dependent =
+      c->overlap && clear_of_last_output(st, {{k, act}, {v, act}, {alpha, gate}, {beta, gate}});
+  if (arl2::launch_commit(*mk, *mv, c->tm_w[1], c->tm_w[2], c->tm_s, a, r, st, dependent) != cudaSuccess)
+    return ARL2_ERR_CUDA;
   c->cur ^= 1;
   ++c->frame;
   return ARL2_OK;
@@ -489,7 +498,7 @@ arl2_status arl2_get_status(arl2_ctx* c) {
   return read_status(c->err);
 }
 
-arl2_status arl2_set_query_overlap(arl2_ctx* c, int enable) {
+arl2_status arl2_set_launch_overlap(arl2_ctx* c, int enable) {
   if (!c) return ARL2_ERR_INVALID_ARG;
   c->overlap = enable != 0;
   return ARL2_OK;

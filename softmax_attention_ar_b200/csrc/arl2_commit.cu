@@ -351,10 +351,21 @@ cudaError_t commit_setup() {
 
 cudaError_t launch_commit(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const CUtensorMap& tm_wk,
                           const CUtensorMap& tm_wv, const CUtensorMap& tm_s, const CommitArgs& a,
-                          const ReduceArgs& r, cudaStream_t stream) {
-  const dim3 grid(a.ngroups, a.H, a.B);
-  arl2_commit_partial_kernel<<<grid, 192, kSmemBytes, stream>>>(tm_k, tm_v, tm_wk, tm_wv, tm_s, a);
-  cudaError_t e = cudaGetLastError();
+                          const ReduceArgs& r, cudaStream_t stream, bool dependent) {
+  // As a programmatic dependent, the partial kernel may start while the preceding kernel (a
+  // query) still runs: it reads S_{N-1}, k, v and the gates, none of which a query writes, and
+  // writes only its own scratch. The reduce kernel, which writes S_N, is launched normally.
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(a.ngroups, a.H, a.B);
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = dependent ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, arl2_commit_partial_kernel, tm_k, tm_v, tm_wk, tm_wv, tm_s, a);
   if (e != cudaSuccess) return e;
   const dim3 rgrid((r.d * r.d / 4 + 255) / 256, r.BH);
   arl2_commit_reduce_kernel<<<rgrid, 256, 0, stream>>>(r);

@@ -137,5 +137,6 @@ extern "C" arl2_status arl2_frame_commit_noalloc(int B, int H, int T, int d, con
   r.ngroups = ngroups;
   r.BH = static_cast<int>(bh);
   r.inv_T = a.inv_T;
-  return arl2::launch_commit(tm_k, tm_v, tm_wk, tm_wv, tm_s, a, r, st) == cudaSuccess ? ARL2_OK : ARL2_ERR_CUDA;
+  return arl2::launch_commit(tm_k, tm_v, tm_wk, tm_wv, tm_s, a, r, st, false) == cudaSuccess ? ARL2_OK
+                                                                                       : ARL2_ERR_CUDA;
 }

@@ -239,14 +239,15 @@ def test_bounded_waits_report_a_timeout_and_leave_the_context_usable():
     assert max(o_errors(o_gpu, o_ref)) <= O_TOL
 
 
-def test_back_to_back_queries_overlapping_the_previous_kernel():
-    # With overlap on, each query is launched as a programmatic dependent of the one before
+def test_back_to_back_calls_overlapping_the_previous_kernel():
+    # With overlap on, each call is launched as a programmatic dependent of the kernel before
     # it (its CTAs start while the previous query's last CTAs still run). Checked: four
     # queries into one output buffer (the last one must win), four into separate buffers,
-    # and a query whose q is the previous query's output (the guard launches it normally).
+    # a query whose q is the previous query's output (the guard launches it normally), and
+    # a commit right behind a query, followed by a query that reads the new state.
     B, T, H, d = 1, 1560, 4, 128
     c = Case(B, T, H, d, config=116)
-    c.gpu.set_query_overlap(True)
+    c.gpu.set_launch_overlap(True)
     host = [c.inputs(0, p) for p in range(4)]
     dev = [tuple(dev_bf16(x) for x in qkv) for qkv in host]
     rows = sample_rows(T, 32, seed=7)
@@ -266,6 +267,12 @@ def test_back_to_back_queries_overlapping_the_previous_kernel():
     q2 = o1.view(torch.int16).cpu().numpy().view(np.uint16)
     ref2 = c.ref.query(synth.bf16_to_f64(q2), synth.bf16_to_f64(host[1][1]), synth.bf16_to_f64(host[1][2]), rows=rows)
     assert max(o_errors(host_f64(o2)[:, rows], ref2)) <= O_TOL
+    # A commit right behind a query also overlaps it; then a query must see the new state.
+    c.gpu.query(*dev[2], out=outs[0])
+    s_gpu, s_ref = c.commit(0)
+    assert s_error(s_gpu, s_ref) <= S_TOL
+    o_gpu, o_ref = c.query(1, 0, rows=rows)
+    assert max(o_errors(o_gpu, o_ref)) <= O_TOL
     assert c.gpu.status() == arl2.ARL2_OK
 
 
