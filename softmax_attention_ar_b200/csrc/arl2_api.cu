@@ -351,13 +351,7 @@ arl2_status arl2_create(int H, int T, int d_k, int d_v, int B, arl2_ctx** out) {
   c->d = d_k;
   c->device = dev;
   c->num_sms = sms;
-  // Commit work split: about one CTA per SM, each taking whole 128-token chunks.
-  const int nchunks = (T + 127) / 128;
-  const long long total = (long long)nchunks * H * B;
-  int cpg = (int)std::max<long long>(1, (total + sms - 1) / sms);
-  cpg = std::min(cpg, nchunks);
-  c->ngroups = (nchunks + cpg - 1) / cpg;
-  c->chunks_per_group = (nchunks + c->ngroups - 1) / c->ngroups;
+  arl2::commit_split(T, H, B, sms, &c->chunks_per_group, &c->ngroups);
   const size_t dd = (size_t)d_k * d_k;
   bool ok = true;
   for (int i = 0; i < 3 && ok; ++i) ok = dev_alloc(&c->W[i], (size_t)H * dd, &c->bytes);

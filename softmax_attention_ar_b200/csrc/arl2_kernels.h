@@ -42,13 +42,13 @@ QueryPlan plan_query(int B, int H, int T, int kv_len, int num_sms);
 size_t query_scratch_floats(const QueryPlan& p);   // part_o + part_ml
 size_t query_flag_count(const QueryPlan& p);       // flags
 
-// One commit, first kernel: per (group of 128-token chunks, head, batch) partial U and
-// partial sum of alpha.
+// One commit: per (group of 128-token chunks, head, batch) CTA; the groups of a (batch, head)
+// form a cluster that reduces U in distributed shared memory.
 struct CommitArgs {
   const float* alpha;     // [B, H, T]
   const float* beta;      // [B, H, T]
-  float* part;            // [B*H*ngroups, d, d] partial K'^T diag(beta/T) (V' - K'S)
-  float* alpha_part;      // [B*H*ngroups] partial sums of alpha
+  float* part;            // unused (the cluster reduces in shared memory)
+  float* alpha_part;      // unused
   int T, B, H, d;
   int chunks_per_group, ngroups;
   int state_slot;         // state buffer read (S_{N-1})
@@ -57,7 +57,8 @@ struct CommitArgs {
   unsigned long long timeout_ns;
 };
 
-// Second kernel: S_N = abar * S_{N-1} + sum of partials, fp32 plus its bf16 copy.
+// The commit's output side: S_N = abar * S_{N-1} + sum of the groups' U, fp32 plus its
+// bf16 copy.
 struct ReduceArgs {
   const float* part;
   const float* alpha_part;
@@ -76,6 +77,9 @@ bool encode_mat_map(CUtensorMap* m, const void* ptr, int n, int d);
 
 size_t query_smem_bytes();
 size_t commit_smem_bytes();
+// The commit's work split: 128-token chunks in groups, one CTA per group; the groups of one
+// (batch, head) form one cluster (at most 8 CTAs) and no group is empty.
+void commit_split(int T, int H, int B, int sms, int* chunks_per_group, int* ngroups);
 cudaError_t query_setup();   // per-device function attributes
 cudaError_t commit_setup();
 

@@ -71,14 +71,9 @@ extern "C" arl2_status arl2_frame_commit_noalloc(int B, int H, int T, int d, con
   const arl2_status ds = static_cast<arl2_status>(arl2::prepare_device(&dev, &sms));
   if (ds != ARL2_OK) return ds;
 
-  // The same work split as a context's commit: about one CTA per SM, whole 128-token chunks.
-  const int nchunks = (T + 127) / 128;
-  const long long total = static_cast<long long>(nchunks) * H * B;
-  int cpg = static_cast<int>((total + sms - 1) / sms);
-  if (cpg < 1) cpg = 1;
-  if (cpg > nchunks) cpg = nchunks;
-  int ngroups = (nchunks + cpg - 1) / cpg;
-  cpg = (nchunks + ngroups - 1) / ngroups;
+  // The same work split as a context's commit.
+  int cpg = 1, ngroups = 1;
+  arl2::commit_split(T, H, B, sms, &cpg, &ngroups);
 
   // Scratch layout: status word | S_{N-1} bf16 | S_{N-1} fp32 (discarded) | S_N bf16 (discarded) |
   // partial U | partial sum of alpha.

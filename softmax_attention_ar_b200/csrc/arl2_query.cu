@@ -130,13 +130,6 @@ struct Smem {
   __device__ uint32_t v(int s) const { return tiles + kVOff + s * kTileBytes; }
 };
 
-// One arrival for the calling warp, after all of its lanes got here (their earlier
-// memory operations are ordered before it).
-__device__ __forceinline__ void warp_arrive(uint32_t bar) {
-  __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-}
-
 // Rendezvous of the 8 softmax warps with a bounded wait (no hang if a warp aborted).
 __device__ __forceinline__ bool group_sync(uint32_t bar, uint32_t& phase, const Guard& g) {
   warp_arrive(bar);
