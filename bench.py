@@ -210,6 +210,62 @@ def cpu_baseline(budget_s: float = 15.0):
                       f"fp64 numpy/BLAS, {os.cpu_count()} host cores"}
 
 
+def kv_cache_baseline(frames, dev, layer_ms_per_frame, layer_bytes):
+    """The growing-KV-cache baseline the layer replaces (softmax attention of the newest frame
+    over every cached frame), on the same seeded q, k, v: time for the 4 queries of frame N
+    (CUDA events, mean of 3) and its KV memory, at N = 21, 60 and 120 cached frames."""
+    import torch
+
+    from softmax_attention_ar_b200.arl2 import KVCacheBaseline
+    Ns = (21, 60, 120)
+    base = KVCacheBaseline(H, T, D, B, max_frames=max(Ns))
+    o = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    frame_kv = B * T * H * D * 2 * 2
+    rows = []
+    for N in Ns:
+        base.reset()
+        for f in range(N - 1):
+            _, k, v = frames[f % CYCLE][0][QUERIES]
+            base.commit(k, v)
+        passes = frames[(N - 1) % CYCLE][0]
+        for p in range(QUERIES):                       # warm-up
+            base.query(*passes[p], out=o)
+        st, en = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        st.record(stream)
+        for _ in range(3):
+            for p in range(QUERIES):
+                base.query(*passes[p], out=o)
+        en.record(stream)
+        torch.cuda.synchronize()
+        rows.append({"N": N, "queries_ms_per_frame": st.elapsed_time(en) / 3, "kv_bytes": N * frame_kv})
+    status = base.status()
+    allocated = base.memory_bytes
+    base.close()
+    return {"what": "softmax attention of each frame's 4 queries over all N cached frames (growing KV cache), "
+                    "same kernel main loop; time excludes the cache appends",
+            "frames": rows, "allocated_bytes": allocated, "status": status,
+            "arl2_ms_per_frame": layer_ms_per_frame, "arl2_state_bytes": layer_bytes}
+
+
+def max_over_ranks(values, device, world):
+    """Each rank's timings -> the maximum over ranks, elementwise (the job is as slow as its
+    slowest rank). Uses the default process group when world > 1."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_rate(world, frames_per_rank, elapsed_ms):
+    """Whole-job frames/s: every rank's frames over the slowest rank's time."""
+    return world * frames_per_rank / (elapsed_ms / 1e3)
+
+
 def run_reference(args, rank, world):
     """Reference arm: the fp64 oracle on the host cores, same metric and workload."""
     if rank != 0:
@@ -288,6 +344,13 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     q_ms = [ev[2 * p].elapsed_time(ev[2 * p + 1]) for ev in ev_all for p in range(QUERIES)]
     c_ms = [ev[2 * QUERIES].elapsed_time(ev[2 * QUERIES + 1]) for ev in ev_all]
+    # Streaming: the layer's per-frame time must not grow with the frame count.
+    f_us = np.array([1e3 * sum(ev[2 * j].elapsed_time(ev[2 * j + 1]) for j in range(QUERIES + 1)) for ev in ev_all])
+    edge = max(1, min(50, len(f_us) // 4))
+    stream_info = {"frames": len(f_us), "us_per_frame_first": float(f_us[:edge].mean()),
+                   "us_per_frame_last": float(f_us[-edge:].mean()),
+                   "slope_us_per_frame": float(np.polyfit(np.arange(len(f_us)), f_us, 1)[0]) if len(f_us) > 1 else 0.0,
+                   "state_bytes_constant": layer.memory_bytes}
     status = layer.status()
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
@@ -323,14 +386,11 @@ def run_ours(args, rank, world, local_rank):
     d2h = QUERIES * act
 
     # Max over ranks.
-    t = torch.tensor([elapsed_ms, e2e_ms], device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    elapsed_ms, e2e_ms = t.tolist()
+    elapsed_ms, e2e_ms = max_over_ranks([elapsed_ms, e2e_ms], dev, world)
     if rank != 0:
         return
-    value = world * B * args.steps / (elapsed_ms / 1e3)
-    e2e_value = world * B * e2e_steps / (e2e_ms / 1e3) if e2e_steps else None
+    value = job_rate(world, B * args.steps, elapsed_ms)
+    e2e_value = job_rate(world, B * e2e_steps, e2e_ms) if e2e_steps else None
     peaks = _peaks()
     q_mean_s = statistics.mean(q_ms) / 1e3
     c_mean_s = statistics.mean(c_ms) / 1e3
@@ -357,6 +417,9 @@ def run_ours(args, rank, world, local_rank):
         "launch_overlap": "queries and commits launched as programmatic dependents of the kernel before them",
         "clocks": clocks.summary(),
     }
+    line["stream"] = stream_info
+    if not args.no_kv_baseline:
+        line["kv_cache_baseline"] = kv_cache_baseline(frames, dev, elapsed_ms / args.steps, layer.memory_bytes)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     print(json.dumps(line), flush=True)
@@ -371,6 +434,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer (e2e) measurement")
+    ap.add_argument("--no-kv-baseline", action="store_true", help="skip the growing-KV-cache comparison")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

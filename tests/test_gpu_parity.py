@@ -61,9 +61,10 @@ def test_maximum_tokens_per_frame():
     c.run(frames=2, queries=1, rows=sample_rows(4096))
 
 
-@pytest.mark.parametrize("B,T", [(1, 390), (4, 3600)])
+@pytest.mark.parametrize("B,T", [(1, 390), (4, 390), (4, 1560), (1, 3600), (4, 3600)])
 def test_sweep_shapes(B, T):
-    # Token/batch sweep shapes, H=12, d=128; the largest is checked on sampled rows.
+    # Token/batch sweep shapes, H=12, d=128 (T=1560 at B=1 is the 480p test); shapes above
+    # 400 tokens are checked on sampled rows.
     c = Case(B=B, T=T, H=12, d=128, config=3)
     rows = None if T <= 400 else sample_rows(T, n=24)
     c.run(frames=2, queries=2 if rows is None else 1, rows=rows)
