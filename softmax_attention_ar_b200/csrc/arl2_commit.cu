@@ -180,11 +180,8 @@ __device__ bool row_role(const Smem& sm, uint32_t tmem, const CommitArgs& a, int
     tc_fence_after();
     {
       uint32_t kv[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + col_kp(i) + 32u * c, kv[c]);
-      tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < 4; ++c) reg_fence(kv[c]);
+      tmem_ld32x2_wait(tmem + lane_off + col_kp(i), kv[0], tmem + lane_off + col_kp(i) + 32u, kv[1]);
+      tmem_ld32x2_wait(tmem + lane_off + col_kp(i) + 64u, kv[2], tmem + lane_off + col_kp(i) + 96u, kv[3]);
       float ss = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
@@ -214,9 +211,7 @@ __device__ bool row_role(const Smem& sm, uint32_t tmem, const CommitArgs& a, int
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       uint32_t vp[32];
-      tmem_ld32(tmem + lane_off + kColVp + 32u * c, vp);
-      tmem_wait_ld();
-      reg_fence(vp);
+      tmem_ld32_wait(tmem + lane_off + kColVp + 32u * c, vp);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         float y[8];
@@ -337,9 +332,7 @@ __global__ void __launch_bounds__(kThreadsC, 1)
         if (32 * c >= d) break;
         uint32_t u[32];
         if (nc > 0) {
-          tmem_ld32(tmem + lane_off + kColU + 32u * c, u);
-          tmem_wait_ld();
-          reg_fence(u);
+          tmem_ld32_wait(tmem + lane_off + kColU + 32u * c, u);
         } else {
 #pragma unroll
           for (int e = 0; e < 32; ++e) u[e] = 0u;

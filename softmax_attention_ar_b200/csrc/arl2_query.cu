@@ -501,14 +501,13 @@ __device__ __forceinline__ void merge_rows(const QueryArgs& a, const Seg& sg, ui
   const int t_row = sg.qt * kRows + static_cast<int>(r);
   const bool row_ok = t_row < a.T;
   uint16_t* out_row = a.o + ((static_cast<size_t>(sg.b) * a.T + t_row) * a.H + sg.h) * a.d + c0;
-  // Four passes of 16 columns: the TMEM loads (O, and O_inter for the layer) are issued
-  // first, the other records are read while they are in flight.
+  // Four passes of 16 columns: the other records first, then the TMEM loads (O, and
+  // O_inter for the layer) with their wait right behind them. No code sits between a TMEM
+  // load and its wait: the load's destination registers are undefined until the wait, and
+  // anything in between gives the compiler room to copy them early.
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     if (16 * c >= ncols) break;
-    uint32_t ov[16], xv[16];
-    tmem_ld16(tO + c0 + 16u * c, ov);
-    if (kHybrid) tmem_ld16(tX + c0 + 16u * c, xv);
     float4 acc[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -527,9 +526,11 @@ __device__ __forceinline__ void merge_rows(const QueryArgs& a, const Seg& sg, ui
         }
       }
     }
-    tmem_wait_ld();
-    reg_fence16(ov);
-    if (kHybrid) reg_fence16(xv);
+    uint32_t ov[16], xv[16];
+    if (kHybrid)
+      tmem_ld16x2_wait(tO + c0 + 16u * c, ov, tX + c0 + 16u * c, xv);
+    else
+      tmem_ld16_wait(tO + c0 + 16u * c, ov);
     float y[16];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -556,6 +557,9 @@ __device__ __forceinline__ void merge_rows(const QueryArgs& a, const Seg& sg, ui
       dst[0] = w0;
       dst[1] = w1;
     }
+    // Rows past T (a ragged last tile) skip the stores: reconverge the warp before the next
+    // pass's warp-wide TMEM loads (.sync.aligned), whatever the compiler made of the branch.
+    __syncwarp();
   }
 }
 
@@ -566,7 +570,9 @@ __device__ __forceinline__ void merge_rows(const QueryArgs& a, const Seg& sg, ui
 // range, so those records are normally published long before. Any other segment stores
 // its partial record (O_acc, running max m, sum l) and the publisher warp raises the
 // record's flag. Loads are issued in batches so their latencies overlap. Kept out of line
-// so its registers do not compete with the softmax loop. Returns false if a wait gave up.
+// so its registers do not compete with the softmax loop; the launch arguments it reads stay
+// in parameter space (the kernel takes them as a grid constant), not in a per-thread copy
+// in local memory. Returns false if a wait gave up.
 template <bool kHybrid>
 __device__ __noinline__ bool segment_epilogue(const Smem& sm, const QueryArgs& a, const Seg& sg, uint32_t r, int half,
                                               int c0, int ncols, uint32_t tO, uint32_t tX, float m, float l_row,
@@ -585,9 +591,7 @@ __device__ __noinline__ bool segment_epilogue(const Smem& sm, const QueryArgs& a
     for (int c = 0; c < 4; ++c) {
       if (16 * c >= ncols) break;
       uint32_t ov[16];
-      tmem_ld16(tO + c0 + 16u * c, ov);
-      tmem_wait_ld();
-      reg_fence16(ov);
+      tmem_ld16_wait(tO + c0 + 16u * c, ov);
 #pragma unroll
       for (int q = 0; q < 4; ++q)
         *quad_ptr(a.part_o, slot, q0 + 4 * c + q, r) =
@@ -738,11 +742,7 @@ __device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const 
       // This half's scores, then the row max: the two warps holding these rows (one per
       // half) swap their half-row maxima. Each half reads and writes only its own columns.
       uint32_t sv[2][32];
-      tmem_ld32(tS + c0, sv[0]);
-      tmem_ld32(tS + c0 + 32, sv[1]);
-      tmem_wait_ld();
-      reg_fence(sv[0]);
-      reg_fence(sv[1]);
+      tmem_ld32x2_wait(tS + c0, sv[0], tS + c0 + 32, sv[1]);
       float h0, h1;
       if (!pair_swap(pair_bar, xch, nx, half, r, half_max(sv, c0, valid), h0, h1, g)) return;
       const float mt = fmaxf(h0, h1) * a.scale_log2;
@@ -762,9 +762,7 @@ __device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const 
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t ov[16];
-          tmem_ld16(tO + c0 + 16u * c, ov);
-          tmem_wait_ld();
-          reg_fence16(ov);
+          tmem_ld16_wait(tO + c0 + 16u * c, ov);
 #pragma unroll
           for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
           tmem_st16(tO + c0 + 16u * c, ov);
@@ -795,11 +793,7 @@ __device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const 
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t x0[16], x1[16], pk[16];
-        tmem_ld16(tY + c0 + 32u * h, x0);
-        tmem_ld16(tY + c0 + 32u * h + 16u, x1);
-        tmem_wait_ld();
-        reg_fence16(x0);
-        reg_fence16(x1);
+        tmem_ld16x2_wait(tY + c0 + 32u * h, x0, tY + c0 + 32u * h + 16u, x1);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           pk[i] = pack_bf16x2(__uint_as_float(x0[2 * i]), __uint_as_float(x0[2 * i + 1]));
@@ -829,7 +823,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     arl2_query_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
                       const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_o,
-                      const QueryArgs a) {
+                      const __grid_constant__ QueryArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t tiles = smem_u32(smem_raw);
   if (tiles & 1023u) {   // the swizzled tiles need a 1 KiB-aligned base: report, do nothing
