@@ -413,7 +413,7 @@ def run_ours(args, rank, world, local_rank):
                     "commit_tflops": COMMIT_FLOPS / c_mean_s / 1e12},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
-        "gpu_launches": args.steps * (QUERIES * 1 + 2),
+        "gpu_launches": args.steps * (QUERIES + 1),   # per frame: the query launches and one commit
         "launch_overlap": "queries and commits launched as programmatic dependents of the kernel before them",
         "clocks": clocks.summary(),
     }
