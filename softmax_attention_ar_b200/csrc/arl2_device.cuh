@@ -56,6 +56,27 @@ __device__ __forceinline__ void raise_timeout(const Guard& g) {
   atomicOr(g.err, kErrTimeoutBit);
 }
 
+// Time spent in one wait, summed from %globaltimer between consecutive polls. A step
+// counts as at most kMaxStepNs, and a read that goes backwards counts as zero, so a jump of
+// the timer (or an unsigned wrap of a difference) can never end a short wait as a timeout;
+// the sum never exceeds the real time waited. The poll count is a backstop in case the
+// timer stalls.
+struct WaitClock {
+  static constexpr uint64_t kMaxStepNs = 1000000ull;       // 1 ms
+  static constexpr uint32_t kMaxPolls = 1u << 31;
+  uint64_t prev, waited = 0;
+  uint32_t polls = 0;
+  __device__ WaitClock() : prev(globaltimer()) {}
+  // Whether the wait has gone on longer than limit_ns.
+  __device__ bool expired(uint64_t limit_ns) {
+    const uint64_t now = globaltimer();
+    const uint64_t step = now > prev ? now - prev : 0ull;
+    prev = now;
+    waited += step < kMaxStepNs ? step : kMaxStepNs;
+    return waited > limit_ns || ++polls > kMaxPolls;
+  }
+};
+
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
@@ -86,11 +107,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // of the CTA aborted.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const Guard& g) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
+  WaitClock clock;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*g.abort) return false;
-    if (globaltimer() - t0 > g.timeout_ns) {
+    if (clock.expired(g.timeout_ns)) {
       raise_timeout(g);
       return false;
     }
@@ -103,9 +124,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const G
 constexpr uint64_t kDrainTimeoutNs = 2000000000ull;
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
+  WaitClock clock;
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer() - t0 > kDrainTimeoutNs) return false;
+    if (clock.expired(kDrainTimeoutNs)) return false;
   }
   return true;
 }

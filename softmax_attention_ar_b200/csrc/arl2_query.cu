@@ -161,10 +161,10 @@ __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
 }
 __device__ __forceinline__ bool wait_flag(const int* f, int value, const Guard& g) {
   if (ld_acquire_gpu(f) == value) return true;
-  const uint64_t t0 = globaltimer();
+  WaitClock clock;
   while (ld_acquire_gpu(f) != value) {
     if (*g.abort) return false;
-    if (globaltimer() - t0 > g.timeout_ns) {
+    if (clock.expired(g.timeout_ns)) {
       raise_timeout(g);
       return false;
     }
