@@ -39,6 +39,12 @@ __device__ __forceinline__ uint64_t globaltimer() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
+// The SM's cycle counter.
+__device__ __forceinline__ uint64_t sm_cycles() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%clock64;" : "=l"(t));
+  return t;
+}
 
 // ---------------------------------------------------------------------------------------
 // Failure handling: every wait is bounded by a time limit. When one runs out, the CTA
@@ -56,24 +62,29 @@ __device__ __forceinline__ void raise_timeout(const Guard& g) {
   atomicOr(g.err, kErrTimeoutBit);
 }
 
-// Time spent in one wait, summed from %globaltimer between consecutive polls. A step
-// counts as at most kMaxStepNs, and a read that goes backwards counts as zero, so a jump of
-// the timer (or an unsigned wrap of a difference) can never end a short wait as a timeout;
-// the sum never exceeds the real time waited. The poll count is a backstop in case the
-// timer stalls.
+// Time spent in one wait, measured two ways, and a wait is over only when both say so:
+//  - %globaltimer, summed between consecutive polls; a step counts as at most kMaxStepNs and
+//    a backwards read as zero, so a jump of the timer cannot end a short wait;
+//  - the SM's cycle counter, against the limit at kMaxCyclesPerNs (above the highest SM
+//    clock), so a global timer that runs fast for a while (catching up after the GPU sat
+//    idle) cannot end it either. At lower clocks the limit stretches in real time.
+// The poll count is a backstop in case both counters stall.
 struct WaitClock {
   static constexpr uint64_t kMaxStepNs = 1000000ull;       // 1 ms
+  static constexpr uint64_t kMaxCyclesPerNs = 2;           // 2 GHz
   static constexpr uint32_t kMaxPolls = 1u << 31;
   uint64_t prev, waited = 0;
+  uint64_t c0;
   uint32_t polls = 0;
-  __device__ WaitClock() : prev(globaltimer()) {}
+  __device__ WaitClock() : prev(globaltimer()), c0(sm_cycles()) {}
   // Whether the wait has gone on longer than limit_ns.
   __device__ bool expired(uint64_t limit_ns) {
     const uint64_t now = globaltimer();
     const uint64_t step = now > prev ? now - prev : 0ull;
     prev = now;
     waited += step < kMaxStepNs ? step : kMaxStepNs;
-    return waited > limit_ns || ++polls > kMaxPolls;
+    const uint64_t cycles = sm_cycles() - c0;
+    return (waited > limit_ns && cycles > kMaxCyclesPerNs * limit_ns) || ++polls > kMaxPolls;
   }
 };
 
