@@ -93,7 +93,8 @@ enum : int {
   kBarRecLoad = 35,   // the merge inputs of the CTA's last segment are staged in shared memory
   kBarLastPV = 36,    // the last P.V MMA of a staged merge's segment is done (V stages idle)
   kBarLastQK = 37,    // its last score MMA is done (K stages idle): staging may start
-  kNumBars = 38
+  kBarVGo = 38,       // the CTA's first K tile landed: the V ring may start filling (completes once)
+  kNumBars = 39
 };
 // Tiles at the (1 KiB-aligned) base of dynamic shared memory, then the control block.
 constexpr uint32_t kQOff = 0;
@@ -250,9 +251,13 @@ __device__ void producer(const Smem& sm, const CUtensorMap* tm_q, const CUtensor
     ++nseg;
     for (int j = sg.kb; j < sg.ke; ++j, ++ring) {
       // Start-up order: the first Q tile and first K tile go out alone (they gate the
-      // first score MMA); the rest of both rings fills once that K tile has landed. The
-      // first fill of K stage 0 is phase 0 of its barrier, waited on from the start.
-      if (ring == (kIsK ? 1u : 0u) && !mbar_wait_warp(sm.bar(kBarKFull), 0, g)) {
+      // first score MMA); the rest of both rings fills once that K tile has landed. The K
+      // producer waits for it right after issuing it (phase 0 of K stage 0, which only it
+      // refills, so the phase cannot pass unseen) and then opens the V ring through a
+      // barrier that completes once. The V producer must not wait on the K stage barrier
+      // itself: if it started late, that barrier could already be in its third phase, and
+      // a parity wait for phase 0 would then wait for a phase that never comes.
+      if (!kIsK && ring == 0 && !mbar_wait_warp(sm.bar(kBarVGo), 0, g)) {
         ok = false;
         break;
       }
@@ -267,6 +272,14 @@ __device__ void producer(const Smem& sm, const CUtensorMap* tm_q, const CUtensor
           tma_load_4d(tile_addr(s) + p * kPanelBytes, tm_kv, sm.bar(full0 + s), 64 * p, sg.h, j * kRows, sg.b);
       }
       ++nissued[s];
+      if (kIsK && ring == 0) {
+        if (!mbar_wait_warp(sm.bar(kBarKFull), 0, g)) {
+          ok = false;
+          break;
+        }
+        if (lead) mbar_arrive(sm.bar(kBarVGo));
+        __syncwarp();
+      }
     }
     if (ok && kHybrid && sg.head) {
       // The readout operand (Wq_h or the bf16 state copy S_h) follows the key tiles.
@@ -864,6 +877,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(sm.bar(kBarRecLoad), 1);
     mbar_init(sm.bar(kBarLastPV), 1);
     mbar_init(sm.bar(kBarLastQK), 1);
+    mbar_init(sm.bar(kBarVGo), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
