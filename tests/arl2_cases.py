@@ -66,6 +66,8 @@ class Case:
         """Run one query on both sides; return (o_gpu rows, o_ref rows) as fp64."""
         q, k, v = self.inputs(frame, pass_)
         o = self.gpu.query(dev_bf16(q), dev_bf16(k), dev_bf16(v))
+        st = self.gpu.status()
+        assert st == 0, f"frame {frame} pass {pass_}: device status {st} after the query (a bounded wait ran out)"
         o_gpu = host_f64(o)
         ref = self.ref.query(*(synth.bf16_to_f64(x) for x in (q, k, v)), rows=rows)
         if rows is not None:
@@ -77,6 +79,8 @@ class Case:
         _, k, v = self.inputs(frame, synth.CLEAN_PASS)
         a, b = self.gates(frame)
         self.gpu.commit(dev_bf16(k), dev_bf16(v), dev_f32(a), dev_f32(b))
+        st = self.gpu.status()
+        assert st == 0, f"frame {frame}: device status {st} after the commit (a bounded wait ran out)"
         s_ref = self.ref.commit(synth.bf16_to_f64(k), synth.bf16_to_f64(v), a, b)
         return host_f64(self.gpu.get_state()), s_ref
 

@@ -70,6 +70,38 @@ def test_sweep_shapes(B, T):
     c.run(frames=2, queries=2 if rows is None else 1, rows=rows)
 
 
+def test_calls_after_idle_pauses_on_split_tiles():
+    # Each launch follows a pause and fresh uploads, so the kernel's code is often cold when
+    # its first CTAs start. A start-up wait that could pass a barrier phase unseen stalled
+    # such CTAs until their wait limit ran out; their tiles, and the tiles whose records they
+    # owe, were then never written. Every call must report no timeout, and repeats must match
+    # bit for bit.
+    import time
+    B, T, H, d = 4, 1560, 12, 128
+    wq, wk, wv = synth.feature_maps(0, 116, H, d)
+    first = None
+    for rep in range(3):
+        layer = arl2.ARL2Layer(H, T, d, B)
+        layer.set_feature_maps(dev_bf16(wq), dev_bf16(wk), dev_bf16(wv))
+        outs = []
+        for f in range(2):
+            q, k, v = (dev_bf16(x) for x in synth.qkv(0, 116, f, 0, B, T, H, d))
+            outs.append(layer.query(q, k, v).float().cpu())
+            assert layer.status() == arl2.ARL2_OK, f"rep {rep} frame {f}: a bounded wait ran out in the query"
+            time.sleep(0.5)
+            _, k, v = (dev_bf16(x) for x in synth.qkv(0, 116, f, synth.CLEAN_PASS, B, T, H, d))
+            a, b = (dev_f32(x) for x in synth.gates(0, 116, f, B, H, T))
+            layer.commit(k, v, a, b)
+            assert layer.status() == arl2.ARL2_OK, f"rep {rep} frame {f}: a bounded wait ran out in the commit"
+            time.sleep(0.5)
+        layer.close()
+        if first is None:
+            first = outs
+        else:
+            for f, (x, y) in enumerate(zip(outs, first)):
+                assert torch.equal(x, y), f"rep {rep} frame {f}: output differs from the first repeat"
+
+
 # ------------------------------------------------------------------ closed forms on the GPU
 def test_queries_leave_the_state_bit_identical():
     c = Case(B=1, T=300, H=2, d=128, config=105)
