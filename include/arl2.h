@@ -174,9 +174,9 @@ void arl2_destroy(arl2_ctx* ctx);
  * The call allocates nothing. Its scratch is a fixed device array of
  * ARL2_NOALLOC_SCRATCH_BYTES inside the library. Every GPU that loads the library holds
  * that array until the process exits. Shapes whose scratch would exceed it return
- * ARL2_ERR_UNSUPPORTED before any work is enqueued. The need is about
- * B*H*d*d*8 + B*H*g*d*d*4 bytes, with g <= ceil(T/128) chunk groups; B=1, H=12, d=128,
- * T=1560 needs about 7.1 MB.
+ * ARL2_ERR_UNSUPPORTED before any work is enqueued. The need is about B*H*d*d*8 bytes
+ * (copies of S_prev and S_next; the chunk groups' partial sums meet in on-chip memory);
+ * B=1, H=12, d=128 needs about 1.6 MB, and d=128 fits up to B*H = 127.
  *
  * The first call on a device looks the array's device address up, with that device
  * current. Make that first call before any stream capture. All calls on a device share

@@ -170,8 +170,6 @@ struct arl2_ctx {
   uint16_t* W[3] = {};            // phi_q, phi_k, phi_v copies, [H, d, d]
   float* S[2] = {};               // fp32 state buffers, [B, H, d, d]
   uint16_t* S_bf16 = nullptr;     // [2][B, H, d, d] bf16 copies of S[0], S[1]
-  float* part = nullptr;          // [B*H*ngroups, d, d]
-  float* alpha_part = nullptr;    // [B*H*ngroups]
   unsigned int* err = nullptr;
   uint16_t* stage_bf16[4] = {};   // q, k, v, o staging for the host-buffer calls
   float* stage_f32[2] = {};       // alpha, beta staging
@@ -252,8 +250,6 @@ void free_ctx(arl2_ctx* c) {
   for (auto& p : c->W) cudaFree(p);
   for (auto& p : c->S) cudaFree(p);
   cudaFree(c->S_bf16);
-  cudaFree(c->part);
-  cudaFree(c->alpha_part);
   cudaFree(c->err);
   for (auto& p : c->stage_bf16) cudaFree(p);
   for (auto& p : c->stage_f32) cudaFree(p);
@@ -298,8 +294,6 @@ arl2_status commit_impl(arl2_ctx* c, const void* k, const void* v, const float* 
   arl2::CommitArgs a{};
   a.alpha = alpha;
   a.beta = beta;
-  a.part = c->part;
-  a.alpha_part = c->alpha_part;
   a.T = c->T;
   a.B = c->B;
   a.H = c->H;
@@ -311,14 +305,10 @@ arl2_status commit_impl(arl2_ctx* c, const void* k, const void* v, const float* 
   a.err = c->err;
   a.timeout_ns = c->timeout_ns;
   arl2::ReduceArgs r{};
-  r.part = c->part;
-  r.alpha_part = c->alpha_part;
   r.S_old = c->S[c->cur];
   r.S_new = c->S[c->cur ^ 1];
   r.S_new_bf16 = c->S_bf16 + (size_t)(c->cur ^ 1) * c->state_elems();
   r.d = c->d;
-  r.ngroups = c->ngroups;
-  r.BH = c->B * c->H;
   r.inv_T = a.inv_T;
   const size_t act = c->act_elems() * 2, gate = (size_t)c->B * c->H * c->T * 4;
   const bool dependent =
@@ -357,8 +347,6 @@ arl2_status arl2_create(int H, int T, int d_k, int d_v, int B, arl2_ctx** out) {
   for (int i = 0; i < 3 && ok; ++i) ok = dev_alloc(&c->W[i], (size_t)H * dd, &c->bytes);
   for (int i = 0; i < 2 && ok; ++i) ok = dev_alloc(&c->S[i], c->state_elems(), &c->bytes);
   ok = ok && dev_alloc(&c->S_bf16, 2 * c->state_elems(), &c->bytes);
-  ok = ok && dev_alloc(&c->part, (size_t)B * H * c->ngroups * dd, &c->bytes);
-  ok = ok && dev_alloc(&c->alpha_part, (size_t)B * H * c->ngroups, &c->bytes);
   ok = ok && dev_alloc(&c->err, 1, &c->bytes);
   for (int i = 0; i < 4 && ok; ++i) ok = dev_alloc(&c->stage_bf16[i], c->act_elems(), &c->bytes);
   for (int i = 0; i < 2 && ok; ++i) ok = dev_alloc(&c->stage_f32[i], (size_t)B * H * T, &c->bytes);

@@ -47,8 +47,6 @@ size_t query_flag_count(const QueryPlan& p);       // flags
 struct CommitArgs {
   const float* alpha;     // [B, H, T]
   const float* beta;      // [B, H, T]
-  float* part;            // unused (the cluster reduces in shared memory)
-  float* alpha_part;      // unused
   int T, B, H, d;
   int chunks_per_group, ngroups;
   int state_slot;         // state buffer read (S_{N-1})
@@ -58,14 +56,13 @@ struct CommitArgs {
 };
 
 // The commit's output side: S_N = abar * S_{N-1} + sum of the groups' U, fp32 plus its
-// bf16 copy.
+// bf16 copy. The groups' U and alpha sums meet in distributed shared memory; nothing goes
+// through global scratch.
 struct ReduceArgs {
-  const float* part;
-  const float* alpha_part;
   const float* S_old;     // [B*H, d, d]
   float* S_new;           // [B*H, d, d]
   uint16_t* S_new_bf16;   // [B*H, d, d]
-  int d, ngroups, BH;
+  int d;
   float inv_T;
 };
 

@@ -9,9 +9,9 @@
 // (k, v, the gates, phi_k, phi_v, S_{N-1}) and the output (S_N). The scratch the commit
 // needs lives in one file-scope device array of fixed size, g_commit_scratch. It holds:
 //   - the bf16 copy of S_{N-1} the MMAs read;
-//   - the per-group partial sums;
 //   - discarded copies (an fp32 copy of S_{N-1}, a bf16 copy of S_N);
 //   - a device status word, used when the caller passes none.
+// The groups' partial sums meet in distributed shared memory, so they need no scratch.
 // The array is part of the library's device image, so every GPU that loads the library
 // holds ARL2_NOALLOC_SCRATCH_BYTES of it until the process exits.
 //
@@ -75,15 +75,12 @@ extern "C" arl2_status arl2_frame_commit_noalloc(int B, int H, int T, int d, con
   int cpg = 1, ngroups = 1;
   arl2::commit_split(T, H, B, sms, &cpg, &ngroups);
 
-  // Scratch layout: status word | S_{N-1} bf16 | S_{N-1} fp32 (discarded) | S_N bf16 (discarded) |
-  // partial U | partial sum of alpha.
+  // Scratch layout: status word | S_{N-1} bf16 | S_{N-1} fp32 (discarded) | S_N bf16 (discarded).
   const size_t bh = static_cast<size_t>(B) * H, dd = static_cast<size_t>(d) * d;
   const size_t off_sprev = 256;
   const size_t off_sdisc = off_sprev + round256(bh * dd * 2);
   const size_t off_snext = off_sdisc + round256(bh * dd * 4);
-  const size_t off_part = off_snext + round256(bh * dd * 2);
-  const size_t off_apart = off_part + round256(bh * ngroups * dd * 4);
-  const size_t needed = off_apart + round256(bh * ngroups * 4);
+  const size_t needed = off_snext + round256(bh * dd * 2);
   if (needed > kScratchBytes) return ARL2_ERR_UNSUPPORTED;
 
   unsigned char* scratch = nullptr;
@@ -92,8 +89,6 @@ extern "C" arl2_status arl2_frame_commit_noalloc(int B, int H, int T, int d, con
   uint16_t* s_prev_bf16 = reinterpret_cast<uint16_t*>(scratch + off_sprev);
   float* s_prev_disc = reinterpret_cast<float*>(scratch + off_sdisc);
   uint16_t* s_next_bf16 = reinterpret_cast<uint16_t*>(scratch + off_snext);
-  float* part = reinterpret_cast<float*>(scratch + off_part);
-  float* apart = reinterpret_cast<float*>(scratch + off_apart);
   unsigned int* err = status ? status : reinterpret_cast<unsigned int*>(scratch);
 
   CUtensorMap tm_k, tm_v, tm_wk, tm_wv, tm_s;
@@ -110,8 +105,6 @@ extern "C" arl2_status arl2_frame_commit_noalloc(int B, int H, int T, int d, con
   arl2::CommitArgs a{};
   a.alpha = alpha;
   a.beta = beta;
-  a.part = part;
-  a.alpha_part = apart;
   a.T = T;
   a.B = B;
   a.H = H;
@@ -123,14 +116,10 @@ extern "C" arl2_status arl2_frame_commit_noalloc(int B, int H, int T, int d, con
   a.err = err;
   a.timeout_ns = kTimeoutNs;
   arl2::ReduceArgs r{};
-  r.part = part;
-  r.alpha_part = apart;
   r.S_old = S_prev;
   r.S_new = S_next;
   r.S_new_bf16 = s_next_bf16;
   r.d = d;
-  r.ngroups = ngroups;
-  r.BH = static_cast<int>(bh);
   r.inv_T = a.inv_T;
   return arl2::launch_commit(tm_k, tm_v, tm_wk, tm_wv, tm_s, a, r, st, false) == cudaSuccess ? ARL2_OK
                                                                                        : ARL2_ERR_CUDA;
