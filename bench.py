@@ -59,6 +59,11 @@ COMMIT_FLOPS = B * H * 4 * 2.0 * T * D * D                             # K Wk, V
 COMMIT_BYTES = B * T * H * D * 2 * 2 + 2 * B * H * T * 4 + B * H * D * D * 4 * 2 + 2 * H * D * D * 2
 
 
+# NVIDIA's dense (no 2:4 sparsity) bf16 tensor-core figure for one B200, for context only; the
+# roofline fraction uses the measured peak.
+DATASHEET_BF16_TFLOPS = 2250.0
+
+
 def _query_traffic():
     """DRAM bytes per query launch from the committed ncu capture, or None when the query
     kernel's sources changed since that capture (the summary records their SHA-256)."""
@@ -404,7 +409,8 @@ def run_ours(args, rank, world, local_rank):
                      "frac": q_tflops / peak, "traffic": _query_traffic(), "traffic_unit": "DRAM bytes per launch",
                      "kernel": "arl2_query_kernel (one query pass)",
                      "peak_source": f"bf16_tflops_sustained ({peaks['source']})",
-                     "frac_of_burst_peak": q_tflops / peaks["bf16_tflops"]},
+                     "frac_of_burst_peak": q_tflops / peaks["bf16_tflops"],
+                     "frac_of_datasheet_dense_bf16": q_tflops / DATASHEET_BF16_TFLOPS},
         "kernels": {"timed_steps": split_steps, "launch_overlap": "off in this split, on for value",
                     "query_us": 1e6 * q_mean_s, "query_p95_us": 1e3 * float(np.percentile(q_ms, 95)),
                     "commit_us": 1e6 * c_mean_s,
