@@ -69,7 +69,8 @@ bool aligned4(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 3u)
 // Small cache of activation maps keyed by base pointer: callers usually reuse buffers.
 struct MapCache {
   static constexpr int kSlots = 64;
-  int rows = 128;                 // box rows of the maps this cache makes
+  explicit MapCache(int box_rows = 128) : rows(box_rows) {}
+  int rows;                       // box rows of the maps this cache makes
   const void* ptr[kSlots] = {};
   CUtensorMap map[kSlots];
   int next = 0;
