@@ -92,10 +92,14 @@ arl2_status arl2_frame_commit(arl2_ctx* ctx, const arl2_bf16* k, const arl2_bf16
                               const float* alpha, const float* beta, arl2_stream stream);
 
 /* Host-buffer forms of the two calls above, for callers whose data is in host memory.
- * Each call enqueues, on the stream, the host-to-device copies into library-owned staging,
- * the kernels, and (for the query) the device-to-host copy of o. With pinned host memory
- * the call returns at once; the caller synchronises the stream before reading o_host or
- * reusing the inputs. With pageable memory the CUDA copies may block. */
+ * Each call copies its inputs into library-owned staging, runs the kernel on the stream
+ * and (for the query) copies o back. The copies run on two internal streams, and the
+ * calls take two staging sets by turns: one call's input copy overlaps the previous
+ * call's kernel and output copy. The stream waits for the call's copies, so its
+ * completion covers the whole call. With pinned host memory the call returns at once;
+ * the caller synchronises the stream before reading o_host or reusing the inputs. With
+ * pageable memory the CUDA copies may block. Calls on one context are made from one host
+ * thread at a time. */
 arl2_status arl2_frame_query_host(arl2_ctx* ctx, const arl2_bf16* q_host, const arl2_bf16* k_host,
                                   const arl2_bf16* v_host, arl2_bf16* o_host, arl2_stream stream);
 arl2_status arl2_frame_commit_host(arl2_ctx* ctx, const arl2_bf16* k_host, const arl2_bf16* v_host,

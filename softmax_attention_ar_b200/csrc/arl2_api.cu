@@ -172,8 +172,15 @@ struct arl2_ctx {
   float* S[2] = {};               // fp32 state buffers, [B, H, d, d]
   uint16_t* S_bf16 = nullptr;     // [2][B, H, d, d] bf16 copies of S[0], S[1]
   unsigned int* err = nullptr;
-  uint16_t* stage_bf16[4] = {};   // q, k, v, o staging for the host-buffer calls
-  float* stage_f32[2] = {};       // alpha, beta staging
+  // Host-buffer calls: two staging sets, used by turns, so that the copy of one call's inputs
+  // (on s_in) overlaps the previous call's kernel (on the caller's stream) and its output
+  // copy (on s_out). ev_in[s]: set s's inputs landed; ev_used[s]: the kernel that read set
+  // s is done; ev_out[s]: set s's output has been copied out.
+  uint16_t* stage_bf16[2][4] = {};   // q, k, v, o
+  float* stage_f32[2][2] = {};       // alpha, beta
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t ev_in[2] = {}, ev_used[2] = {}, ev_out[2] = {};
+  unsigned host_turn = 0;
   arl2::QueryPlan qplan{};        // stream-K split of the query kernel
   float* qscratch = nullptr;      // its partial records
   int* qflags = nullptr;          // their published flags
@@ -252,14 +259,24 @@ void free_ctx(arl2_ctx* c) {
   for (auto& p : c->S) cudaFree(p);
   cudaFree(c->S_bf16);
   cudaFree(c->err);
-  for (auto& p : c->stage_bf16) cudaFree(p);
-  for (auto& p : c->stage_f32) cudaFree(p);
+  for (auto& set : c->stage_bf16)
+    for (auto& p : set) cudaFree(p);
+  for (auto& set : c->stage_f32)
+    for (auto& p : set) cudaFree(p);
+  for (int i = 0; i < 2; ++i) {
+    if (c->ev_in[i]) cudaEventDestroy(c->ev_in[i]);
+    if (c->ev_used[i]) cudaEventDestroy(c->ev_used[i]);
+    if (c->ev_out[i]) cudaEventDestroy(c->ev_out[i]);
+  }
+  if (c->s_in) cudaStreamDestroy(c->s_in);
+  if (c->s_out) cudaStreamDestroy(c->s_out);
   cudaFree(c->qscratch);
   cudaFree(c->qflags);
   delete c;
 }
 
-arl2_status query_impl(arl2_ctx* c, const void* q, const void* k, const void* v, void* o, cudaStream_t st) {
+arl2_status query_impl(arl2_ctx* c, const void* q, const void* k, const void* v, void* o, cudaStream_t st,
+                       bool may_overlap = true) {
   const CUtensorMap* mq = c->acts.get(q, c->B, c->T, c->H, c->d);
   const CUtensorMap* mk = c->acts.get(k, c->B, c->T, c->H, c->d);
   const CUtensorMap* mv = c->acts.get(v, c->B, c->T, c->H, c->d);
@@ -280,7 +297,7 @@ arl2_status query_impl(arl2_ctx* c, const void* q, const void* k, const void* v,
   c->stall_next = false;
   set_plan(&a, c->qplan, c->qscratch, c->qflags, next_epoch(&c->qepoch));
   const size_t act = c->act_elems() * 2;
-  const bool dependent = c->overlap && clear_of_last_output(st, {{q, act}, {k, act}, {v, act}});
+  const bool dependent = may_overlap && c->overlap && clear_of_last_output(st, {{q, act}, {k, act}, {v, act}});
   record_query_output(st, o, act);
   return arl2::launch_query(true, *mq, *mk, *mv, c->tm_w[0], c->tm_s, *mo, a, st, dependent) == cudaSuccess
              ? ARL2_OK
@@ -288,7 +305,7 @@ arl2_status query_impl(arl2_ctx* c, const void* q, const void* k, const void* v,
 }
 
 arl2_status commit_impl(arl2_ctx* c, const void* k, const void* v, const float* alpha, const float* beta,
-                        cudaStream_t st) {
+                        cudaStream_t st, bool may_overlap = true) {
   const CUtensorMap* mk = c->acts.get(k, c->B, c->T, c->H, c->d);
   const CUtensorMap* mv = c->acts.get(v, c->B, c->T, c->H, c->d);
   if (!mk || !mv) return ARL2_ERR_CUDA;
@@ -312,8 +329,8 @@ arl2_status commit_impl(arl2_ctx* c, const void* k, const void* v, const float* 
   r.d = c->d;
   r.inv_T = a.inv_T;
   const size_t act = c->act_elems() * 2, gate = (size_t)c->B * c->H * c->T * 4;
-  const bool dependent =
-      c->overlap && clear_of_last_output(st, {{k, act}, {v, act}, {alpha, gate}, {beta, gate}});
+  const bool dependent = may_overlap && c->overlap &&
+                         clear_of_last_output(st, {{k, act}, {v, act}, {alpha, gate}, {beta, gate}});
   if (arl2::launch_commit(*mk, *mv, c->tm_w[1], c->tm_w[2], c->tm_s, a, r, st, dependent) != cudaSuccess)
     return ARL2_ERR_CUDA;
   c->cur ^= 1;
@@ -349,8 +366,10 @@ arl2_status arl2_create(int H, int T, int d_k, int d_v, int B, arl2_ctx** out) {
   for (int i = 0; i < 2 && ok; ++i) ok = dev_alloc(&c->S[i], c->state_elems(), &c->bytes);
   ok = ok && dev_alloc(&c->S_bf16, 2 * c->state_elems(), &c->bytes);
   ok = ok && dev_alloc(&c->err, 1, &c->bytes);
-  for (int i = 0; i < 4 && ok; ++i) ok = dev_alloc(&c->stage_bf16[i], c->act_elems(), &c->bytes);
-  for (int i = 0; i < 2 && ok; ++i) ok = dev_alloc(&c->stage_f32[i], (size_t)B * H * T, &c->bytes);
+  for (int s = 0; s < 2; ++s) {
+    for (int i = 0; i < 4 && ok; ++i) ok = dev_alloc(&c->stage_bf16[s][i], c->act_elems(), &c->bytes);
+    for (int i = 0; i < 2 && ok; ++i) ok = dev_alloc(&c->stage_f32[s][i], (size_t)B * H * T, &c->bytes);
+  }
   c->qplan = arl2::plan_query(B, H, T, T, sms);
   ok = ok && dev_alloc(&c->qscratch, arl2::query_scratch_floats(c->qplan), &c->bytes);
   ok = ok && dev_alloc(&c->qflags, arl2::query_flag_count(c->qplan), &c->bytes);
@@ -358,7 +377,13 @@ arl2_status arl2_create(int H, int T, int d_k, int d_v, int B, arl2_ctx** out) {
     free_ctx(c);
     return ARL2_ERR_OOM;
   }
-  ok = cudaMemset(c->S[0], 0, c->state_elems() * 4) == cudaSuccess &&
+  ok = cudaStreamCreateWithFlags(&c->s_in, cudaStreamNonBlocking) == cudaSuccess &&
+       cudaStreamCreateWithFlags(&c->s_out, cudaStreamNonBlocking) == cudaSuccess;
+  for (int i = 0; i < 2 && ok; ++i)
+    ok = cudaEventCreateWithFlags(&c->ev_in[i], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&c->ev_used[i], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&c->ev_out[i], cudaEventDisableTiming) == cudaSuccess;
+  ok = ok && cudaMemset(c->S[0], 0, c->state_elems() * 4) == cudaSuccess &&
        cudaMemset(c->S[1], 0, c->state_elems() * 4) == cudaSuccess &&
        cudaMemset(c->S_bf16, 0, 2 * c->state_elems() * 2) == cudaSuccess &&
        cudaMemset(c->qflags, 0, arl2::query_flag_count(c->qplan) * sizeof(int)) == cudaSuccess &&
@@ -406,14 +431,27 @@ arl2_status arl2_frame_query_host(arl2_ctx* c, const arl2_bf16* q, const arl2_bf
   if (!c->maps_set) return ARL2_ERR_STATE;
   cudaStream_t st = (cudaStream_t)stream;
   const size_t bytes = c->act_elems() * 2;
+  const int s = static_cast<int>(c->host_turn++ & 1u);
+  uint16_t* const* buf = c->stage_bf16[s];
   const arl2_bf16* src[3] = {q, k, v};
-  for (int i = 0; i < 3; ++i)
-    if (cudaMemcpyAsync(c->stage_bf16[i], src[i], bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
-      return ARL2_ERR_CUDA;
-  arl2_status s = query_impl(c, c->stage_bf16[0], c->stage_bf16[1], c->stage_bf16[2], c->stage_bf16[3], st);
-  if (s != ARL2_OK) return s;
-  return cudaMemcpyAsync(o, c->stage_bf16[3], bytes, cudaMemcpyDeviceToHost, st) == cudaSuccess ? ARL2_OK
-                                                                                                : ARL2_ERR_CUDA;
+  // Inputs in, once the kernel that last read this set is done.
+  bool ok = cudaStreamWaitEvent(c->s_in, c->ev_used[s], 0) == cudaSuccess;
+  for (int i = 0; i < 3 && ok; ++i)
+    ok = cudaMemcpyAsync(buf[i], src[i], bytes, cudaMemcpyHostToDevice, c->s_in) == cudaSuccess;
+  ok = ok && cudaEventRecord(c->ev_in[s], c->s_in) == cudaSuccess;
+  // The kernel, once they landed and this set's previous output has been copied out.
+  ok = ok && cudaStreamWaitEvent(st, c->ev_in[s], 0) == cudaSuccess &&
+       cudaStreamWaitEvent(st, c->ev_out[s], 0) == cudaSuccess;
+  if (!ok) return ARL2_ERR_CUDA;
+  arl2_status r = query_impl(c, buf[0], buf[1], buf[2], buf[3], st, false);
+  if (r != ARL2_OK) return r;
+  // Output out; the call completes on the caller's stream only with its output copied.
+  ok = cudaEventRecord(c->ev_used[s], st) == cudaSuccess &&
+       cudaStreamWaitEvent(c->s_out, c->ev_used[s], 0) == cudaSuccess &&
+       cudaMemcpyAsync(o, buf[3], bytes, cudaMemcpyDeviceToHost, c->s_out) == cudaSuccess &&
+       cudaEventRecord(c->ev_out[s], c->s_out) == cudaSuccess &&
+       cudaStreamWaitEvent(st, c->ev_out[s], 0) == cudaSuccess;
+  return ok ? ARL2_OK : ARL2_ERR_CUDA;
 }
 
 arl2_status arl2_frame_commit_host(arl2_ctx* c, const arl2_bf16* k, const arl2_bf16* v, const float* alpha,
@@ -422,12 +460,20 @@ arl2_status arl2_frame_commit_host(arl2_ctx* c, const arl2_bf16* k, const arl2_b
   if (!c->maps_set) return ARL2_ERR_STATE;
   cudaStream_t st = (cudaStream_t)stream;
   const size_t bytes = c->act_elems() * 2, gbytes = (size_t)c->B * c->H * c->T * 4;
-  if (cudaMemcpyAsync(c->stage_bf16[1], k, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(c->stage_bf16[2], v, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(c->stage_f32[0], alpha, gbytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(c->stage_f32[1], beta, gbytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
-    return ARL2_ERR_CUDA;
-  return commit_impl(c, c->stage_bf16[1], c->stage_bf16[2], c->stage_f32[0], c->stage_f32[1], st);
+  const int s = static_cast<int>(c->host_turn++ & 1u);
+  uint16_t* const* buf = c->stage_bf16[s];
+  float* const* gbuf = c->stage_f32[s];
+  bool ok = cudaStreamWaitEvent(c->s_in, c->ev_used[s], 0) == cudaSuccess &&
+            cudaMemcpyAsync(buf[1], k, bytes, cudaMemcpyHostToDevice, c->s_in) == cudaSuccess &&
+            cudaMemcpyAsync(buf[2], v, bytes, cudaMemcpyHostToDevice, c->s_in) == cudaSuccess &&
+            cudaMemcpyAsync(gbuf[0], alpha, gbytes, cudaMemcpyHostToDevice, c->s_in) == cudaSuccess &&
+            cudaMemcpyAsync(gbuf[1], beta, gbytes, cudaMemcpyHostToDevice, c->s_in) == cudaSuccess &&
+            cudaEventRecord(c->ev_in[s], c->s_in) == cudaSuccess &&
+            cudaStreamWaitEvent(st, c->ev_in[s], 0) == cudaSuccess;
+  if (!ok) return ARL2_ERR_CUDA;
+  arl2_status r = commit_impl(c, buf[1], buf[2], gbuf[0], gbuf[1], st, false);
+  if (r != ARL2_OK) return r;
+  return cudaEventRecord(c->ev_used[s], st) == cudaSuccess ? ARL2_OK : ARL2_ERR_CUDA;
 }
 
 arl2_status arl2_reset(arl2_ctx* c, arl2_stream stream) {

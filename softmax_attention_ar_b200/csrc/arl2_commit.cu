@@ -169,12 +169,21 @@ __device__ bool row_role(const Smem& sm, uint32_t tmem, const CommitArgs& a, int
   const float* alpha = a.alpha + bh * a.T;
   const float* beta = a.beta + bh * a.T;
   float asum = 0.f;
+  // This row's gates, loaded one chunk ahead so that their latency hides behind the
+  // previous chunk's work.
+  auto gate_at = [&](int i, float& coef, float& al) {
+    const int t = (c0 + i) * kRows + static_cast<int>(r);
+    const bool valid = i < nc && t < a.T;
+    coef = valid ? beta[t] * a.inv_T : 0.f;
+    al = valid ? alpha[t] : 0.f;
+  };
+  float coef_next, alpha_next;
+  gate_at(0, coef_next, alpha_next);
   for (int i = 0; i < nc; ++i) {
     const int st = i & 1;
-    const int t = (c0 + i) * kRows + static_cast<int>(r);
-    const bool valid = t < a.T;
-    const float coef = valid ? beta[t] * a.inv_T : 0.f;
-    if (valid) asum += alpha[t];
+    const float coef = coef_next;
+    asum += alpha_next;
+    gate_at(i + 1, coef_next, alpha_next);
     // K' = Kp / max(|Kp|, eps) -> bf16, over the K tile (its MMA has finished).
     if (!mbar_wait_warp(sm.bar(kBarProjK + st), (i >> 1) & 1, g)) return false;
     tc_fence_after();
@@ -373,22 +382,38 @@ __global__ void __launch_bounds__(kThreadsC, 1)
     float* S_new = rd.S_new + bh * dd;
     uint16_t* S_new_bf16 = rd.S_new_bf16 + bh * dd;
     const float4* recv = reinterpret_cast<const float4*>(gbase + kRecvOff);
+    // Up to kBatch items a thread per pass, their S_{N-1} loads issued together so that one
+    // L2 round trip covers them all (at 480p a single pass covers every item).
+    constexpr int kBatch = 4;
 #pragma unroll 1
-    for (int it = threadIdx.x; it < items; it += kThreadsC) {
-      const int lr = it / quads, q = it % quads, k = k0 + lr;
-      const float4 so = *reinterpret_cast<const float4*>(S_old + static_cast<size_t>(k) * d + 4 * q);
-      float4 acc = make_float4(abar * so.x, abar * so.y, abar * so.z, abar * so.w);
-#pragma unroll 1
-      for (int j = 0; j < G; ++j) {
-        const float4 u = recv[(j * 32 + q) * rows_per + lr];
-        acc.x += u.x;
-        acc.y += u.y;
-        acc.z += u.z;
-        acc.w += u.w;
+    for (int it0 = threadIdx.x; it0 < items; it0 += kBatch * kThreadsC) {
+      float4 so[kBatch];
+#pragma unroll
+      for (int e = 0; e < kBatch; ++e) {
+        const int it = it0 + e * kThreadsC;
+        if (it < items) {
+          const int lr = it / quads, q = it % quads;
+          so[e] = *reinterpret_cast<const float4*>(S_old + static_cast<size_t>(k0 + lr) * d + 4 * q);
+        }
       }
-      *reinterpret_cast<float4*>(S_new + static_cast<size_t>(k) * d + 4 * q) = acc;
-      *reinterpret_cast<uint2*>(S_new_bf16 + static_cast<size_t>(k) * d + 4 * q) =
-          make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+#pragma unroll
+      for (int e = 0; e < kBatch; ++e) {
+        const int it = it0 + e * kThreadsC;
+        if (it >= items) break;
+        const int lr = it / quads, q = it % quads, k = k0 + lr;
+        float4 acc = make_float4(abar * so[e].x, abar * so[e].y, abar * so[e].z, abar * so[e].w);
+#pragma unroll 1
+        for (int j = 0; j < G; ++j) {
+          const float4 u = recv[(j * 32 + q) * rows_per + lr];
+          acc.x += u.x;
+          acc.y += u.y;
+          acc.z += u.z;
+          acc.w += u.w;
+        }
+        *reinterpret_cast<float4*>(S_new + static_cast<size_t>(k) * d + 4 * q) = acc;
+        *reinterpret_cast<uint2*>(S_new_bf16 + static_cast<size_t>(k) * d + 4 * q) =
+            make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+      }
     }
   }
 

@@ -181,34 +181,66 @@ struct Seg {
   bool last;   // the CTA's last segment
 };
 
-struct Sched {
-  long long u, u1;
-  int nq, nkv, H;
-  __device__ Sched(const QueryArgs& a, int c) : nq(a.nq), nkv(a.nkv), H(a.H) {
-    u = static_cast<long long>(c) * a.units / a.num_ctas;
-    u1 = static_cast<long long>(c + 1) * a.units / a.num_ctas;
-  }
-  __device__ bool next(Seg& s) {
-    if (u >= u1) return false;
-    s.Q = static_cast<int>(u / nkv);
-    s.kb = static_cast<int>(u % nkv);
-    s.ke = static_cast<int>(min(static_cast<long long>(nkv), s.kb + (u1 - u)));
-    u = static_cast<long long>(s.Q) * nkv + s.ke;
-    const int bh = s.Q / nq;
-    s.qt = s.Q % nq;
-    s.b = bh / H;
-    s.h = bh % H;
-    s.head = s.kb == 0;
-    s.tail = s.ke == nkv;
-    s.last = u >= u1;
-    return true;
-  }
-};
-
 // The CTA whose unit range holds unit u.
 __device__ __forceinline__ int owner(long long u, const QueryArgs& a) {
   return static_cast<int>(((u + 1) * a.num_ctas - 1) / a.units);
 }
+
+// A CTA's walk over its unit range, one segment at a time. The divisions happen once, when
+// the walk is set up at kernel start (their latency hides behind the first loads); each
+// step then moves to the next query tile by increments, so no segment boundary waits on an
+// integer division. The two facts about tiles shared with other CTAs are fixed at set-up
+// too: only the range's first segment can lack key tile 0, and only its last can hold key
+// tile 0 without the last key tile.
+struct Sched {
+  long long u, u1;
+  int nq, nkv, H;
+  int Q, kb, qt, b, h;   // the tile and key tile of unit u
+  int first_rec;         // the first segment's record slot within its tile (this CTA - the tile's first CTA)
+  int last_nsegs;        // CTAs sharing the last segment's tile (counted from this one)
+  __device__ Sched(const QueryArgs& a, int c) : nq(a.nq), nkv(a.nkv), H(a.H) {
+    u = static_cast<long long>(c) * a.units / a.num_ctas;
+    u1 = static_cast<long long>(c + 1) * a.units / a.num_ctas;
+    Q = static_cast<int>(u / nkv);
+    kb = static_cast<int>(u % nkv);
+    const int bh = Q / nq;
+    qt = Q % nq;
+    b = bh / H;
+    h = bh % H;
+    first_rec = c - owner(static_cast<long long>(Q) * nkv, a);
+    const long long q_last = (u1 - 1) / nkv;
+    last_nsegs = owner(q_last * nkv + nkv - 1, a) - c + 1;
+  }
+  __device__ bool next(Seg& s) {
+    if (u >= u1) return false;
+    s.Q = Q;
+    s.kb = kb;
+    s.qt = qt;
+    s.b = b;
+    s.h = h;
+    const long long left = u1 - u;
+    s.ke = left < nkv - kb ? kb + static_cast<int>(left) : nkv;
+    u += s.ke - s.kb;
+    s.head = s.kb == 0;
+    s.tail = s.ke == nkv;
+    s.last = u >= u1;
+    if (s.tail) {   // on to key tile 0 of the next query tile
+      ++Q;
+      kb = 0;
+      if (++qt == nq) {
+        qt = 0;
+        if (++h == H) {
+          h = 0;
+          ++b;
+        }
+      }
+    } else {
+      kb = s.ke;   // only when the range ended inside the tile: there is no next segment
+    }
+    return true;
+  }
+};
+
 
 // Ring slot g: stage g % 3, used for the (g / 3)-th time. S buffers cycle the same way.
 __device__ __forceinline__ int ring_stage(uint32_t g) { return static_cast<int>(g % kStages); }
@@ -346,10 +378,7 @@ __device__ void mma_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, co
     const bool rd = kHybrid && sg.head;
     const uint32_t t0 = tile, n = sg.ke - sg.kb;
     bool staged = false;   // a staged merge: the K, then V, stages it uses are signalled idle
-    if (sg.head && !sg.tail) {
-      const long long first = static_cast<long long>(sg.Q) * a.nkv;
-      staged = staged_merge(owner(first + a.nkv - 1, a) - owner(first, a) + 1);
-    }
+    if (sg.head && !sg.tail) staged = staged_merge(sch.last_nsegs);   // the CTA's last segment
     const uint32_t r0 = ring, r_rd = ring + n;   // first key tile's ring slot, the readout operands' slot
     // Score tiles issued before the P.V loop: two. Afterwards the scores of tile t + 2 are
     // issued right behind the P.V MMA of tile t: they go to the buffer whose P was read by
@@ -587,19 +616,18 @@ __device__ __forceinline__ void merge_rows(const QueryArgs& a, const Seg& sg, ui
 // in parameter space (the kernel takes them as a grid constant), not in a per-thread copy
 // in local memory. Returns false if a wait gave up.
 template <bool kHybrid>
-__device__ __noinline__ bool segment_epilogue(const Smem& sm, const QueryArgs& a, const Seg& sg, uint32_t r, int half,
-                                              int c0, int ncols, uint32_t tO, uint32_t tX, float m, float l_row,
-                                              uint32_t& gphase, volatile int* merge_ok, const float* stage, int rs,
+__device__ __noinline__ bool segment_epilogue(const Smem& sm, const QueryArgs& a, const Seg& sg, int first_rec,
+                                              int last_nsegs, uint32_t r, int half, int c0, int ncols, uint32_t tO,
+                                              uint32_t tX, float m, float l_row, uint32_t& gphase,
+                                              volatile int* merge_ok, const float* stage, int rs,
                                               const CUtensorMap* tm_o, const Guard& g) {
   const int q0 = c0 / 4;   // this half's first column quad
   // First global write of this thread in the launch: a query launched as the programmatic
   // dependent of the previous one waits for it here (shared scratch, maybe the same output).
   griddep_wait();
-  const long long first = static_cast<long long>(sg.Q) * a.nkv;
-  const int c_first = owner(first, a);
   const size_t slot0 = static_cast<size_t>(sg.Q) * a.max_segs;
-  if (!sg.head) {
-    const size_t slot = slot0 + (static_cast<int>(blockIdx.x) - c_first);
+  if (!sg.head) {   // the CTA's first segment
+    const size_t slot = slot0 + first_rec;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       if (16 * c >= ncols) break;
@@ -622,7 +650,7 @@ __device__ __noinline__ bool segment_epilogue(const Smem& sm, const QueryArgs& a
   }
   // Head segment: the tile's other records (if any), then the merge. Warp 3 stages them
   // in shared memory when they fit; otherwise they are read from scratch here.
-  const int nsegs = sg.tail ? 1 : owner(first + a.nkv - 1, a) - c_first + 1;
+  const int nsegs = sg.tail ? 1 : last_nsegs;   // not a tail: the CTA's last segment
   const bool staged = staged_merge(nsegs);
   const int k1 = (rs + 1) % kStages, k2 = (rs + 2) % kStages;   // idle ring stages (see staged_merge)
   if (staged) {
@@ -677,8 +705,6 @@ __device__ void publisher(const Smem& sm, const QueryArgs& a, const Guard& g) {
   Sched sch(a, blockIdx.x);
   Seg sg;
   while (sch.next(sg)) {
-    const long long first = static_cast<long long>(sg.Q) * a.nkv;
-    const int c_first = owner(first, a);
     const size_t slot0 = static_cast<size_t>(sg.Q) * a.max_segs;
     const uint32_t n = sg.ke - sg.kb;
     const int ws = ring_stage(ring + n);   // the readout operands' stage
@@ -689,10 +715,10 @@ __device__ void publisher(const Smem& sm, const QueryArgs& a, const Guard& g) {
       griddep_wait();   // the previous launch may still poll this flag for its own epoch
       if (lead) {
         __threadfence();
-        atomicExch(a.flags + slot0 + (static_cast<int>(blockIdx.x) - c_first), a.epoch);
+        atomicExch(a.flags + slot0 + sch.first_rec, a.epoch);
       }
       __syncwarp();
-    } else if (!sg.tail && staged_merge(owner(first + a.nkv - 1, a) - c_first + 1)) {
+    } else if (!sg.tail && staged_merge(sch.last_nsegs)) {
       bool ok = true;
       if (lead) ok = wait_flag(a.flags + slot0 + 1, a.epoch, g);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
@@ -824,8 +850,8 @@ __device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const 
     tc_fence_after();
     float l0, l1;
     if (!pair_swap(pair_bar, xch, nx, half, r, l, l0, l1, g)) return;
-    if (!segment_epilogue<kHybrid>(sm, a, sg, r, half, c0, ncols, tO, tX, m, l0 + l1, gphase, merge_ok,
-                                   reinterpret_cast<const float*>(ctl - kTileRegion), rs, tm_o, g))
+    if (!segment_epilogue<kHybrid>(sm, a, sg, sch.first_rec, sch.last_nsegs, r, half, c0, ncols, tO, tX, m, l0 + l1,
+                                   gphase, merge_ok, reinterpret_cast<const float*>(ctl - kTileRegion), rs, tm_o, g))
       return;
     ++nseg;
   }
