@@ -366,9 +366,9 @@ arl2_status arl2_create(int H, int T, int d_k, int d_v, int B, arl2_ctx** out) {
   for (int i = 0; i < 2 && ok; ++i) ok = dev_alloc(&c->S[i], c->state_elems(), &c->bytes);
   ok = ok && dev_alloc(&c->S_bf16, 2 * c->state_elems(), &c->bytes);
   ok = ok && dev_alloc(&c->err, 1, &c->bytes);
-  for (int s = 0; s < 2; ++s) {
-    for (int i = 0; i < 4 && ok; ++i) ok = dev_alloc(&c->stage_bf16[s][i], c->act_elems(), &c->bytes);
-    for (int i = 0; i < 2 && ok; ++i) ok = dev_alloc(&c->stage_f32[s][i], (size_t)B * H * T, &c->bytes);
+  for (int set = 0; set < 2; ++set) {
+    for (int i = 0; i < 4 && ok; ++i) ok = dev_alloc(&c->stage_bf16[set][i], c->act_elems(), &c->bytes);
+    for (int i = 0; i < 2 && ok; ++i) ok = dev_alloc(&c->stage_f32[set][i], (size_t)B * H * T, &c->bytes);
   }
   c->qplan = arl2::plan_query(B, H, T, T, sms);
   ok = ok && dev_alloc(&c->qscratch, arl2::query_scratch_floats(c->qplan), &c->bytes);
