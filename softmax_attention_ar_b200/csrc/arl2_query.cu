@@ -694,8 +694,9 @@ __device__ __noinline__ bool segment_epilogue(const Smem& sm, const QueryArgs& a
 // device-scope fence, so a CTA that reads the flag (acquire) sees the whole record.
 // (2) For a staged merge (the CTA's last segment): waits for the other record's flag while
 // the segment runs, then bulk-copies that record into the idle K stages once the last score
-// MMA is done, and its (m, l) rows into an idle V stage once the last P.V MMA is done. Every barrier this warp waits on completes at
-// most once per launch, so a parity wait can never alias an earlier phase.
+// MMA is done, and its (m, l) rows into an idle V stage once the last P.V MMA is done.
+// Every barrier this warp waits on completes at most once per launch, so a parity wait can
+// never alias an earlier phase.
 template <bool kHybrid>
 __device__ void publisher(const Smem& sm, const QueryArgs& a, const Guard& g) {
   const bool lead = (threadIdx.x & 31) == 0;
