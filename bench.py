@@ -16,9 +16,17 @@ The bench prints one JSON line (rank 0):
   - value: whole-job frames/s, timed on the device with CUDA events between barriers.
   - e2e: the same metric through the host-buffer entry points. Each step copies its
     inputs from pinned host memory and its outputs back.
+  - repeats: the same timed window of K frames, repeated; median and spread of frames/s.
   - roofline: the query kernel's achieved TFLOP/s (algorithmic FLOPs / mean launch time,
     CUDA events on the launching stream, from a second timed region in which every launch
-    is bracketed by events and queries do not overlap) against the measured bf16 peak.
+    is bracketed by events and runs alone) against the measured bf16 burst peak (a kernel
+    timed alone). roofline_commit: the commit's achieved GB/s (algorithmic bytes / mean
+    launch time, timed the same way) against the measured HBM copy bandwidth.
+  - frame_roofline: the whole frame (4 queries + 1 commit, overlapped) against both peaks.
+  - stream: 240 frames, each bracketed by events: per-frame time first/last and its slope,
+    and device memory (cudaMemGetInfo) before and after.
+  - sweep: frames/s and the two kernels' roofline fractions at B in {1, 4} and
+    T in {390, 1560, 3600} (device-generated seeded inputs, larger than L2 per cycle).
   - cpu_baseline: the fp64 oracle on this host's cores over a bounded sample.
   - clocks: SM clocks and throttle reasons sampled with NVML during the timed region.
 With --gpus N under torchrun, each rank runs its own independent layer (the layer has no
@@ -53,10 +61,26 @@ CONFIG = {"workload": "480p single layer: B=1, H=12, d=128, T=1560 tokens/frame;
           "l2": "inputs larger than L2 (8-frame cycle of distinct q/k/v, 575 MB)"}
 
 # Algorithmic work (only what the layer must do; padding of ragged tiles is not credited).
-QUERY_FLOPS = B * H * (4.0 * T * T * D + 2 * 2.0 * T * D * D)        # QK^T + PV, phi_q + readout
-QUERY_BYTES = B * T * H * D * 2 * 4 + B * H * D * D * (2 + 2)          # q,k,v,o bf16; S bf16 copy, Wq
-COMMIT_FLOPS = B * H * 4 * 2.0 * T * D * D                             # K Wk, V Wv, K'S, K'^T R
-COMMIT_BYTES = B * T * H * D * 2 * 2 + 2 * B * H * T * 4 + B * H * D * D * 4 * 2 + 2 * H * D * D * 2
+def query_flops(b, t, h, d):      # QK^T + PV, phi_q + readout
+    return b * h * (4.0 * t * t * d + 2 * 2.0 * t * d * d)
+
+
+def query_bytes(b, t, h, d):      # q, k, v, o bf16; S bf16 copy, Wq
+    return b * t * h * d * 2 * 4 + b * h * d * d * (2 + 2)
+
+
+def commit_flops(b, t, h, d):     # K Wk, V Wv, K'S, K'^T R
+    return b * h * 4 * 2.0 * t * d * d
+
+
+def commit_bytes(b, t, h, d):     # k, v bf16; alpha, beta; S read + write fp32; Wk, Wv
+    return b * t * h * d * 2 * 2 + 2 * b * h * t * 4 + b * h * d * d * 4 * 2 + 2 * h * d * d * 2
+
+
+QUERY_FLOPS, QUERY_BYTES = query_flops(B, T, H, D), query_bytes(B, T, H, D)
+COMMIT_FLOPS, COMMIT_BYTES = commit_flops(B, T, H, D), commit_bytes(B, T, H, D)
+FRAME_FLOPS = QUERIES * QUERY_FLOPS + COMMIT_FLOPS
+FRAME_BYTES = QUERIES * QUERY_BYTES + COMMIT_BYTES
 
 
 # NVIDIA's dense (no 2:4 sparsity) bf16 tensor-core figure for one B200, for context only; the
@@ -64,12 +88,22 @@ COMMIT_BYTES = B * T * H * D * 2 * 2 + 2 * B * H * T * 4 + B * H * D * D * 4 * 2
 DATASHEET_BF16_TFLOPS = 2250.0
 
 
-def _query_traffic():
-    """DRAM bytes per query launch from the committed ncu capture, or None when the query
-    kernel's sources changed since that capture (the summary records their SHA-256)."""
+def kernel_sources_sha256(kernel_file: str) -> str:
+    """SHA-256 over a kernel's source file and the headers it includes."""
     import hashlib
+    csrc = os.path.join(ROOT, "softmax_attention_ar_b200", "csrc")
+    digest = hashlib.sha256()
+    for f in (kernel_file, "arl2_device.cuh", "arl2_kernels.h"):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            digest.update(fh.read())
+    return digest.hexdigest()
+
+
+def _profile_traffic(summary: str, kernel_file: str):
+    """DRAM bytes per launch from a committed ncu summary, or None when the kernel's sources
+    changed since that capture (the summary records their SHA-256)."""
     import re
-    path = os.path.join(ROOT, "profiles", "arl2_query_kernel_480p.md")
+    path = os.path.join(ROOT, "profiles", summary)
     if not os.path.exists(path):
         return None
     text = open(path).read()
@@ -77,12 +111,7 @@ def _query_traffic():
     h = re.search(r"^kernel_sources_sha256: ([0-9a-f]{64})$", text, re.M)
     if not t or not h:
         return None
-    csrc = os.path.join(ROOT, "softmax_attention_ar_b200", "csrc")
-    digest = hashlib.sha256()
-    for f in ("arl2_query.cu", "arl2_device.cuh", "arl2_kernels.h"):
-        with open(os.path.join(csrc, f), "rb") as fh:
-            digest.update(fh.read())
-    return int(t.group(1)) if digest.hexdigest() == h.group(1) else None
+    return int(t.group(1)) if kernel_sources_sha256(kernel_file) == h.group(1) else None
 
 
 def _peaks():
@@ -231,9 +260,9 @@ def kv_cache_baseline(frames, dev, layer_ms_per_frame, layer_bytes):
     for N in Ns:
         base.reset()
         for f in range(N - 1):
-            _, k, v = frames[f % CYCLE][0][QUERIES]
+            _, k, v = frames[f % CYCLE][0][QUERIES][:3]
             base.commit(k, v)
-        passes = frames[(N - 1) % CYCLE][0]
+        passes = [p[:3] for p in frames[(N - 1) % CYCLE][0]]
         for p in range(QUERIES):                       # warm-up
             base.query(*passes[p], out=o)
         st, en = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -287,6 +316,148 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def _time_windows(run_frame, stream, n_windows, frames_per_window, start, barrier):
+    """n_windows back-to-back windows of frames_per_window frames; each window bracketed by
+    CUDA events on the launching stream. Returns the frames/s of each window."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_windows)]
+    barrier()
+    i = start
+    for s, e in evs:
+        s.record(stream)
+        for _ in range(frames_per_window):
+            run_frame(i)
+            i += 1
+        e.record(stream)
+    barrier()
+    return [frames_per_window / (s.elapsed_time(e) / 1e3) for s, e in evs]
+
+
+def _split_times(layer, frames, stream, n, barrier, queries=QUERIES):
+    """Per-kernel split: every launch bracketed by its own events and run alone (overlap
+    off). Returns (query launch times in ms, commit launch times in ms, per-frame us)."""
+    import torch
+    layer.set_launch_overlap(False)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * (queries + 1))] for _ in range(n)]
+    barrier()
+    for i in range(n):
+        passes, a, b = frames[i % len(frames)]
+        for p in range(queries):
+            ev[i][2 * p].record(stream)
+            layer.query(*passes[p][:3], out=passes[p][3])
+            ev[i][2 * p + 1].record(stream)
+        _, k, v, _ = passes[queries]
+        ev[i][2 * queries].record(stream)
+        layer.commit(k, v, a, b)
+        ev[i][2 * queries + 1].record(stream)
+    barrier()
+    q_ms = [e[2 * p].elapsed_time(e[2 * p + 1]) for e in ev for p in range(queries)]
+    c_ms = [e[2 * queries].elapsed_time(e[2 * queries + 1]) for e in ev]
+    return q_ms, c_ms
+
+
+def _rooflines(q_ms, c_ms, b, t, h, d, peaks):
+    """Achieved rates of the two kernels, each launch timed alone, against the burst peaks."""
+    q_s, c_s = statistics.mean(q_ms) / 1e3, statistics.mean(c_ms) / 1e3
+    q_tf = query_flops(b, t, h, d) / q_s / 1e12
+    c_gbs = commit_bytes(b, t, h, d) / c_s / 1e9
+    return {"query_us": 1e6 * q_s, "query_p95_us": 1e3 * float(np.percentile(q_ms, 95)),
+            "query_tflops": q_tf, "query_frac_of_bf16_burst": q_tf / peaks["bf16_tflops"],
+            "commit_us": 1e6 * c_s, "commit_p95_us": 1e3 * float(np.percentile(c_ms, 95)),
+            "commit_hbm_gbs": c_gbs, "commit_frac_of_hbm": c_gbs / peaks["hbm_gbs"],
+            "commit_tflops": commit_flops(b, t, h, d) / c_s / 1e12}
+
+
+def _device_frames(dev, b, t, h, d, n_frames, seed):
+    """Seeded synthetic frames generated on the device (timing-only shapes): per frame the 5
+    passes' (q, k, v, o) and the gates, with the distributions of the 480p workload."""
+    import torch
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    frames = []
+    for _ in range(n_frames):
+        passes = []
+        for _ in range(QUERIES + 1):
+            q, k, v = (torch.randn((b, t, h, d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+                       for _ in range(3))
+            passes.append((q, k, v, torch.empty_like(q)))
+        a = torch.sigmoid(2.0 + 0.5 * torch.randn((b, h, t), generator=g, device=dev))
+        be = torch.sigmoid(torch.randn((b, h, t), generator=g, device=dev))
+        frames.append((passes, a, be))
+    wq, wk, wv = ((torch.randn((h, d, d), generator=g, device=dev) / d ** 0.5).to(torch.bfloat16) for _ in range(3))
+    return frames, (wq, wk, wv)
+
+
+def sweep(dev, stream, barrier, peaks, n_frames=30, n_split=30):
+    """The token/batch sweep: B in {1, 4} x T in {390, 1560, 3600}, H=12, d=128."""
+    import torch
+
+    from softmax_attention_ar_b200.arl2 import ARL2Layer
+    rows = []
+    for b in (1, 4):
+        for t in (390, 1560, 3600):
+            act = b * t * H * D * 2
+            cycle = max(2, min(8, int(np.ceil(3 * 128e6 / (5 * 3 * act)))))   # > L2 per cycle
+            frames, maps = _device_frames(dev, b, t, H, D, cycle, seed=1000 + 10 * b + t)
+            layer = ARL2Layer(H, t, D, b)
+            layer.set_feature_maps(*maps)
+
+            def frame(i):
+                passes, a, be = frames[i % cycle]
+                for p in range(QUERIES):
+                    layer.query(*passes[p][:3], out=passes[p][3])
+                _, k, v, _ = passes[QUERIES]
+                layer.commit(k, v, a, be)
+
+            layer.set_launch_overlap(True)
+            for i in range(3):
+                frame(i)
+            fps = _time_windows(frame, stream, 3, n_frames // 3, 3, barrier)
+            q_ms, c_ms = _split_times(layer, frames, stream, n_split, barrier)
+            st = layer.status()
+            ms_frame = 1e3 / statistics.median(fps)   # one frame of all B streams
+            row = {"B": b, "T": t, "frames_per_s": b * statistics.median(fps), "ms_per_frame": ms_frame,
+                   "frame_frac_of_bf16_burst": (QUERIES * query_flops(b, t, H, D) + commit_flops(b, t, H, D))
+                   / (ms_frame / 1e3) / 1e12 / peaks["bf16_tflops"],
+                   "status": st, "input_cycle_frames": cycle}
+            row.update(_rooflines(q_ms, c_ms, b, t, H, D, peaks))
+            rows.append(row)
+            layer.close()
+            del frames
+            torch.cuda.empty_cache()
+    return {"what": "4 queries + 1 commit per frame, overlapped; per-kernel times with each launch alone; "
+                    "frames/s counts B streams' frames", "H": H, "d": D, "rows": rows}
+
+
+def stream_leg(layer, frames, stream, barrier, n=240):
+    """Per-frame time over n frames (each frame bracketed by events, overlap on inside it) and
+    device memory before and after: the layer's cost must not grow with the frame count."""
+    import torch
+    layer.reset()
+    layer.set_launch_overlap(True)
+    barrier()
+    free0, _ = torch.cuda.mem_get_info()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for i, (s, e) in enumerate(ev):
+        passes, a, b = frames[i % len(frames)]
+        s.record(stream)
+        for p in range(QUERIES):
+            layer.query(*passes[p][:3], out=passes[p][3])
+        _, k, v, _ = passes[QUERIES]
+        layer.commit(k, v, a, b)
+        e.record(stream)
+    barrier()
+    free1, _ = torch.cuda.mem_get_info()
+    f_us = np.array([1e3 * s.elapsed_time(e) for s, e in ev])
+    edge = 50
+    return {"frames": n, "us_per_frame_first50": float(f_us[:edge].mean()),
+            "us_per_frame_last50": float(f_us[-edge:].mean()),
+            "us_per_frame_median": float(np.median(f_us)),
+            "slope_us_per_frame": float(np.polyfit(np.arange(n), f_us, 1)[0]),
+            "device_free_bytes_before": int(free0), "device_free_bytes_after": int(free1),
+            "layer_bytes": layer.memory_bytes, "frame_index_after": layer.frame_index}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -299,6 +470,7 @@ def run_ours(args, rank, world, local_rank):
     layer = ARL2Layer(H, T, D, B)
     layer.set_feature_maps(*maps)
     o = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
+    frames = [([p + (o,) for p in passes], a, b) for passes, a, b in frames]
     stream = torch.cuda.current_stream()
 
     def barrier():
@@ -306,25 +478,16 @@ def run_ours(args, rank, world, local_rank):
             dist.barrier()
         torch.cuda.synchronize()
 
-    def step(i, ev=None):
+    def step(i):
         passes, a, b = frames[i % CYCLE]
         for p in range(QUERIES):
-            if ev is not None:
-                ev[0].record(stream)
-            layer.query(*passes[p], out=o)
-            if ev is not None:
-                ev[1].record(stream)
-                ev = ev[2:]
-        _, k, v = passes[QUERIES]
-        if ev is not None:
-            ev[0].record(stream)
+            layer.query(*passes[p][:3], out=o)
+        _, k, v, _ = passes[QUERIES]
         layer.commit(k, v, a, b)
-        if ev is not None:
-            ev[1].record(stream)
 
     # Device-resident run. Throughput: the frames back to back, queries and commits
     # overlapping the kernel before them (programmatic dependent launch), only start/end
-    # events.
+    # events around exactly `steps` frames.
     layer.set_launch_overlap(True)
     for i in range(args.warmup):
         step(i)
@@ -337,28 +500,20 @@ def run_ours(args, rank, world, local_rank):
             step(args.warmup + i)
         end.record(stream)
         barrier()
+        # The same window, repeated (the clock sampler keeps running): median and spread.
+        reps = _time_windows(step, stream, 20, args.steps, args.warmup + args.steps, barrier)
     elapsed_ms = start.elapsed_time(end)
-    # Per-kernel split for the roofline: a second timed region with an event pair around
-    # every launch and overlap off, so each interval is one kernel alone.
-    layer.set_launch_overlap(False)
-    split_steps = max(1, min(args.steps, 400))
-    ev_all = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * (QUERIES + 1))] for _ in range(split_steps)]
-    barrier()
-    for i in range(split_steps):
-        step(args.warmup + i, ev_all[i])
-    barrier()
-    q_ms = [ev[2 * p].elapsed_time(ev[2 * p + 1]) for ev in ev_all for p in range(QUERIES)]
-    c_ms = [ev[2 * QUERIES].elapsed_time(ev[2 * QUERIES + 1]) for ev in ev_all]
-    # Streaming: the layer's per-frame time must not grow with the frame count.
-    f_us = np.array([1e3 * sum(ev[2 * j].elapsed_time(ev[2 * j + 1]) for j in range(QUERIES + 1)) for ev in ev_all])
-    edge = max(1, min(50, len(f_us) // 4))
-    stream_info = {"frames": len(f_us), "us_per_frame_first": float(f_us[:edge].mean()),
-                   "us_per_frame_last": float(f_us[-edge:].mean()),
-                   "slope_us_per_frame": float(np.polyfit(np.arange(len(f_us)), f_us, 1)[0]) if len(f_us) > 1 else 0.0,
-                   "state_bytes_constant": layer.memory_bytes}
+    # Per-kernel split for the roofline: every launch bracketed by events and run alone.
+    split_frames = 200
+    q_ms, c_ms = _split_times(layer, frames, stream, split_frames, barrier)
     status = layer.status()
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
+    peaks = _peaks()
+    stream_info = stream_leg(layer, frames, stream, barrier)
+    if layer.status() != 0:
+        raise RuntimeError("device status after the streaming leg")
+    sweep_info = None if args.no_sweep else sweep(dev, stream, barrier, peaks)
 
     # End-to-end through the host-buffer entry points (pinned host memory).
     pinned = [([tuple(t.pin_memory() for t in p) for p in passes], a.pin_memory(), b.pin_memory())
@@ -396,34 +551,46 @@ def run_ours(args, rank, world, local_rank):
         return
     value = job_rate(world, B * args.steps, elapsed_ms)
     e2e_value = job_rate(world, B * e2e_steps, e2e_ms) if e2e_steps else None
-    peaks = _peaks()
-    q_mean_s = statistics.mean(q_ms) / 1e3
-    c_mean_s = statistics.mean(c_ms) / 1e3
-    q_tflops = QUERY_FLOPS / q_mean_s / 1e12
-    peak = peaks["bf16_tflops_sustained"]
+    k = _rooflines(q_ms, c_ms, B, T, H, D, peaks)
+    q_tflops, c_gbs = k["query_tflops"], k["commit_hbm_gbs"]
+    frame_s = elapsed_ms / args.steps / 1e3
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": CONFIG,
-        "roofline": {"bound": "tensor", "achieved": q_tflops, "peak": peak, "unit": "TFLOP/s",
-                     "frac": q_tflops / peak, "traffic": _query_traffic(), "traffic_unit": "DRAM bytes per launch",
-                     "kernel": "arl2_query_kernel (one query pass)",
-                     "peak_source": f"bf16_tflops_sustained ({peaks['source']})",
-                     "frac_of_burst_peak": q_tflops / peaks["bf16_tflops"],
+        "roofline": {"bound": "tensor", "achieved": q_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": q_tflops / peaks["bf16_tflops"],
+                     "traffic": _profile_traffic("arl2_query_kernel_480p.md", "arl2_query.cu"),
+                     "traffic_unit": "DRAM bytes per launch",
+                     "kernel": "arl2_query_kernel (one query pass, each launch timed alone)",
+                     "algorithmic_flops_per_launch": QUERY_FLOPS,
+                     "peak_source": f"bf16_tflops, burst ({peaks['source']})",
+                     "frac_of_sustained_peak": q_tflops / peaks["bf16_tflops_sustained"],
                      "frac_of_datasheet_dense_bf16": q_tflops / DATASHEET_BF16_TFLOPS},
-        "kernels": {"timed_steps": split_steps, "launch_overlap": "off in this split, on for value",
-                    "query_us": 1e6 * q_mean_s, "query_p95_us": 1e3 * float(np.percentile(q_ms, 95)),
-                    "commit_us": 1e6 * c_mean_s,
-                    "commit_hbm_gbs": COMMIT_BYTES / c_mean_s / 1e9,
-                    "commit_hbm_frac": COMMIT_BYTES / c_mean_s / 1e9 / peaks["hbm_gbs"],
-                    "commit_tflops": COMMIT_FLOPS / c_mean_s / 1e12},
+        "roofline_commit": {"bound": "hbm", "achieved": c_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": c_gbs / peaks["hbm_gbs"],
+                            "traffic": _profile_traffic("arl2_commit_kernel_480p.md", "arl2_commit.cu"),
+                            "kernel": "arl2_commit_kernel (one commit, each launch timed alone)",
+                            "algorithmic_bytes_per_launch": COMMIT_BYTES,
+                            "peak_source": f"hbm_gbs ({peaks['source']})",
+                            "tflops": k["commit_tflops"]},
+        "frame_roofline": {"what": "4 queries + 1 commit back to back (ms_per_step)",
+                           "tflops": FRAME_FLOPS / frame_s / 1e12,
+                           "frac_of_bf16_burst": FRAME_FLOPS / frame_s / 1e12 / peaks["bf16_tflops"],
+                           "gbs": FRAME_BYTES / frame_s / 1e9,
+                           "frac_of_hbm": FRAME_BYTES / frame_s / 1e9 / peaks["hbm_gbs"]},
+        "kernels": dict(k, timed_frames=split_frames, launch_overlap="off in this split, on for value"),
+        "repeats": {"windows": len(reps), "frames_per_window": args.steps,
+                    "median": statistics.median(reps), "min": min(reps), "max": max(reps)},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
         "gpu_launches": args.steps * (QUERIES + 1),   # per frame: the query launches and one commit
         "launch_overlap": "queries and commits launched as programmatic dependents of the kernel before them",
         "clocks": clocks.summary(),
+        "stream": stream_info,
     }
-    line["stream"] = stream_info
+    if sweep_info is not None:
+        line["sweep"] = sweep_info
     if not args.no_kv_baseline:
         line["kv_cache_baseline"] = kv_cache_baseline(frames, dev, elapsed_ms / args.steps, layer.memory_bytes)
     if world == 1 and not args.no_cpu_baseline:
@@ -441,6 +608,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer (e2e) measurement")
     ap.add_argument("--no-kv-baseline", action="store_true", help="skip the growing-KV-cache comparison")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the token/batch sweep")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -172,20 +172,24 @@ void arl2_destroy(arl2_ctx* ctx);
  *   - Wk, Wv: bf16 [H, d, d].
  *   - S_prev, S_next: fp32 [B, H, d, d]. S_next may be S_prev itself (an in-place
  *     update) or must not overlap it.
- *   - status: optional device word, ORed with 1 if a kernel's bounded wait ran out. The
- *     caller zeroes it; NULL uses an internal word.
+ *   - status: a device word (4-byte aligned, required), ORed with 1 if a bounded wait in
+ *     the kernel ran out. The caller zeroes it before the call and reads it after the
+ *     stream has passed the call. Without a context there is nowhere else a time-out could
+ *     be reported, so NULL returns ARL2_ERR_INVALID_ARG. After a time-out S_next is
+ *     undefined; for an in-place call (S_next == S_prev) that includes S_prev.
  *
  * The call allocates nothing. Its scratch is a fixed device array of
  * ARL2_NOALLOC_SCRATCH_BYTES inside the library. Every GPU that loads the library holds
  * that array until the process exits. Shapes whose scratch would exceed it return
- * ARL2_ERR_UNSUPPORTED before any work is enqueued. The need is about B*H*d*d*8 bytes
- * (copies of S_prev and S_next; the chunk groups' partial sums meet in on-chip memory);
- * B=1, H=12, d=128 needs about 1.6 MB, and d=128 fits up to B*H = 127.
+ * ARL2_ERR_UNSUPPORTED before any work is enqueued. The need is about B*H*d*d*4 bytes
+ * (bf16 copies of S_prev and S_next; the chunk groups' partial sums meet in on-chip
+ * memory); B=1, H=12, d=128 needs about 0.8 MB, and d=128 fits up to B*H = 256.
  *
  * The first call on a device looks the array's device address up, with that device
  * current. Make that first call before any stream capture. All calls on a device share
- * the one array and leave their contents in it. Each call clears what it needs at zero.
- * Calls that overlap on the GPU, for example on two streams, race on the array.
+ * the one array and leave their contents in it; each call writes what it reads before
+ * reading it, and nothing in it needs to start at zero. Calls that overlap on the GPU,
+ * for example on two streams, race on the array.
  * Supported shapes are as for arl2_create. */
 #define ARL2_NOALLOC_SCRATCH_BYTES (16u << 20)
 arl2_status arl2_frame_commit_noalloc(int B, int H, int T, int d, const arl2_bf16* k, const arl2_bf16* v,

@@ -223,21 +223,19 @@ class ARL2Layer:
         return self._lib.arl2_memory_bytes(self._ctx)
 
 
-def frame_commit_noalloc(k, v, alpha, beta, Wk, Wv, S_prev, S_next, status=None, stream=None) -> None:
+def frame_commit_noalloc(k, v, alpha, beta, Wk, Wv, S_prev, S_next, status, stream=None) -> None:
     """Commit without a context or any allocation (arl2_frame_commit_noalloc).
 
     For callers that cannot allocate device memory: the library's fixed scratch array is
     used instead. k, v bf16 [B, T, H, d]; alpha, beta fp32 [B, H, T]; Wk, Wv bf16 [H, d, d];
-    S_prev, S_next fp32 [B, H, d, d] (S_next may be S_prev); status an optional int32 [1]
-    device word the caller zeroed.
+    S_prev, S_next fp32 [B, H, d, d] (S_next may be S_prev); status an int32 [1] device word
+    the caller zeroed, which reads nonzero after the call if a bounded wait ran out.
     """
     B, T, H, d = k.shape
     s, g, w, st = (B, T, H, d), (B, H, T), (H, d, d), (B, H, d, d)
-    status_ptr = None
-    if status is not None:
-        if status.dtype != torch.int32 or status.numel() != 1:
-            raise ValueError("status: expected one int32 element")
-        status_ptr = status.data_ptr()
+    if status is None or status.dtype != torch.int32 or status.numel() != 1 or not status.is_cuda:
+        raise ValueError("status: expected one int32 element in device memory")
+    status_ptr = status.data_ptr()
     _check(load_library().arl2_frame_commit_noalloc(
         B, H, T, d, _dev(k, torch.bfloat16, s, "k"), _dev(v, torch.bfloat16, s, "v"),
         _dev(alpha, torch.float32, g, "alpha"), _dev(beta, torch.float32, g, "beta"),

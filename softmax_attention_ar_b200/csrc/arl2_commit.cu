@@ -43,7 +43,7 @@ constexpr uint32_t kVOff = 5 * kTileBytes;   // two stages
 constexpr uint32_t kRecvOff = kWkOff;
 constexpr uint32_t kCtlOff = 7 * kTileBytes;
 enum : int {
-  kBarW = 0,          // Wk, Wv, S landed
+  kBarW = 0,          // Wk, Wv landed
   kBarKVFull = 1,     // +stage (2)
   kBarKVEmpty = 3,    // +stage
   kBarProjK = 5,      // +Kp buffer (2): Kp of the chunk in TMEM
@@ -52,7 +52,8 @@ enum : int {
   kBarR = 9,          // R bf16 over the V tile (one arrival per row warp)
   kBarU = 10,         // U complete
   kBarFinal = 11,     // every MMA done (drain before TMEM is freed)
-  kNumBars = 12
+  kBarS = 12,         // the bf16 copy of S_{N-1} landed
+  kNumBars = 13
 };
 constexpr uint32_t kCtlMisc = 128;           // tmem slot, abort flag, alpha sums, status
 constexpr uint32_t kSmemBytes = kCtlOff + kCtlMisc + 64;
@@ -76,21 +77,32 @@ struct Smem {
 };
 __device__ __forceinline__ uint32_t col_kp(int i) { return (i & 1) ? kColKp1 : kColKp0; }
 
-// Warp 0 (warp-wide, lead lane issues): Wk, Wv and the bf16 S once, then K and V chunk
-// tiles through two stages.
+// Warp 0 (warp-wide, lead lane issues): Wk and Wv once, the first K and V chunk tiles, then
+// the bf16 S once, then the remaining K and V chunk tiles through two stages. S_{N-1} is the
+// previous commit's output; when this grid was launched as a programmatic dependent of the
+// kernel before it, that output is visible only after griddepcontrol.wait, so S waits for
+// it and goes out after the first chunk (the projections do not need S).
 __device__ void producer(const Smem& sm, const CUtensorMap* tm_k, const CUtensorMap* tm_v, const CUtensorMap* tm_wk,
                          const CUtensorMap* tm_wv, const CUtensorMap* tm_s, const CommitArgs& a, int c0, int nc,
                          int h, int b, bool lead, const Guard& g) {
   uint32_t n[2] = {0, 0};
   const int slot = a.state_slot * a.B * a.H + b * a.H + h;
   if (lead) {
-    mbar_expect_tx(sm.bar(kBarW), 3 * kTileBytes);
+    mbar_expect_tx(sm.bar(kBarW), 2 * kTileBytes);
     for (int p = 0; p < 2; ++p) {
       tma_load_3d(sm.wk() + p * kPanelBytes, tm_wk, sm.bar(kBarW), 64 * p, 0, h);
       tma_load_3d(sm.wv() + p * kPanelBytes, tm_wv, sm.bar(kBarW), 64 * p, 0, h);
-      tma_load_3d(sm.s() + p * kPanelBytes, tm_s, sm.bar(kBarW), 64 * p, 0, slot);
     }
   }
+  auto load_s = [&]() {
+    griddep_wait();
+    if (lead) {
+      mbar_expect_tx(sm.bar(kBarS), kTileBytes);
+      for (int p = 0; p < 2; ++p) tma_load_3d(sm.s() + p * kPanelBytes, tm_s, sm.bar(kBarS), 64 * p, 0, slot);
+    }
+    __syncwarp();
+  };
+  if (nc == 0) load_s();
   for (int i = 0; i < nc; ++i) {
     const int s = i & 1;
     if (i >= 2 && !mbar_wait_warp(sm.bar(kBarKVEmpty + s), ((i - 2) >> 1) & 1, g)) break;
@@ -103,8 +115,10 @@ __device__ void producer(const Smem& sm, const CUtensorMap* tm_k, const CUtensor
       }
     }
     ++n[s];
+    if (i == 0) load_s();
   }
   mbar_wait_drain(sm.bar(kBarW), 0);
+  mbar_wait_drain(sm.bar(kBarS), 0);
   for (int s = 0; s < 2; ++s)
     if (n[s]) mbar_wait_drain(sm.bar(kBarKVFull + s), (n[s] - 1) & 1);
 }
@@ -140,6 +154,7 @@ __device__ void mma_issuer(const Smem& sm, uint32_t tmem, int nc, bool lead, con
       proj_k(i + 1);
     }
     // Vp -= K'S: K' (bf16) over the K tile, S from its bf16 copy, B negated.
+    if (i == 0 && !mbar_wait_warp(sm.bar(kBarS), 0, g)) return;
     if (!mbar_wait_warp(sm.bar(kBarKn), i & 1, g)) return;
     tc_fence_after();
     if (lead) {
@@ -284,6 +299,7 @@ __global__ void __launch_bounds__(kThreadsC, 1)
     mbar_init(sm.bar(kBarR), kRowWarps);
     mbar_init(sm.bar(kBarU), 1);
     mbar_init(sm.bar(kBarFinal), 1);
+    mbar_init(sm.bar(kBarS), 1);
     *abort_flag = 0;
     *rows_failed = 0;
     fence_barrier_init();
@@ -430,7 +446,7 @@ __global__ void arl2_state_import_kernel(const float* __restrict__ src, float* _
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const float x = src[i];
-    S[i] = x;
+    if (S) S[i] = x;
     __nv_bfloat16 y = __float2bfloat16_rn(x);
     S_bf16[i] = *reinterpret_cast<uint16_t*>(&y);
   }

@@ -89,7 +89,7 @@ cudaError_t launch_query(bool hybrid, const CUtensorMap& tm_q, const CUtensorMap
 cudaError_t launch_commit(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const CUtensorMap& tm_wk,
                           const CUtensorMap& tm_wv, const CUtensorMap& tm_s, const CommitArgs& a,
                           const ReduceArgs& r, cudaStream_t stream, bool dependent);
-// fp32 state -> state buffer + bf16 copy.
+// fp32 state -> state buffer (skipped when S is null) + bf16 copy.
 cudaError_t launch_state_import(const float* src, float* S, uint16_t* S_bf16, size_t n, cudaStream_t stream);
 
 }  // namespace arl2

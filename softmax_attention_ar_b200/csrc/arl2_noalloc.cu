@@ -9,9 +9,10 @@
 // (k, v, the gates, phi_k, phi_v, S_{N-1}) and the output (S_N). The scratch the commit
 // needs lives in one file-scope device array of fixed size, g_commit_scratch. It holds:
 //   - the bf16 copy of S_{N-1} the MMAs read;
-//   - discarded copies (an fp32 copy of S_{N-1}, a bf16 copy of S_N);
-//   - a device status word, used when the caller passes none.
-// The groups' partial sums meet in distributed shared memory, so they need no scratch.
+//   - a discarded bf16 copy of S_N (the kernel writes one for the context's queries).
+// The groups' partial sums meet in distributed shared memory, so they need no scratch. The
+// caller passes a device status word: a kernel whose bounded wait ran out reports it there,
+// and there is no other place it could be read back without a context.
 // The array is part of the library's device image, so every GPU that loads the library
 // holds ARL2_NOALLOC_SCRATCH_BYTES of it until the process exits.
 //
@@ -19,9 +20,8 @@
 // looked up once per device, with that device current, by cudaGetSymbolAddress on the
 // first call made on the device. That first call should therefore come before any stream
 // capture. Every call on a device shares the one array and leaves its contents behind.
-// Each call writes everything it reads back before reading it, and it clears the status
-// word. Calls that overlap on the GPU (on different streams, say) race on the array and
-// must not be made.
+// Each call writes everything it reads back before reading it. Calls that overlap on the
+// GPU (on different streams, say) race on the array and must not be made.
 #include <mutex>
 
 #include "../../include/arl2.h"
@@ -63,7 +63,7 @@ extern "C" arl2_status arl2_frame_commit_noalloc(int B, int H, int T, int d, con
                                                  unsigned int* status, arl2_stream stream) {
   if (B < 1 || H < 1 || T < 1 || d < 1) return ARL2_ERR_INVALID_ARG;
   if (!aligned(k, 16) || !aligned(v, 16) || !aligned(Wk, 16) || !aligned(Wv, 16) || !aligned(S_prev, 16) ||
-      !aligned(S_next, 16) || !aligned(alpha, 4) || !aligned(beta, 4) || (status && !aligned(status, 4)))
+      !aligned(S_next, 16) || !aligned(alpha, 4) || !aligned(beta, 4) || !aligned(status, 4))
     return ARL2_ERR_INVALID_ARG;
   if ((d != 32 && d != 64 && d != 128) || T > 4096 || static_cast<long long>(B) * H > 65535)
     return ARL2_ERR_UNSUPPORTED;
@@ -75,11 +75,10 @@ extern "C" arl2_status arl2_frame_commit_noalloc(int B, int H, int T, int d, con
   int cpg = 1, ngroups = 1;
   arl2::commit_split(T, H, B, sms, &cpg, &ngroups);
 
-  // Scratch layout: status word | S_{N-1} bf16 | S_{N-1} fp32 (discarded) | S_N bf16 (discarded).
+  // Scratch layout: S_{N-1} bf16 | S_N bf16 (discarded).
   const size_t bh = static_cast<size_t>(B) * H, dd = static_cast<size_t>(d) * d;
-  const size_t off_sprev = 256;
-  const size_t off_sdisc = off_sprev + round256(bh * dd * 2);
-  const size_t off_snext = off_sdisc + round256(bh * dd * 4);
+  const size_t off_sprev = 0;
+  const size_t off_snext = off_sprev + round256(bh * dd * 2);
   const size_t needed = off_snext + round256(bh * dd * 2);
   if (needed > kScratchBytes) return ARL2_ERR_UNSUPPORTED;
 
@@ -87,9 +86,7 @@ extern "C" arl2_status arl2_frame_commit_noalloc(int B, int H, int T, int d, con
   const arl2_status ss = scratch_on_device(dev, &scratch);
   if (ss != ARL2_OK) return ss;
   uint16_t* s_prev_bf16 = reinterpret_cast<uint16_t*>(scratch + off_sprev);
-  float* s_prev_disc = reinterpret_cast<float*>(scratch + off_sdisc);
   uint16_t* s_next_bf16 = reinterpret_cast<uint16_t*>(scratch + off_snext);
-  unsigned int* err = status ? status : reinterpret_cast<unsigned int*>(scratch);
 
   CUtensorMap tm_k, tm_v, tm_wk, tm_wv, tm_s;
   if (!arl2::encode_act_map(&tm_k, k, B, T, H, d) || !arl2::encode_act_map(&tm_v, v, B, T, H, d) ||
@@ -98,9 +95,8 @@ extern "C" arl2_status arl2_frame_commit_noalloc(int B, int H, int T, int d, con
     return ARL2_ERR_CUDA;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (!status && cudaMemsetAsync(err, 0, sizeof(unsigned int), st) != cudaSuccess) return ARL2_ERR_CUDA;
-  // bf16 copy of S_{N-1} for the K'S MMA (the import's fp32 copy goes to a discarded area).
-  if (arl2::launch_state_import(S_prev, s_prev_disc, s_prev_bf16, bh * dd, st) != cudaSuccess) return ARL2_ERR_CUDA;
+  // bf16 copy of S_{N-1} for the K'S MMA (no fp32 copy: the commit reads S_prev itself).
+  if (arl2::launch_state_import(S_prev, nullptr, s_prev_bf16, bh * dd, st) != cudaSuccess) return ARL2_ERR_CUDA;
 
   arl2::CommitArgs a{};
   a.alpha = alpha;
@@ -113,7 +109,7 @@ extern "C" arl2_status arl2_frame_commit_noalloc(int B, int H, int T, int d, con
   a.ngroups = ngroups;
   a.state_slot = 0;
   a.inv_T = 1.0f / static_cast<float>(T);
-  a.err = err;
+  a.err = status;
   a.timeout_ns = kTimeoutNs;
   arl2::ReduceArgs r{};
   r.S_old = S_prev;

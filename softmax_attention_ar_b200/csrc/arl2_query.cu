@@ -267,6 +267,7 @@ __device__ void producer(const Smem& sm, const CUtensorMap* tm_q, const CUtensor
   Sched sch(a, blockIdx.x);
   Seg sg;
   bool ok = true;
+  bool waited = false;   // V producer: griddepcontrol.wait done before the first state load
   auto slot_wait = [&](uint32_t gidx) -> bool {
     return gidx < kStages || mbar_wait_warp(sm.bar(empty0 + ring_stage(gidx)), ring_phase(gidx - kStages), g);
   };
@@ -315,6 +316,14 @@ __device__ void producer(const Smem& sm, const CUtensorMap* tm_q, const CUtensor
     }
     if (ok && kHybrid && sg.head) {
       // The readout operand (Wq_h or the bf16 state copy S_h) follows the key tiles.
+      // S_{N-1} may be the output of the commit right before this launch: when this grid
+      // was launched as its programmatic dependent, that commit's writes are visible only
+      // after griddepcontrol.wait. The V producer waits once, before its first state load
+      // (a no-op for a normal launch, and long past by then behind another query).
+      if (!kIsK && !waited) {
+        griddep_wait();
+        waited = true;
+      }
       if (!slot_wait(ring)) break;
       const int s = ring_stage(ring);
       const int c2 = kIsK ? sg.h : a.state_slot * a.B * a.H + sg.b * a.H + sg.h;
@@ -922,9 +931,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // A query launched right behind this one may start its CTAs as SMs free up. It reads
-  // nothing this one writes; it waits for this grid before its first global write (its
-  // scratch and output may be this grid's).
+  // A kernel launched right behind this one as its programmatic dependent may start its
+  // CTAs as SMs free up. A query or commit reads nothing a query writes (the host launches
+  // a call whose inputs overlap this grid's output normally). A query waits for the grid
+  // before it (this one, or a commit) before its first global write (its scratch and
+  // output may be this grid's) and before its first load of the state (a commit's output).
   griddep_launch_dependents();
 
   // Producers and the MMA issuer run warp-wide (uniform control flow and waits); one

@@ -84,13 +84,18 @@ class Case:
         s_ref = self.ref.commit(synth.bf16_to_f64(k), synth.bf16_to_f64(v), a, b)
         return host_f64(self.gpu.get_state()), s_ref
 
-    def run(self, frames, queries, rows=None, check_every_query=True):
-        """Drive frames x (queries + commit); assert the tolerances; return the worst errors."""
+    def run(self, frames, queries, rows=None, check_every_query=True, full_rows_at=(), s_errors=None):
+        """Drive frames x (queries + commit); assert the tolerances; return the worst errors.
+
+        rows: the query rows compared (None = all); on the frames in full_rows_at the first
+        query is compared on every row whatever rows says. s_errors, if a list, receives the
+        worst per-(b,h) state error after each commit."""
         worst_o, worst_s = 0.0, 0.0
         for f in range(frames):
             for p in range(queries):
                 if check_every_query or p == queries - 1:
-                    o_gpu, o_ref = self.query(f, p, rows)
+                    sel = None if (f in full_rows_at and p == 0) else rows
+                    o_gpu, o_ref = self.query(f, p, sel)
                     g, per = o_errors(o_gpu, o_ref)
                     assert g <= O_TOL and per <= O_TOL, f"frame {f} pass {p}: O error {g:.3e} / {per:.3e}"
                     worst_o = max(worst_o, per)
@@ -98,6 +103,8 @@ class Case:
             e = s_error(s_gpu, s_ref)
             assert e <= S_TOL, f"frame {f}: S error {e:.3e}"
             worst_s = max(worst_s, e)
+            if s_errors is not None:
+                s_errors.append(e)
         return worst_o, worst_s
 
 

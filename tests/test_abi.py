@@ -60,6 +60,11 @@ def test_argument_checks_need_no_gpu(lib):
     lib.arl2_destroy(None)
     assert lib.arl2_kvcache_create(12, 1560, 128, 1, 0, ctypes.byref(out)) == arl2.ARL2_ERR_INVALID_ARG
     lib.arl2_kvcache_destroy(None)
+    # The allocation-free commit has no context to report a time-out through, so its status
+    # word is required; a missing one is refused before any CUDA call.
+    p = 1 << 20   # an aligned address; never dereferenced by the argument checks
+    assert lib.arl2_frame_commit_noalloc(1, 12, 1560, 128, p, p, p, p, p, p, p, p, None, None) == \
+        arl2.ARL2_ERR_INVALID_ARG
 
 
 def test_built_for_sm100a_only():
