@@ -316,12 +316,25 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+HOST_MS_PER_LAUNCH = 0.05   # generous bound on the host's cost to enqueue one launch or event
+
+
+def queue_ahead(launches: int):
+    """Keep the device busy while the host enqueues the next timed region: a spin kernel
+    (torch.cuda._sleep) long enough for the host to queue `launches` launches behind it, so
+    the region's launches run back to back and its events measure device time only, not the
+    host's enqueue rate. Goes on the current stream before the region's first event."""
+    import torch
+    torch.cuda._sleep(int(2.0e6 * (0.5 + HOST_MS_PER_LAUNCH * launches)))   # ~2e6 cycles per ms
+
+
 def _time_windows(run_frame, stream, n_windows, frames_per_window, start, barrier):
     """n_windows back-to-back windows of frames_per_window frames; each window bracketed by
     CUDA events on the launching stream. Returns the frames/s of each window."""
     import torch
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_windows)]
     barrier()
+    queue_ahead(n_windows * frames_per_window * (QUERIES + 1) + 2 * n_windows)
     i = start
     for s, e in evs:
         s.record(stream)
@@ -340,6 +353,7 @@ def _split_times(layer, frames, stream, n, barrier, queries=QUERIES):
     layer.set_launch_overlap(False)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * (queries + 1))] for _ in range(n)]
     barrier()
+    queue_ahead(3 * n * (queries + 1))
     for i in range(n):
         passes, a, b = frames[i % len(frames)]
         for p in range(queries):
@@ -438,6 +452,7 @@ def stream_leg(layer, frames, stream, barrier, n=240):
     barrier()
     free0, _ = torch.cuda.mem_get_info()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    queue_ahead(n * (QUERIES + 3))
     for i, (s, e) in enumerate(ev):
         passes, a, b = frames[i % len(frames)]
         s.record(stream)
@@ -495,6 +510,7 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     with clocks:
         start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        queue_ahead(args.steps * (QUERIES + 1) + 2)
         start.record(stream)
         for i in range(args.steps):
             step(args.warmup + i)

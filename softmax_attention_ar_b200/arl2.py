@@ -97,6 +97,22 @@ def _dev(t: torch.Tensor, dtype: torch.dtype, shape, name: str) -> int:
     return t.data_ptr()
 
 
+def _cuda(t: torch.Tensor, dtype: torch.dtype, shape, name: str) -> int:
+    """_dev for arguments that must be device memory (the kernels read them through TMA)."""
+    p = _dev(t, dtype, shape, name)
+    if not t.is_cuda:
+        raise ValueError(f"{name}: expected a CUDA tensor")
+    return p
+
+
+def _host(t: torch.Tensor, dtype: torch.dtype, shape, name: str) -> int:
+    """_dev for arguments of the host-buffer calls, which must be host memory."""
+    p = _dev(t, dtype, shape, name)
+    if t.is_cuda:
+        raise ValueError(f"{name}: expected a host (CPU) tensor")
+    return p
+
+
 # ------------------------------------------------------------------ raw C-ABI mirrors
 def arl2_create(H: int, T: int, d_k: int, d_v: int, B: int) -> ctypes.c_void_p:
     out = _P()
@@ -157,32 +173,32 @@ class ARL2Layer:
         if out is None:
             out = torch.empty(self.act_shape, dtype=torch.bfloat16, device=q.device)
         s = self.act_shape
-        _check(self._lib.arl2_frame_query(self._ctx, _dev(q, torch.bfloat16, s, "q"), _dev(k, torch.bfloat16, s, "k"),
-                                          _dev(v, torch.bfloat16, s, "v"), _dev(out, torch.bfloat16, s, "o"),
+        _check(self._lib.arl2_frame_query(self._ctx, _cuda(q, torch.bfloat16, s, "q"), _cuda(k, torch.bfloat16, s, "k"),
+                                          _cuda(v, torch.bfloat16, s, "v"), _cuda(out, torch.bfloat16, s, "o"),
                                           _stream(stream)), "arl2_frame_query")
         return out
 
     def commit(self, k, v, alpha, beta, stream=None) -> None:
         s, g = self.act_shape, self.gate_shape
-        _check(self._lib.arl2_frame_commit(self._ctx, _dev(k, torch.bfloat16, s, "k"), _dev(v, torch.bfloat16, s, "v"),
-                                           _dev(alpha, torch.float32, g, "alpha"), _dev(beta, torch.float32, g, "beta"),
+        _check(self._lib.arl2_frame_commit(self._ctx, _cuda(k, torch.bfloat16, s, "k"), _cuda(v, torch.bfloat16, s, "v"),
+                                           _cuda(alpha, torch.float32, g, "alpha"), _cuda(beta, torch.float32, g, "beta"),
                                            _stream(stream)), "arl2_frame_commit")
 
     def query_host(self, q, k, v, out, stream=None) -> torch.Tensor:
         """Host-buffer query: q, k, v, out are CPU tensors (pinned for asynchrony)."""
         s = self.act_shape
-        _check(self._lib.arl2_frame_query_host(self._ctx, _dev(q, torch.bfloat16, s, "q"),
-                                               _dev(k, torch.bfloat16, s, "k"), _dev(v, torch.bfloat16, s, "v"),
-                                               _dev(out, torch.bfloat16, s, "o"), _stream(stream)),
+        _check(self._lib.arl2_frame_query_host(self._ctx, _host(q, torch.bfloat16, s, "q"),
+                                               _host(k, torch.bfloat16, s, "k"), _host(v, torch.bfloat16, s, "v"),
+                                               _host(out, torch.bfloat16, s, "o"), _stream(stream)),
                "arl2_frame_query_host")
         return out
 
     def commit_host(self, k, v, alpha, beta, stream=None) -> None:
         s, g = self.act_shape, self.gate_shape
-        _check(self._lib.arl2_frame_commit_host(self._ctx, _dev(k, torch.bfloat16, s, "k"),
-                                                _dev(v, torch.bfloat16, s, "v"),
-                                                _dev(alpha, torch.float32, g, "alpha"),
-                                                _dev(beta, torch.float32, g, "beta"), _stream(stream)),
+        _check(self._lib.arl2_frame_commit_host(self._ctx, _host(k, torch.bfloat16, s, "k"),
+                                                _host(v, torch.bfloat16, s, "v"),
+                                                _host(alpha, torch.float32, g, "alpha"),
+                                                _host(beta, torch.float32, g, "beta"), _stream(stream)),
                "arl2_frame_commit_host")
 
     def reset(self, stream=None) -> None:
@@ -237,10 +253,10 @@ def frame_commit_noalloc(k, v, alpha, beta, Wk, Wv, S_prev, S_next, status, stre
         raise ValueError("status: expected one int32 element in device memory")
     status_ptr = status.data_ptr()
     _check(load_library().arl2_frame_commit_noalloc(
-        B, H, T, d, _dev(k, torch.bfloat16, s, "k"), _dev(v, torch.bfloat16, s, "v"),
-        _dev(alpha, torch.float32, g, "alpha"), _dev(beta, torch.float32, g, "beta"),
-        _dev(Wk, torch.bfloat16, w, "Wk"), _dev(Wv, torch.bfloat16, w, "Wv"),
-        _dev(S_prev, torch.float32, st, "S_prev"), _dev(S_next, torch.float32, st, "S_next"),
+        B, H, T, d, _cuda(k, torch.bfloat16, s, "k"), _cuda(v, torch.bfloat16, s, "v"),
+        _cuda(alpha, torch.float32, g, "alpha"), _cuda(beta, torch.float32, g, "beta"),
+        _cuda(Wk, torch.bfloat16, w, "Wk"), _cuda(Wv, torch.bfloat16, w, "Wv"),
+        _cuda(S_prev, torch.float32, st, "S_prev"), _cuda(S_next, torch.float32, st, "S_next"),
         status_ptr, _stream(stream)), "arl2_frame_commit_noalloc")
 
 
@@ -273,14 +289,14 @@ class KVCacheBaseline:
         if out is None:
             out = torch.empty(self.act_shape, dtype=torch.bfloat16, device=q.device)
         s = self.act_shape
-        _check(self._lib.arl2_kvcache_query(self._c, _dev(q, torch.bfloat16, s, "q"), _dev(k, torch.bfloat16, s, "k"),
-                                            _dev(v, torch.bfloat16, s, "v"), _dev(out, torch.bfloat16, s, "o"),
+        _check(self._lib.arl2_kvcache_query(self._c, _cuda(q, torch.bfloat16, s, "q"), _cuda(k, torch.bfloat16, s, "k"),
+                                            _cuda(v, torch.bfloat16, s, "v"), _cuda(out, torch.bfloat16, s, "o"),
                                             _stream(stream)), "arl2_kvcache_query")
         return out
 
     def commit(self, k, v, stream=None) -> None:
         s = self.act_shape
-        _check(self._lib.arl2_kvcache_commit(self._c, _dev(k, torch.bfloat16, s, "k"), _dev(v, torch.bfloat16, s, "v"),
+        _check(self._lib.arl2_kvcache_commit(self._c, _cuda(k, torch.bfloat16, s, "k"), _cuda(v, torch.bfloat16, s, "v"),
                                              _stream(stream)), "arl2_kvcache_commit")
 
     def reset(self) -> None:
