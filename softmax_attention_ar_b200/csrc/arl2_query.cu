@@ -614,13 +614,15 @@ __device__ __forceinline__ void merge_rows(const QueryArgs& a, const Seg& sg, ui
 // record's flag. Loads are issued in batches so their latencies overlap. Kept out of line
 // so its registers do not compete with the softmax loop; the launch arguments it reads stay
 // in parameter space (the kernel takes them as a grid constant), not in a per-thread copy
-// in local memory. Returns false if a wait gave up.
+// in local memory; the small structs come by value for the same reason. Returns the number
+// of group rendezvous it took (0 or 1), or -1 if a wait gave up.
 template <bool kHybrid>
-__device__ __noinline__ bool segment_epilogue(const Smem& sm, const QueryArgs& a, const Seg& sg, int first_rec,
-                                              int last_nsegs, uint32_t r, int half, int c0, int ncols, uint32_t tO,
-                                              uint32_t tX, float m, float l_row, uint32_t& gphase,
-                                              volatile int* merge_ok, const float* stage, int rs,
-                                              const CUtensorMap* tm_o, const Guard& g) {
+__device__ __noinline__ int segment_epilogue(const Smem sm, const QueryArgs& a, const Seg sg, int first_rec,
+                                             int last_nsegs, uint32_t r, int half, int c0, int ncols, uint32_t tO,
+                                             uint32_t tX, float m, float l_row, uint32_t gphase,
+                                             volatile int* merge_ok, const float* stage, int rs,
+                                             const CUtensorMap* tm_o, const Guard g) {
+  const uint32_t gphase0 = gphase;
   const int q0 = c0 / 4;   // this half's first column quad
   // First global write of this thread in the launch: a query launched as the programmatic
   // dependent of the previous one waits for it here (shared scratch, maybe the same output).
@@ -646,7 +648,7 @@ __device__ __noinline__ bool segment_epilogue(const Smem& sm, const QueryArgs& a
     tc_fence_before();
     warp_arrive(sm.bar(kBarOEmpty));   // TMEM read: the next segment may reuse O
     warp_arrive(sm.bar(kBarRec));      // record stored: the publisher may raise its flag
-    return true;
+    return 0;
   }
   // Head segment: the tile's other records (if any), then the merge. Warp 3 stages them
   // in shared memory when they fit; otherwise they are read from scratch here.
@@ -655,15 +657,15 @@ __device__ __noinline__ bool segment_epilogue(const Smem& sm, const QueryArgs& a
   const int k1 = (rs + 1) % kStages, k2 = (rs + 2) % kStages;   // idle ring stages (see staged_merge)
   if (staged) {
     // At most one staged merge per CTA and launch: the barrier completes once (phase 0).
-    if (!mbar_wait_warp(sm.bar(kBarRecLoad), 0, g)) return false;
+    if (!mbar_wait_warp(sm.bar(kBarRecLoad), 0, g)) return -1;
   } else if (nsegs > 1) {
     if (half == 0 && r == 0) {
       bool ok = true;
       for (int s = 1; s < nsegs && ok; ++s) ok = wait_flag(a.flags + slot0 + s, a.epoch, g);
       *merge_ok = ok ? 1 : 0;
     }
-    if (!group_sync(sm.bar(kBarGroup), gphase, g)) return false;
-    if (!*merge_ok) return false;
+    if (!group_sync(sm.bar(kBarGroup), gphase, g)) return -1;
+    if (!*merge_ok) return -1;
   }
   const uint32_t otile = sm.v(k2);   // staged: the output tile (two 128-byte-swizzled panels)
   if (staged)
@@ -686,7 +688,7 @@ __device__ __noinline__ bool segment_epilogue(const Smem& sm, const QueryArgs& a
   }
   tc_fence_before();
   warp_arrive(sm.bar(kBarOEmpty));
-  return true;
+  return static_cast<int>(gphase - gphase0);
 }
 
 // Warp 3. (1) Raises the flag of each partial record this CTA stores, once the softmax
@@ -850,9 +852,11 @@ __device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const 
     tc_fence_after();
     float l0, l1;
     if (!pair_swap(pair_bar, xch, nx, half, r, l, l0, l1, g)) return;
-    if (!segment_epilogue<kHybrid>(sm, a, sg, sch.first_rec, sch.last_nsegs, r, half, c0, ncols, tO, tX, m, l0 + l1,
-                                   gphase, merge_ok, reinterpret_cast<const float*>(ctl - kTileRegion), rs, tm_o, g))
-      return;
+    const int syncs =
+        segment_epilogue<kHybrid>(sm, a, sg, sch.first_rec, sch.last_nsegs, r, half, c0, ncols, tO, tX, m, l0 + l1,
+                                  gphase, merge_ok, reinterpret_cast<const float*>(ctl - kTileRegion), rs, tm_o, g);
+    if (syncs < 0) return;
+    gphase += static_cast<uint32_t>(syncs);
     ++nseg;
   }
 }
