@@ -181,9 +181,11 @@ void arl2_destroy(arl2_ctx* ctx);
  * The call allocates nothing. Its scratch is a fixed device array of
  * ARL2_NOALLOC_SCRATCH_BYTES inside the library. Every GPU that loads the library holds
  * that array until the process exits. Shapes whose scratch would exceed it return
- * ARL2_ERR_UNSUPPORTED before any work is enqueued. The need is about B*H*d*d*4 bytes
- * (bf16 copies of S_prev and S_next; the chunk groups' partial sums meet in on-chip
- * memory); B=1, H=12, d=128 needs about 0.8 MB, and d=128 fits up to B*H = 256.
+ * ARL2_ERR_UNSUPPORTED before any work is enqueued. The need is about
+ * B*H*(d*d*4 + G*64 KiB) bytes: bf16 copies of S_prev and S_next, and the partial update of
+ * each of the G <= 8 groups of 128-token chunks a (batch, head) is split into (G = 7 at
+ * T = 1560). B=1, H=12, T=1560, d=128 needs about 6.1 MB; at G = 8 the array fits
+ * B*H <= 28.
  *
  * The first call on a device looks the array's device address up, with that device
  * current. Make that first call before any stream capture. All calls on a device share

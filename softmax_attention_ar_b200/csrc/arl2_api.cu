@@ -182,6 +182,7 @@ struct arl2_ctx {
   cudaEvent_t ev_in[2] = {}, ev_used[2] = {}, ev_out[2] = {};
   unsigned host_turn = 0;
   arl2::QueryPlan qplan{};        // stream-K split of the query kernel
+  float* cscratch = nullptr;      // the commit's per-group partial U and alpha sums
   float* qscratch = nullptr;      // its partial records
   int* qflags = nullptr;          // their published flags
   int qepoch = 0;                 // epoch of the last query launch
@@ -272,6 +273,7 @@ void free_ctx(arl2_ctx* c) {
   if (c->s_out) cudaStreamDestroy(c->s_out);
   cudaFree(c->qscratch);
   cudaFree(c->qflags);
+  cudaFree(c->cscratch);
   delete c;
 }
 
@@ -326,6 +328,8 @@ arl2_status commit_impl(arl2_ctx* c, const void* k, const void* v, const float* 
   r.S_old = c->S[c->cur];
   r.S_new = c->S[c->cur ^ 1];
   r.S_new_bf16 = c->S_bf16 + (size_t)(c->cur ^ 1) * c->state_elems();
+  r.part_u = c->cscratch;
+  r.part_alpha = c->cscratch + arl2::commit_scratch_floats(c->B, c->H, c->ngroups) - (size_t)c->B * c->H * c->ngroups;
   r.d = c->d;
   r.inv_T = a.inv_T;
   const size_t act = c->act_elems() * 2, gate = (size_t)c->B * c->H * c->T * 4;
@@ -373,6 +377,7 @@ arl2_status arl2_create(int H, int T, int d_k, int d_v, int B, arl2_ctx** out) {
   c->qplan = arl2::plan_query(B, H, T, T, sms);
   ok = ok && dev_alloc(&c->qscratch, arl2::query_scratch_floats(c->qplan), &c->bytes);
   ok = ok && dev_alloc(&c->qflags, arl2::query_flag_count(c->qplan), &c->bytes);
+  ok = ok && dev_alloc(&c->cscratch, arl2::commit_scratch_floats(B, H, c->ngroups), &c->bytes);
   if (!ok) {
     free_ctx(c);
     return ARL2_ERR_OOM;

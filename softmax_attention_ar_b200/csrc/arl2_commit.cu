@@ -11,18 +11,22 @@
 //     Vp -= K' S_{N-1}                (MMA with the B operand negated, S from its bf16 copy)
 //     R  = Vp beta_t / T              (thread = token row; bf16 over the V tile)
 //     U += K'^T R                     (MMA, both operands MN-major; accumulates over the chunks)
-// Chunk i+1's K projection runs while the rows normalise chunk i (Kp is double-buffered).
-// Then every CTA pushes each row of its U, and its sum of alpha, to the CTA of the cluster
-// that owns that row of S_N (distributed shared memory), and each CTA sums its rows in a
-// fixed order (the result does not depend on timing) and writes S_N in fp32 and bf16. One
-// launch, no scratch in global memory.
+// The first K projection starts as soon as W_k and the first K tile have landed; chunk i+1's
+// K projection runs while the rows normalise chunk i (Kp is double-buffered).
+//
+// Reduction through L2. Every CTA writes its partial U (fp32, column-quad-major so that a
+// warp's stores are contiguous) and its sum of alpha to a scratch slot of its own, then the
+// cluster meets once at a barrier (release/acquire: the partials are visible after it). CTA
+// g then owns a block of columns of S_N: for each of its elements it sums the G partials in
+// a fixed order (the result does not depend on timing), adds abar S_{N-1} and writes S_N in
+// fp32 and bf16. The scratch is private to the launch's own clusters and is fully written
+// before it is read, so it never needs clearing.
 //
 // Roles (192 threads): warp 0 TMA, warp 1 TMEM owner and MMA issuer (warp-wide loop, one
 // elected lane issues), warps 2-5 row warps (thread = token row for K' and R, = state row k
-// for the U staging).
+// for writing U). Every thread takes part in the owner phase.
 // TMEM: Kp of even chunks at 0, Vp at 128, U at 256, Kp of odd chunks at 384.
-// Shared memory: Wk | Wv | S | K0 K1 | V0 V1 (32 KiB tiles), then a control block. After
-// every MMA is done the Wk, Wv and S tiles hold the receive buffer of the reduction.
+// Shared memory: Wk | Wv | S | K0 K1 | V0 V1 (32 KiB tiles), then a control block.
 #include <algorithm>
 
 #include "arl2_device.cuh"
@@ -38,29 +42,27 @@ constexpr uint32_t kWvOff = kTileBytes;
 constexpr uint32_t kSOff = 2 * kTileBytes;
 constexpr uint32_t kKOff = 3 * kTileBytes;   // two stages
 constexpr uint32_t kVOff = 5 * kTileBytes;   // two stages
-// Receive buffer of the cluster reduction, over Wk | Wv | S: [G][32 column quads][rows per
-// CTA] float4, at most (128 + G - 1) * 512 bytes.
-constexpr uint32_t kRecvOff = kWkOff;
 constexpr uint32_t kCtlOff = 7 * kTileBytes;
 enum : int {
-  kBarW = 0,          // Wk, Wv landed
-  kBarKVFull = 1,     // +stage (2)
-  kBarKVEmpty = 3,    // +stage
-  kBarProjK = 5,      // +Kp buffer (2): Kp of the chunk in TMEM
-  kBarKn = 7,         // K' bf16 over the K tile (one arrival per row warp)
-  kBarKS = 8,         // Vp - K'S in TMEM
-  kBarR = 9,          // R bf16 over the V tile (one arrival per row warp)
-  kBarU = 10,         // U complete
-  kBarFinal = 11,     // every MMA done (drain before TMEM is freed)
-  kBarS = 12,         // the bf16 copy of S_{N-1} landed
-  kNumBars = 13
+  kBarWk = 0,         // Wk landed
+  kBarWv = 1,         // Wv landed
+  kBarS = 2,          // the bf16 copy of S_{N-1} landed
+  kBarKFull = 3,      // +stage (2): K chunk tile landed
+  kBarVFull = 5,      // +stage (2): V chunk tile landed
+  kBarKVEmpty = 7,    // +stage (2): the chunk's last MMA (K'^T R) is done with its K and V tiles
+  kBarProjK = 9,      // +Kp buffer (2): Kp of the chunk in TMEM
+  kBarKn = 11,        // K' bf16 over the K tile (one arrival per row warp)
+  kBarKS = 12,        // Vp - K'S in TMEM
+  kBarR = 13,         // R bf16 over the V tile (one arrival per row warp)
+  kBarU = 14,         // U complete
+  kBarFinal = 15,     // every MMA done (drain before TMEM is freed)
+  kNumBars = 16
 };
-constexpr uint32_t kCtlMisc = 128;           // tmem slot, abort flag, alpha sums, status
+constexpr uint32_t kCtlMisc = 128;           // tmem slot, abort flag, rows-failed flag, warp alpha sums
 constexpr uint32_t kSmemBytes = kCtlOff + kCtlMisc + 64;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;   // room to align the base to 1 KiB
 static_assert(kNumBars * 8 <= kCtlMisc, "barriers must fit their slot");
 static_assert(kSmemAlloc <= 232448, "shared memory per CTA");
-static_assert(kRecvOff + (kDP + kMaxCluster - 1) * kDP * 4 <= kKOff, "the receive buffer must fit Wk, Wv and S");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColKp0 = 0, kColVp = 128, kColU = 256, kColKp1 = 384;
 constexpr float kNormEps = 1e-12f;
@@ -77,50 +79,60 @@ struct Smem {
 };
 __device__ __forceinline__ uint32_t col_kp(int i) { return (i & 1) ? kColKp1 : kColKp0; }
 
-// Warp 0 (warp-wide, lead lane issues): Wk and Wv once, the first K and V chunk tiles, then
-// the bf16 S once, then the remaining K and V chunk tiles through two stages. S_{N-1} is the
-// previous commit's output; when this grid was launched as a programmatic dependent of the
-// kernel before it, that output is visible only after griddepcontrol.wait, so S waits for
-// it and goes out after the first chunk (the projections do not need S).
+// Warp 0 (warp-wide, lead lane issues). Order: Wk and the first K tile (the first MMA needs
+// only these), Wv and the first V tile, the second chunk's tiles, then the bf16 S, then the
+// remaining chunks through two stages. S_{N-1} is the previous commit's output; when this
+// grid was launched as a programmatic dependent of the kernel before it, that output is
+// visible only after griddepcontrol.wait, so the S load waits for it. The K and V tiles are
+// this frame's activations, read once: they are loaded with an evict-first L2 policy.
 __device__ void producer(const Smem& sm, const CUtensorMap* tm_k, const CUtensorMap* tm_v, const CUtensorMap* tm_wk,
                          const CUtensorMap* tm_wv, const CUtensorMap* tm_s, const CommitArgs& a, int c0, int nc,
                          int h, int b, bool lead, const Guard& g) {
-  uint32_t n[2] = {0, 0};
+  uint32_t nk[2] = {0, 0};
   const int slot = a.state_slot * a.B * a.H + b * a.H + h;
-  if (lead) {
-    mbar_expect_tx(sm.bar(kBarW), 2 * kTileBytes);
-    for (int p = 0; p < 2; ++p) {
-      tma_load_3d(sm.wk() + p * kPanelBytes, tm_wk, sm.bar(kBarW), 64 * p, 0, h);
-      tma_load_3d(sm.wv() + p * kPanelBytes, tm_wv, sm.bar(kBarW), 64 * p, 0, h);
-    }
-  }
-  auto load_s = [&]() {
-    griddep_wait();
+  const uint64_t stream_policy = l2_evict_first_policy();
+  auto load_tile = [&](const CUtensorMap* map, uint32_t dst, int bar, int i) {
     if (lead) {
-      mbar_expect_tx(sm.bar(kBarS), kTileBytes);
-      for (int p = 0; p < 2; ++p) tma_load_3d(sm.s() + p * kPanelBytes, tm_s, sm.bar(kBarS), 64 * p, 0, slot);
+      mbar_expect_tx(sm.bar(bar), kTileBytes);
+      for (int p = 0; p < 2; ++p)
+        tma_load_4d_hint(dst + p * kPanelBytes, map, sm.bar(bar), 64 * p, h, (c0 + i) * kRows, b, stream_policy);
     }
-    __syncwarp();
   };
-  if (nc == 0) load_s();
-  for (int i = 0; i < nc; ++i) {
-    const int s = i & 1;
-    if (i >= 2 && !mbar_wait_warp(sm.bar(kBarKVEmpty + s), ((i - 2) >> 1) & 1, g)) break;
-    const int row = (c0 + i) * kRows;
+  auto load_weight = [&](const CUtensorMap* map, uint32_t dst, int bar, int c2) {
     if (lead) {
-      mbar_expect_tx(sm.bar(kBarKVFull + s), 2 * kTileBytes);
-      for (int p = 0; p < 2; ++p) {
-        tma_load_4d(sm.k(s) + p * kPanelBytes, tm_k, sm.bar(kBarKVFull + s), 64 * p, h, row, b);
-        tma_load_4d(sm.v(s) + p * kPanelBytes, tm_v, sm.bar(kBarKVFull + s), 64 * p, h, row, b);
-      }
+      mbar_expect_tx(sm.bar(bar), kTileBytes);
+      for (int p = 0; p < 2; ++p) tma_load_3d(dst + p * kPanelBytes, map, sm.bar(bar), 64 * p, 0, c2);
     }
-    ++n[s];
-    if (i == 0) load_s();
+  };
+  auto load_chunk = [&](int i) {
+    load_tile(tm_k, sm.k(i & 1), kBarKFull + (i & 1), i);
+    load_tile(tm_v, sm.v(i & 1), kBarVFull + (i & 1), i);
+    ++nk[i & 1];
+  };
+  load_weight(tm_wk, sm.wk(), kBarWk, h);
+  if (nc > 0) load_tile(tm_k, sm.k(0), kBarKFull, 0);
+  load_weight(tm_wv, sm.wv(), kBarWv, h);
+  if (nc > 0) {
+    load_tile(tm_v, sm.v(0), kBarVFull, 0);
+    ++nk[0];
   }
-  mbar_wait_drain(sm.bar(kBarW), 0);
+  if (nc > 1) load_chunk(1);
+  griddep_wait();
+  load_weight(tm_s, sm.s(), kBarS, slot);
+  __syncwarp();
+  for (int i = 2; i < nc; ++i) {
+    if (!mbar_wait_warp(sm.bar(kBarKVEmpty + (i & 1)), ((i - 2) >> 1) & 1, g)) break;
+    load_chunk(i);
+  }
+  // Every load issued must land before the CTA may exit (matters only after an abort).
+  mbar_wait_drain(sm.bar(kBarWk), 0);
+  mbar_wait_drain(sm.bar(kBarWv), 0);
   mbar_wait_drain(sm.bar(kBarS), 0);
   for (int s = 0; s < 2; ++s)
-    if (n[s]) mbar_wait_drain(sm.bar(kBarKVFull + s), (n[s] - 1) & 1);
+    if (nk[s]) {
+      mbar_wait_drain(sm.bar(kBarKFull + s), (nk[s] - 1) & 1);
+      mbar_wait_drain(sm.bar(kBarVFull + s), (nk[s] - 1) & 1);
+    }
 }
 
 // Warp 1 (warp-wide, lead lane issues every MMA and commit).
@@ -137,11 +149,13 @@ __device__ void mma_issuer(const Smem& sm, uint32_t tmem, int nc, bool lead, con
   auto proj_v = [&](int i) {   // Vp of chunk i from V stage i % 2
     if (lead) mma8_ss<false, true>(tmem + kColVp, desc_kmajor(sm.v(i & 1), 0), desc_mnmajor(sm.wv(), 0), id_kmn, 0u);
   };
+  auto chunk_ready = [&](int bar0, int i) { return mbar_wait_warp(sm.bar(bar0 + (i & 1)), (i >> 1) & 1, g); };
   if (nc > 0) {
-    if (!mbar_wait_warp(sm.bar(kBarW), 0, g)) return;
-    if (!mbar_wait_warp(sm.bar(kBarKVFull), 0, g)) return;
+    if (!mbar_wait_warp(sm.bar(kBarWk), 0, g) || !chunk_ready(kBarKFull, 0)) return;
     tc_fence_after();
     proj_k(0);
+    if (!mbar_wait_warp(sm.bar(kBarWv), 0, g) || !chunk_ready(kBarVFull, 0)) return;
+    tc_fence_after();
     proj_v(0);
   }
   for (int i = 0; i < nc; ++i) {
@@ -149,7 +163,7 @@ __device__ void mma_issuer(const Smem& sm, uint32_t tmem, int nc, bool lead, con
     if (i + 1 < nc) {
       // The next chunk's K projection: its Kp buffer was read out (K' of chunk i-1) before
       // this warp issued chunk i-1's K'S.
-      if (!mbar_wait_warp(sm.bar(kBarKVFull + ((i + 1) & 1)), ((i + 1) >> 1) & 1, g)) return;
+      if (!chunk_ready(kBarKFull, i + 1)) return;
       tc_fence_after();
       proj_k(i + 1);
     }
@@ -168,13 +182,18 @@ __device__ void mma_issuer(const Smem& sm, uint32_t tmem, int nc, bool lead, con
       mma8_ss<true, true>(tmem + kColU, desc_mnmajor(sm.k(st), 0), desc_mnmajor(sm.v(st), 0), id_mnmn, i > 0 ? 1u : 0u);
       mma_commit(sm.bar(kBarKVEmpty + st));
     }
-    if (i + 1 < nc) proj_v(i + 1);
+    if (i + 1 < nc) {
+      if (!chunk_ready(kBarVFull, i + 1)) return;
+      tc_fence_after();
+      proj_v(i + 1);
+    }
   }
   if (lead) mma_commit(sm.bar(kBarU));
 }
 
 // Warps 2-5: K' and R per chunk (thread = token row), then wait for U. Returns false if a
-// wait gave up.
+// wait gave up. Sums of squares and the scalings run on paired fp32 operations with
+// independent accumulators, so the row's dependent chains stay short.
 __device__ bool row_role(const Smem& sm, uint32_t tmem, const CommitArgs& a, int c0, int nc, int h, int b, int warp,
                          int lane, float* warp_sums, const Guard& g) {
   const int quarter = warp & 3;
@@ -206,23 +225,32 @@ __device__ bool row_role(const Smem& sm, uint32_t tmem, const CommitArgs& a, int
       uint32_t kv[4][32];
       tmem_ld32x2_wait(tmem + lane_off + col_kp(i), kv[0], tmem + lane_off + col_kp(i) + 32u, kv[1]);
       tmem_ld32x2_wait(tmem + lane_off + col_kp(i) + 64u, kv[2], tmem + lane_off + col_kp(i) + 96u, kv[3]);
-      float ss = 0.f;
+      float2 ss[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) ss[j] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int e = 0; e < 32; ++e) ss = fmaf(__uint_as_float(kv[c][e]), __uint_as_float(kv[c][e]), ss);
-      const float inv = 1.f / fmaxf(sqrtf(ss), kNormEps);
+        for (int e = 0; e < 32; e += 2) {
+          const float2 x = make_float2(__uint_as_float(kv[c][e]), __uint_as_float(kv[c][e + 1]));
+          ss[(e >> 1) & 3] = __ffma2_rn(x, x, ss[(e >> 1) & 3]);
+        }
+      const float2 s01 = __fadd2_rn(__fadd2_rn(ss[0], ss[1]), __fadd2_rn(ss[2], ss[3]));
+      const float inv = 1.f / fmaxf(sqrtf(s01.x + s01.y), kNormEps);
+      const float2 inv2 = make_float2(inv, inv);
       const uint32_t tile = sm.k(st);
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const uint32_t* x = kv[c] + 8 * q;
-          st_shared_v4(tile + swz_chunk(r, 4 * c + q),
-                       pack_bf16x2(__uint_as_float(x[0]) * inv, __uint_as_float(x[1]) * inv),
-                       pack_bf16x2(__uint_as_float(x[2]) * inv, __uint_as_float(x[3]) * inv),
-                       pack_bf16x2(__uint_as_float(x[4]) * inv, __uint_as_float(x[5]) * inv),
-                       pack_bf16x2(__uint_as_float(x[6]) * inv, __uint_as_float(x[7]) * inv));
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 y = __fmul2_rn(make_float2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), inv2);
+            w[e] = pack_bf16x2(y.x, y.y);
+          }
+          st_shared_v4(tile + swz_chunk(r, 4 * c + q), w[0], w[1], w[2], w[3]);
         }
     }
     fence_proxy_async_smem();
@@ -231,18 +259,27 @@ __device__ bool row_role(const Smem& sm, uint32_t tmem, const CommitArgs& a, int
     // R = (Vp - K'S) * beta_t / T -> bf16, over the V tile (its MMA has finished).
     if (!mbar_wait_warp(sm.bar(kBarKS), i & 1, g)) return false;
     tc_fence_after();
-    const uint32_t tile = sm.v(st);
+    {
+      const uint32_t tile = sm.v(st);
+      const float2 cf = make_float2(coef, coef);
+      uint32_t vp[2][32];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t vp[32];
-      tmem_ld32_wait(tmem + lane_off + kColVp + 32u * c, vp);
+      for (int c2 = 0; c2 < 2; ++c2) {
+        tmem_ld32x2_wait(tmem + lane_off + kColVp + 64u * c2, vp[0], tmem + lane_off + kColVp + 64u * c2 + 32u,
+                         vp[1]);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float y[8];
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) y[e] = __uint_as_float(vp[8 * q + e]) * coef;
-        st_shared_v4(tile + swz_chunk(r, 4 * c + q), pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
-                     pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
+          for (int q = 0; q < 4; ++q) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 y = __fmul2_rn(
+                  make_float2(__uint_as_float(vp[c][8 * q + 2 * e]), __uint_as_float(vp[c][8 * q + 2 * e + 1])), cf);
+              w[e] = pack_bf16x2(y.x, y.y);
+            }
+            st_shared_v4(tile + swz_chunk(r, 4 * (2 * c2 + c) + q), w[0], w[1], w[2], w[3]);
+          }
       }
     }
     fence_proxy_async_smem();
@@ -254,19 +291,23 @@ __device__ bool row_role(const Smem& sm, uint32_t tmem, const CommitArgs& a, int
   for (int o = 16; o > 0; o >>= 1) asum += __shfl_xor_sync(0xffffffffu, asum, o);
   if (lane == 0) warp_sums[quarter] = asum;
 
-  // U is complete (every MMA of this CTA is done); the tail pushes it to its owners.
+  // U is complete (every MMA of this CTA is done).
   if (!mbar_wait_warp(sm.bar(kBarU), 0, g)) return false;
   tc_fence_after();
   return true;
 }
 
+// Scratch slot of (batch-head bh, group g): [32 column quads][128 rows] float4.
+__device__ __forceinline__ float4* part_slot(float* part_u, size_t bh, int G, int g) {
+  return reinterpret_cast<float4*>(part_u) + (bh * G + g) * (32 * kRows);
+}
+
 __global__ void __launch_bounds__(kThreadsC, 1)
     arl2_commit_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                        const __grid_constant__ CUtensorMap tm_wk, const __grid_constant__ CUtensorMap tm_wv,
-                       const __grid_constant__ CUtensorMap tm_s, const CommitArgs a, const ReduceArgs rd) {
+                       const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CommitArgs a,
+                       const __grid_constant__ ReduceArgs rd) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  // Align the base to 1 KiB. The offset is the same in every CTA of the cluster (same
-  // kernel, same dynamic shared memory), so a peer's staging sits at the same address.
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
@@ -274,32 +315,20 @@ __global__ void __launch_bounds__(kThreadsC, 1)
   uint8_t* ctl = gbase + kCtlOff;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + kCtlMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + kCtlMisc + 4);
-  float* alpha_cta = reinterpret_cast<float*>(ctl + kCtlMisc + 8);
-  volatile int* rows_failed = reinterpret_cast<volatile int*>(ctl + kCtlMisc + 12);
+  volatile int* rows_failed = reinterpret_cast<volatile int*>(ctl + kCtlMisc + 8);
   float* warp_sums = reinterpret_cast<float*>(ctl + kCtlMisc + 16);
-  float* recv_alpha = reinterpret_cast<float*>(ctl + kCtlMisc + 32);   // [G] alpha sums pushed by the CTAs
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y, b = blockIdx.z;
   const int G = static_cast<int>(gridDim.x);   // CTAs of the cluster = chunk groups
-  const uint32_t rank = cluster_rank();         // equals blockIdx.x: the cluster spans x
+  const int rank = static_cast<int>(cluster_rank());   // equals blockIdx.x: the cluster spans x
   const int nchunks = (a.T + kRows - 1) / kRows;
-  const int c0 = static_cast<int>(rank) * a.chunks_per_group;
+  const int c0 = rank * a.chunks_per_group;
   const int nc = max(0, min(a.chunks_per_group, nchunks - c0));
   const Guard g{abort_flag, a.err, a.timeout_ns};
+  const size_t bh = static_cast<size_t>(b) * a.H + h;
 
   if (threadIdx.x == 0) {
-    mbar_init(sm.bar(kBarW), 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(sm.bar(kBarKVFull + s), 1);
-      mbar_init(sm.bar(kBarKVEmpty + s), 1);
-      mbar_init(sm.bar(kBarProjK + s), 1);
-    }
-    mbar_init(sm.bar(kBarKn), kRowWarps);
-    mbar_init(sm.bar(kBarKS), 1);
-    mbar_init(sm.bar(kBarR), kRowWarps);
-    mbar_init(sm.bar(kBarU), 1);
-    mbar_init(sm.bar(kBarFinal), 1);
-    mbar_init(sm.bar(kBarS), 1);
+    for (int i = 0; i < kNumBars; ++i) mbar_init(sm.bar(i), (i == kBarKn || i == kBarR) ? kRowWarps : 1);
     *abort_flag = 0;
     *rows_failed = 0;
     fence_barrier_init();
@@ -330,29 +359,18 @@ __global__ void __launch_bounds__(kThreadsC, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (threadIdx.x == 0) *alpha_cta = (warp_sums[0] + warp_sums[1]) + (warp_sums[2] + warp_sums[3]);
-
-  // ---- S_N from the whole cluster's U. The rows of S_N are split among the CTAs; every
-  // CTA pushes each of its U rows to the CTA that owns it (remote stores into the owner's
-  // receive buffer over its Wk/Wv/S tiles, free once that CTA's MMAs are done), then every
-  // CTA sums its rows locally in a fixed order. Every thread of every CTA takes both cluster
-  // barriers on every path, so no CTA can leave its peers waiting. A CTA that gave up wrote
-  // its error bit; the state of that call is then undefined.
   const int d = rd.d;
-  const int rows_per = (d + G - 1) / G;
   const bool ok_here = !*abort_flag && !*rows_failed;
-  cluster_sync();   // 1: every CTA's MMAs are done (its receive buffer is free)
+
+  // This CTA's partial U and alpha sum into its scratch slot (a CTA with no chunk writes
+  // zeros). A CTA that gave up wrote its error bit and skips the write; the state of that
+  // call is then undefined.
   if (ok_here) {
+    float4* slot = part_slot(rd.part_u, bh, G, rank);
     if (warp >= 2) {
-      const uint32_t r = static_cast<uint32_t>(warp & 3) * 32 + lane;
+      const uint32_t r = static_cast<uint32_t>(warp & 3) * 32 + lane;   // state row k == TMEM lane
       const uint32_t lane_off = static_cast<uint32_t>(warp & 3) * 32 << 16;
-      // Rows r < d only: then the owner r / rows_per is a rank of the cluster (< G).
-      const bool row_ok = static_cast<int>(r) < d;
-      const int owner = row_ok ? static_cast<int>(r) / rows_per : 0;
-      const int lr = static_cast<int>(r) - owner * rows_per;
-      // Receive layout [source rank][column quad][row of the owner]: a warp's consecutive
-      // rows store to consecutive 16-byte slots of one owner.
-      const uint32_t dst = row_ok ? peer_smem(sm.base + kRecvOff + (rank * 32u * rows_per + lr) * 16u, owner) : 0u;
+      tc_fence_after();
       for (int c = 0; c < 4; ++c) {
         if (32 * c >= d) break;
         uint32_t u[32];
@@ -362,82 +380,71 @@ __global__ void __launch_bounds__(kThreadsC, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) u[e] = 0u;
         }
-        if (row_ok) {
+        if (static_cast<int>(r) < d) {
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            st_cluster_v4(dst + (8u * c + q) * rows_per * 16u,
-                          make_float4(__uint_as_float(u[4 * q]), __uint_as_float(u[4 * q + 1]),
-                                      __uint_as_float(u[4 * q + 2]), __uint_as_float(u[4 * q + 3])));
+            slot[(8 * c + q) * kRows + r] = make_float4(__uint_as_float(u[4 * q]), __uint_as_float(u[4 * q + 1]),
+                                                       __uint_as_float(u[4 * q + 2]), __uint_as_float(u[4 * q + 3]));
         }
       }
-    } else if (threadIdx.x < static_cast<unsigned>(G)) {
-      // Threads 0..G-1: this CTA's alpha sum into slot `rank` of CTA threadIdx.x.
-      st_cluster_f32(peer_smem(smem_u32(recv_alpha + rank), threadIdx.x), *alpha_cta);
+    } else if (threadIdx.x == 0) {
+      rd.part_alpha[bh * G + rank] = (warp_sums[0] + warp_sums[1]) + (warp_sums[2] + warp_sums[3]);
     }
   }
-  // This CTA's rows of S_{N-1} go to L2 ahead of the barrier (no other CTA writes them). The
-  // reduction below is a plain rolled loop: it runs once per launch, and when its code is
-  // not cached (the commit runs once per frame) a long unrolled body costs more in
-  // instruction fetch than it saves.
+  // This CTA's columns of S_{N-1} go to L2 ahead of the barrier (no other CTA writes them):
+  // for each row, the 128-byte lines that hold the first and last of its columns.
   const int quads = d / 4;
-  const int k0 = static_cast<int>(rank) * rows_per, k1 = min(d, k0 + rows_per);
-  const int items = (k1 > k0 ? k1 - k0 : 0) * quads;
-  const size_t bh = static_cast<size_t>(b) * a.H + h;
+  const int qpo = (quads + G - 1) / G;   // column quads owned per CTA
+  const int q0 = min(quads, rank * qpo), q1 = min(quads, q0 + qpo);
   const size_t dd = static_cast<size_t>(d) * d;
-  if (ok_here) {
-    const int lines = (d + 31) / 32;   // 128-byte lines per row
-    for (int i = threadIdx.x; i < (k1 - k0) * lines; i += kThreadsC)
-      prefetch_l2(rd.S_old + bh * dd + static_cast<size_t>(k0 + i / lines) * d + 32 * (i % lines));
-  }
-  cluster_sync();   // 2: every push has landed
-  if (ok_here) {
-    float asum = 0.f;
-    for (int j = 0; j < G; ++j) asum += recv_alpha[j];
-    const float abar = asum * rd.inv_T;
-    const float* S_old = rd.S_old + bh * dd;
-    float* S_new = rd.S_new + bh * dd;
-    uint16_t* S_new_bf16 = rd.S_new_bf16 + bh * dd;
-    const float4* recv = reinterpret_cast<const float4*>(gbase + kRecvOff);
-    // Up to kBatch items a thread per pass, their S_{N-1} loads issued together so that one
-    // L2 round trip covers them all (at 480p a single pass covers every item).
-    constexpr int kBatch = 4;
-#pragma unroll 1
-    for (int it0 = threadIdx.x; it0 < items; it0 += kBatch * kThreadsC) {
-      float4 so[kBatch];
-#pragma unroll
-      for (int e = 0; e < kBatch; ++e) {
-        const int it = it0 + e * kThreadsC;
-        if (it < items) {
-          const int lr = it / quads, q = it % quads;
-          so[e] = *reinterpret_cast<const float4*>(S_old + static_cast<size_t>(k0 + lr) * d + 4 * q);
-        }
-      }
-#pragma unroll
-      for (int e = 0; e < kBatch; ++e) {
-        const int it = it0 + e * kThreadsC;
-        if (it >= items) break;
-        const int lr = it / quads, q = it % quads, k = k0 + lr;
-        float4 acc = make_float4(abar * so[e].x, abar * so[e].y, abar * so[e].z, abar * so[e].w);
-#pragma unroll 1
-        for (int j = 0; j < G; ++j) {
-          const float4 u = recv[(j * 32 + q) * rows_per + lr];
-          acc.x += u.x;
-          acc.y += u.y;
-          acc.z += u.z;
-          acc.w += u.w;
-        }
-        *reinterpret_cast<float4*>(S_new + static_cast<size_t>(k) * d + 4 * q) = acc;
-        *reinterpret_cast<uint2*>(S_new_bf16 + static_cast<size_t>(k) * d + 4 * q) =
-            make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
-      }
+  if (ok_here && q1 > q0) {
+    for (int i = threadIdx.x; i < 2 * d; i += kThreadsC) {
+      const int k = i >> 1, col = (i & 1) ? 4 * q1 - 1 : 4 * q0;
+      prefetch_l2(rd.S_old + bh * dd + static_cast<size_t>(k) * d + col);
     }
   }
-
-  if (warp == 1) {
+  __threadfence();
+  tc_fence_before();
+  cluster_sync();   // every CTA's partial is written and visible
+  if (warp == 1) {   // every TMEM read of this CTA happened before the barrier
     tc_fence_after();
     mbar_wait_drain(sm.bar(kBarFinal), 0);
     __syncwarp();
     tmem_dealloc(tmem, kTmemCols);
+  }
+  if (!ok_here) return;
+
+  // Owner phase: S_N over columns [4 q0, 4 q1), every row, from the G partials summed in a
+  // fixed order. Item (row k, quad q), rows fastest, so a warp's partial loads are contiguous.
+  float asum = 0.f;
+  for (int j = 0; j < G; ++j) asum += __ldcg(rd.part_alpha + bh * G + j);
+  const float abar = asum * rd.inv_T;
+  const float* S_old = rd.S_old + bh * dd;
+  float* S_new = rd.S_new + bh * dd;
+  uint16_t* S_new_bf16 = rd.S_new_bf16 + bh * dd;
+  const float4* part0 = part_slot(rd.part_u, bh, G, 0);
+  const int items = d * (q1 - q0);
+#pragma unroll 1
+  for (int it = threadIdx.x; it < items; it += kThreadsC) {
+    const int k = it % d, q = q0 + it / d;
+    const float4 so = *reinterpret_cast<const float4*>(S_old + static_cast<size_t>(k) * d + 4 * q);
+    float4 u[kMaxCluster];
+#pragma unroll
+    for (int j = 0; j < kMaxCluster; ++j)
+      if (j < G) u[j] = __ldcg(part0 + (static_cast<size_t>(j) * 32 + q) * kRows + k);
+    float4 acc = make_float4(abar * so.x, abar * so.y, abar * so.z, abar * so.w);
+#pragma unroll
+    for (int j = 0; j < kMaxCluster; ++j) {
+      if (j < G) {
+        acc.x += u[j].x;
+        acc.y += u[j].y;
+        acc.z += u[j].z;
+        acc.w += u[j].w;
+      }
+    }
+    *reinterpret_cast<float4*>(S_new + static_cast<size_t>(k) * d + 4 * q) = acc;
+    *reinterpret_cast<uint2*>(S_new_bf16 + static_cast<size_t>(k) * d + 4 * q) =
+        make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
   }
 }
 
@@ -469,6 +476,11 @@ void commit_split(int T, int H, int B, int sms, int* chunks_per_group, int* ngro
   *ngroups = ng;
 }
 
+size_t commit_scratch_floats(int B, int H, int ngroups) {
+  const size_t slots = static_cast<size_t>(B) * H * ngroups;
+  return slots * 32 * kRows * 4 + slots;   // partial U, then the alpha sums
+}
+
 cudaError_t commit_setup() {
   return cudaFuncSetAttribute(arl2_commit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(kSmemAlloc));
@@ -478,8 +490,9 @@ cudaError_t launch_commit(const CUtensorMap& tm_k, const CUtensorMap& tm_v, cons
                           const CUtensorMap& tm_wv, const CUtensorMap& tm_s, const CommitArgs& a,
                           const ReduceArgs& r, cudaStream_t stream, bool dependent) {
   // One cluster of a.ngroups CTAs per (batch, head). As a programmatic dependent the kernel
-  // may start while the preceding kernel (a query) still runs: it reads S_{N-1}, k, v and the
-  // gates, none of which a query writes, and writes only the other state buffer.
+  // may start while the preceding kernel (a query) still runs: it reads k, v and the gates,
+  // which a query does not write, before griddepcontrol.wait, and S_{N-1} after it; it writes
+  // only the other state buffer and its own scratch.
   if (a.ngroups < 1 || a.ngroups > kMaxCluster) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(a.ngroups, a.H, a.B);

@@ -56,12 +56,14 @@ struct CommitArgs {
 };
 
 // The commit's output side: S_N = abar * S_{N-1} + sum of the groups' U, fp32 plus its
-// bf16 copy. The groups' U and alpha sums meet in distributed shared memory; nothing goes
-// through global scratch.
+// bf16 copy. Each group writes its U and alpha sum to its own scratch slot; after one
+// cluster barrier each CTA sums its block of columns over the groups in a fixed order.
 struct ReduceArgs {
   const float* S_old;     // [B*H, d, d]
   float* S_new;           // [B*H, d, d]
   uint16_t* S_new_bf16;   // [B*H, d, d]
+  float* part_u;          // [B*H*ngroups][32 column quads][128 rows] float4 partial U
+  float* part_alpha;      // [B*H*ngroups] alpha sums
   int d;
   float inv_T;
 };
@@ -77,6 +79,8 @@ size_t commit_smem_bytes();
 // The commit's work split: 128-token chunks in groups, one CTA per group; the groups of one
 // (batch, head) form one cluster (at most 8 CTAs) and no group is empty.
 void commit_split(int T, int H, int B, int sms, int* chunks_per_group, int* ngroups);
+// Scratch of one commit launch (part_u, then part_alpha), in floats.
+size_t commit_scratch_floats(int B, int H, int ngroups);
 cudaError_t query_setup();   // per-device function attributes
 cudaError_t commit_setup();
 

@@ -9,10 +9,11 @@
 // (k, v, the gates, phi_k, phi_v, S_{N-1}) and the output (S_N). The scratch the commit
 // needs lives in one file-scope device array of fixed size, g_commit_scratch. It holds:
 //   - the bf16 copy of S_{N-1} the MMAs read;
-//   - a discarded bf16 copy of S_N (the kernel writes one for the context's queries).
-// The groups' partial sums meet in distributed shared memory, so they need no scratch. The
-// caller passes a device status word: a kernel whose bounded wait ran out reports it there,
-// and there is no other place it could be read back without a context.
+//   - a discarded bf16 copy of S_N (the kernel writes one for the context's queries);
+//   - the chunk groups' partial sums of the update and of alpha (64 KiB per group and
+//     (batch, head)), which the groups of a cluster reduce after one barrier.
+// The caller passes a device status word: a kernel whose bounded wait ran out reports it
+// there, and there is no other place it could be read back without a context.
 // The array is part of the library's device image, so every GPU that loads the library
 // holds ARL2_NOALLOC_SCRATCH_BYTES of it until the process exits.
 //
@@ -75,11 +76,13 @@ extern "C" arl2_status arl2_frame_commit_noalloc(int B, int H, int T, int d, con
   int cpg = 1, ngroups = 1;
   arl2::commit_split(T, H, B, sms, &cpg, &ngroups);
 
-  // Scratch layout: S_{N-1} bf16 | S_N bf16 (discarded).
+  // Scratch layout: S_{N-1} bf16 | S_N bf16 (discarded) | partial U | partial alpha sums.
   const size_t bh = static_cast<size_t>(B) * H, dd = static_cast<size_t>(d) * d;
   const size_t off_sprev = 0;
   const size_t off_snext = off_sprev + round256(bh * dd * 2);
-  const size_t needed = off_snext + round256(bh * dd * 2);
+  const size_t off_part = off_snext + round256(bh * dd * 2);
+  const size_t part_floats = arl2::commit_scratch_floats(B, H, ngroups);
+  const size_t needed = off_part + round256(part_floats * 4);
   if (needed > kScratchBytes) return ARL2_ERR_UNSUPPORTED;
 
   unsigned char* scratch = nullptr;
@@ -115,6 +118,8 @@ extern "C" arl2_status arl2_frame_commit_noalloc(int B, int H, int T, int d, con
   r.S_old = S_prev;
   r.S_new = S_next;
   r.S_new_bf16 = s_next_bf16;
+  r.part_u = reinterpret_cast<float*>(scratch + off_part);
+  r.part_alpha = r.part_u + part_floats - bh * ngroups;
   r.d = d;
   r.inv_T = a.inv_T;
   return arl2::launch_commit(tm_k, tm_v, tm_wk, tm_wv, tm_s, a, r, st, false) == cudaSuccess ? ARL2_OK

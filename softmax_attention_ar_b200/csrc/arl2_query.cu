@@ -259,13 +259,22 @@ __device__ void producer(const Smem& sm, const CUtensorMap* tm_q, const CUtensor
     return gidx < kStages || mbar_wait_warp(sm.bar(empty0 + ring_stage(gidx)), ring_phase(gidx - kStages), g);
   };
   auto tile_addr = [&](int s) { return kIsK ? sm.k(s) : sm.v(s); };
+  // q, k and v are this launch's activations: evict-first in L2, so they do not push out
+  // what later launches reuse. (A key tile's other readers in this launch still hit L2: the
+  // launch's working set is far below its size.)
+  const uint64_t stream_policy = l2_evict_first_policy();
   while (ok && sch.next(sg)) {
     if (kIsK) {
+      // The next segment's Q tile goes to L2 now, so that its load (issued only once this
+      // segment's MMAs are done with Q) does not wait on HBM.
+      if (lead && sch.u < sch.u1)
+        for (int p = 0; p < 2; ++p) tma_prefetch_4d(tm_q, 64 * p, sch.h, sch.qt * kRows, sch.b);
       if (nseg > 0 && !mbar_wait_warp(sm.bar(kBarQEmpty), (nseg - 1) & 1, g)) break;
       if (lead) {
         mbar_expect_tx(sm.bar(kBarQFull), kTileBytes);
         for (int p = 0; p < 2; ++p)
-          tma_load_4d(sm.q() + p * kPanelBytes, tm_q, sm.bar(kBarQFull), 64 * p, sg.h, sg.qt * kRows, sg.b);
+          tma_load_4d_hint(sm.q() + p * kPanelBytes, tm_q, sm.bar(kBarQFull), 64 * p, sg.h, sg.qt * kRows, sg.b,
+                           stream_policy);
       }
     }
     ++nseg;
@@ -289,7 +298,8 @@ __device__ void producer(const Smem& sm, const CUtensorMap* tm_q, const CUtensor
       if (lead) {
         mbar_expect_tx(sm.bar(full0 + s), kTileBytes);
         for (int p = 0; p < 2; ++p)
-          tma_load_4d(tile_addr(s) + p * kPanelBytes, tm_kv, sm.bar(full0 + s), 64 * p, sg.h, j * kRows, sg.b);
+          tma_load_4d_hint(tile_addr(s) + p * kPanelBytes, tm_kv, sm.bar(full0 + s), 64 * p, sg.h, j * kRows, sg.b,
+                           stream_policy);
       }
       ++nissued[s];
       if (kIsK && ring == 0) {
