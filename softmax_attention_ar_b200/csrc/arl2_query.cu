@@ -32,19 +32,21 @@
 //   warp 2      V producer: V tiles into a three-stage ring. When a segment starts a tile,
 //               the bf16 state copy S_h goes first, through the ring.
 //   warp 3      publisher: raises the flag of each partial record the CTA stores.
-//   warps 4-11  two softmax warpgroups. Thread = query row = TMEM lane; warps 4-7 own
-//               score and output columns 0-63, warps 8-11 columns 64-127. A thread reads
-//               and writes only its own half-row; warps w and w+4 (same rows, same SM
-//               sub-partition) swap half-row maxima through shared memory each tile.
-//               These threads also pack Q' for the readout MMA and write outputs and
-//               partial records. Warp 3 stages the records a merge reads.
+//   warps 4-11  two softmax warpgroups. Warps w and w+4 share a TMEM lane quarter (the
+//               same SM sub-partition). In the tile loop, w takes the quarter's first 16
+//               rows and w+4 the last 16, whole rows of 128 scores through the 16-lane
+//               TMEM shapes, four threads a row, so a row's max and sum need only shuffles.
+//               For the Q' packing and the epilogue, thread = row = TMEM lane, and warps
+//               4-7 own output columns 0-63, warps 8-11 columns 64-127; a row's max and sum
+//               reach that layout through shared memory once per segment. These threads
+//               also write outputs and partial records. Warp 3 stages the records a merge
+//               reads.
 // TMEM (512 columns):
 //   - cols 0, 128, 256: three S tiles. The score MMA of tile t+2 is queued right behind
 //     the P.V MMA of tile t and writes the buffer last read two MMA groups earlier, so no
 //     MMA group overwrites TMEM columns that the group just ahead of it still reads (that
-//     stalls the tensor pipe). P (bf16) overwrites its own S tile, scores 0-63 packed into
-//     columns 0-31 and scores 64-127 into columns 64-95, and feeds the P.V MMA straight
-//     from TMEM.
+//     stalls the tensor pipe). P (bf16 pairs) overwrites the first 64 columns of its own S
+//     tile, keys in order, and feeds the P.V MMA straight from TMEM.
 //   - col 384: O.
 //   - Readout, after the last P.V MMA of a segment holding key tile 0: Q' = Q Wq_h goes to
 //     the S tile of tile t0 + n (fp32, then packed in place to bf16 like P), and
@@ -52,7 +54,7 @@
 //     its first two score tiles into neither of them before its O wait, and its third
 //     (into O_inter's tile) only after that wait.
 // Shared memory: Q | K0 K1 K2 | V0 V1 V2 (32 KiB tiles) from its 1 KiB-aligned base, then a
-// small control block (mbarriers, flags, the half-row exchange slots).
+// small control block (mbarriers, flags, the row-statistics exchange slots).
 //
 // Online softmax: scores are kept in log2 units. The running max m is raised only when a
 // tile's max exceeds it by more than 8 (a factor of 256), so O in TMEM is rescaled rarely.
@@ -87,7 +89,7 @@ enum : int {
   kBarOEmpty = 26,    // the segment's O and O_inter were read (per-warp arrivals)
   kBarFinal = 27,
   kBarGroup = 28,     // bounded rendezvous of the softmax threads (per-warp arrivals)
-  kBarPair = 29,      // +row quarter (4): the two warps of those rows swapped half-row values
+  kBarPair = 29,      // +row quarter (4): the quarter's two warps stored their rows' max and sum
   kBarNever = 33,     // never signalled: target of the failure-detection test hook
   kBarRec = 34,       // a partial record is stored (per-warp arrivals); warp 3 publishes it
   kBarRecLoad = 35,   // the merge inputs of the CTA's last segment are staged in shared memory
@@ -103,8 +105,8 @@ constexpr uint32_t kVOff = kKOff + kStages * kTileBytes;
 constexpr uint32_t kTileRegion = kVOff + kStages * kTileBytes;
 constexpr uint32_t kCtlBars = 0;
 constexpr uint32_t kCtlMisc = 320;           // tmem slot, abort flag, merge flag
-// [2 slots][2 halves][128] fp32: per-tile half-row maxima (slot = tile parity); slot 0
-// also carries the end-of-segment row sums.
+// [2 slots][m | l][128] fp32: each row's max and sum at the end of a segment, on their way
+// from the tile loop's layout to the epilogue's (slot = exchange parity).
 constexpr uint32_t kCtlX = 384;
 constexpr uint32_t kCtlBytes = kCtlX + 2 * 2 * 128 * 4;
 static_assert(kNumBars * 8 <= kCtlMisc, "barriers must fit their slot");
@@ -136,21 +138,6 @@ __device__ __forceinline__ bool group_sync(uint32_t bar, uint32_t& phase, const 
   warp_arrive(bar);
   const bool ok = mbar_wait_warp(bar, phase & 1, g);
   ++phase;
-  return ok;
-}
-
-// The two warps holding the same rows (one per column half) swap one value per row through
-// the exchange slots (double-buffered by exchange count). Returns the half-0 and half-1
-// values in that order, so both warps see identical operands.
-__device__ __forceinline__ bool pair_swap(uint32_t bar, float* xch, uint32_t& nx, int half, uint32_t r, float mine,
-                                          float& v0, float& v1, const Guard& g) {
-  float* xs = xch + (nx & 1) * 256;
-  xs[half * 128 + r] = mine;
-  warp_arrive(bar);
-  const bool ok = mbar_wait_warp(bar, nx & 1, g);
-  ++nx;
-  v0 = xs[r];
-  v1 = xs[128 + r];
   return ok;
 }
 
@@ -358,7 +345,10 @@ __device__ void mma_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, co
   constexpr uint32_t id_kk = idesc_bf16(128, 128, false, false);   // A, B K-major
   constexpr uint32_t id_kmn = idesc_bf16(128, 128, false, true);   // A K-major (smem or TMEM), B MN-major
   const uint32_t tO = tmem + kColO;
-  const uint32_t kPacked[8] = {0, 8, 16, 24, 64, 72, 80, 88};   // see the TMEM layout above
+  // A operands in TMEM, by K step of 16: P packed by the softmax's .16x128b stores (its
+  // 64 words in order), and Q' packed in place by column halves (words 0-31 and 64-95).
+  const uint32_t kPackedP[8] = {0, 8, 16, 24, 32, 40, 48, 56};
+  const uint32_t kPackedQ[8] = {0, 8, 16, 24, 64, 72, 80, 88};
   uint32_t nseg = 0, nhead = 0, tile = 0, ring = 0;
   Sched sch(a, blockIdx.x);
   Seg sg;
@@ -426,7 +416,7 @@ __device__ void mma_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, co
       tc_fence_after();
       const uint32_t tP = tmem + 128u * sb;
       if (lead) {
-        mma8_ts(tO, tP, kPacked, desc_mnmajor(sm.v(vs), 0), id_kmn, i > 0 ? 1u : 0u);
+        mma8_ts(tO, tP, kPackedP, desc_mnmajor(sm.v(vs), 0), id_kmn, i > 0 ? 1u : 0u);
         mma_commit(sm.bar(kBarPVDone + sb));
         mma_commit(sm.bar(kBarVEmpty + vs));
       }
@@ -449,7 +439,7 @@ __device__ void mma_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, co
       if (!mbar_wait_warp(sm.bar(kBarVFull + rs), ring_phase(r_rd), g)) return;
       tc_fence_after();
       if (lead) {
-        mma8_ts(tX, tY, kPacked, desc_mnmajor(sm.v(rs), 0), id_kmn, 0u);
+        mma8_ts(tX, tY, kPackedQ, desc_mnmajor(sm.v(rs), 0), id_kmn, 0u);
         mma_commit(sm.bar(kBarVEmpty + rs));
       }
       ++nhead;
@@ -461,23 +451,41 @@ __device__ void mma_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, co
   }
 }
 
-// Max of this half's 64 score columns (raw units), with keys at or beyond `valid` masked
-// to -inf. Three-input maxima, four independent chains.
-__device__ __forceinline__ float half_max(uint32_t (&sv)[2][32], int col0, int valid) {
-  if (valid < col0 + 64) {
+// Score layout in the softmax threads: the two warps of a lane quarter split its 32 rows
+// (the first takes lanes 0-15, the second 16-31), and each reads whole rows with the
+// .16x256b shape. Thread t of a warp holds rows (t / 4) and (t / 4) + 8 of its 16, and in
+// every 8-column chunk the two columns 2 (t % 4) and 2 (t % 4) + 1; the four threads of a
+// row (consecutive lanes) hold all 128 columns between them. sv[p][4c + 2h + j] is row
+// (t / 4) + 8h, column 64p + 8c + 2 (t % 4) + j. Row statistics need only shuffles among
+// those four lanes, never another warp.
+
+// Row maxima (raw units) of this thread's two rows over its 32 columns each, with keys at
+// or beyond `valid` masked to -inf, then over the row's four threads.
+__device__ __forceinline__ void row_max2(uint32_t (&sv)[2][32], int g4, int valid, float (&mx)[2]) {
+  if (valid < kRows) {
 #pragma unroll
-    for (int c = 0; c < 2; ++c)
+    for (int p = 0; p < 2; ++p)
 #pragma unroll
-      for (int e = 0; e < 32; ++e)
-        if (col0 + 32 * c + e >= valid) sv[c][e] = __float_as_uint(-INFINITY);
+      for (int c = 0; c < 8; ++c)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (64 * p + 8 * c + 2 * g4 + (e & 1) >= valid) sv[p][4 * c + e] = __float_as_uint(-INFINITY);
   }
-  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-  for (int c = 0; c < 2; ++c)
+  for (int h = 0; h < 2; ++h) {
+    float m4[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-    for (int e = 0; e < 32; e += 2)
-      mx[(e >> 1) & 3] = fmax3(mx[(e >> 1) & 3], __uint_as_float(sv[c][e]), __uint_as_float(sv[c][e + 1]));
-  return fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
+    for (int p = 0; p < 2; ++p)
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        m4[c & 1] = fmax3(m4[c & 1], __uint_as_float(sv[p][4 * c + 2 * h]), __uint_as_float(sv[p][4 * c + 2 * h + 1]));
+    mx[h] = fmaxf(m4[0], m4[1]);
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
+    mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+  }
 }
 
 // Column pairs (of every 8) whose exponentials run on the FMA pipe (exp2_poly2); the
@@ -485,27 +493,36 @@ __device__ __forceinline__ float half_max(uint32_t (&sv)[2][32], int col0, int v
 constexpr uint32_t kPolyPairs = 0xA4u;   // pairs 2, 5, 7
 __host__ __device__ constexpr bool poly_pair(int j) { return (kPolyPairs >> (j & 7)) & 1u; }
 
-// P for 64 score columns (raw fp32 in sv; masked ones are -inf) as 32 packed bf16 pairs
-// in pk. Returns their sum; m is the log2-unit max in use. Scaling and sums run on
-// column pairs.
-__device__ __forceinline__ float half_probs(const uint32_t (&sv)[2][32], float m, float scale_log2,
-                                            uint32_t (&pk)[32]) {
-  const float2 sc = make_float2(scale_log2, scale_log2), nm = make_float2(-m, -m);
-  float2 acc[4];
+// P for this thread's 64 scores (raw fp32 in sv; masked ones are -inf), as 32 packed bf16
+// pairs in the .16x128b layout: pk[2 cc + h] is row (t / 4) + 8h, packed column
+// 4 cc + (t % 4), which holds keys 8 cc + 2 (t % 4) and the next. Adds this thread's share
+// of each row's sum to lsum[h]; m[h] is the log2-unit max in use for row h.
+__device__ __forceinline__ void row_probs2(const uint32_t (&sv)[2][32], const float (&m)[2], float scale_log2,
+                                           uint32_t (&pk)[32], float (&lsum)[2]) {
+  const float2 sc = make_float2(scale_log2, scale_log2);
+  float2 acc[2][2];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
+  for (int h = 0; h < 2; ++h) acc[h][0] = acc[h][1] = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int c = 0; c < 2; ++c) {
+  for (int p = 0; p < 2; ++p) {
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[c][2 * j]), __uint_as_float(sv[c][2 * j + 1])), sc, nm);
-      const float2 p = poly_pair(j) ? exp2_poly2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
-      acc[j & 3] = __fadd2_rn(acc[j & 3], p);
-      pk[16 * c + j] = pack_bf16x2(p.x, p.y);
+    for (int c = 0; c < 8; ++c) {
+      const int cc = 8 * p + c;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[p][4 * c + 2 * h]), __uint_as_float(sv[p][4 * c + 2 * h + 1])),
+                                    sc, make_float2(-m[h], -m[h]));
+        const float2 pr = poly_pair(cc) ? exp2_poly2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+        acc[h][cc & 1] = __fadd2_rn(acc[h][cc & 1], pr);
+        pk[2 * cc + h] = pack_bf16x2(pr.x, pr.y);
+      }
     }
   }
-  const float2 s = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
-  return s.x + s.y;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const float2 s2 = __fadd2_rn(acc[h][0], acc[h][1]);
+    lsum[h] += s2.x + s2.y;
+  }
 }
 
 // Scratch records are stored column-quad-major: float4 (record, quad q of 4 columns, row r)
@@ -633,13 +650,15 @@ __device__ __forceinline__ void merge_rows(const QueryArgs& a, const Seg& sg, ui
 // record's flag. Loads are issued in batches so their latencies overlap. Kept out of line
 // so its registers do not compete with the softmax loop; the launch arguments it reads stay
 // in parameter space (the kernel takes them as a grid constant), not in a per-thread copy
-// in local memory. Returns false if a wait gave up.
+// in local memory; the small structs come by value for the same reason. Returns the number
+// of group rendezvous it took (0 or 1), or -1 if a wait gave up.
 template <bool kHybrid>
-__device__ __noinline__ bool segment_epilogue(const Smem& sm, const QueryArgs& a, const Seg& sg, int first_rec,
-                                              int last_nsegs, uint32_t r, int half, int c0, int ncols, uint32_t tO,
-                                              uint32_t tX, float m, float l_row, uint32_t& gphase,
-                                              volatile int* merge_ok, const float* stage, int rs,
-                                              const CUtensorMap* tm_o, const Guard& g) {
+__device__ __noinline__ int segment_epilogue(const Smem sm, const QueryArgs& a, const Seg sg, int first_rec,
+                                             int last_nsegs, uint32_t r, int half, int c0, int ncols, uint32_t tO,
+                                             uint32_t tX, float m, float l_row, uint32_t gphase,
+                                             volatile int* merge_ok, const float* stage, int rs,
+                                             const CUtensorMap* tm_o, const Guard g) {
+  const uint32_t gphase0 = gphase;
   const int q0 = c0 / 4;   // this half's first column quad
   // First global write of this thread in the launch: a query launched as the programmatic
   // dependent of the previous one waits for it here (shared scratch, maybe the same output).
@@ -665,7 +684,7 @@ __device__ __noinline__ bool segment_epilogue(const Smem& sm, const QueryArgs& a
     tc_fence_before();
     warp_arrive(sm.bar(kBarOEmpty));   // TMEM read: the next segment may reuse O
     warp_arrive(sm.bar(kBarRec));      // record stored: the publisher may raise its flag
-    return true;
+    return 0;
   }
   // Head segment: the tile's other records (if any), then the merge. Warp 3 stages them
   // in shared memory when they fit; otherwise they are read from scratch here.
@@ -674,15 +693,15 @@ __device__ __noinline__ bool segment_epilogue(const Smem& sm, const QueryArgs& a
   const int k1 = (rs + 1) % kStages, k2 = (rs + 2) % kStages;   // idle ring stages (see staged_merge)
   if (staged) {
     // At most one staged merge per CTA and launch: the barrier completes once (phase 0).
-    if (!mbar_wait_warp(sm.bar(kBarRecLoad), 0, g)) return false;
+    if (!mbar_wait_warp(sm.bar(kBarRecLoad), 0, g)) return -1;
   } else if (nsegs > 1) {
     if (half == 0 && r == 0) {
       bool ok = true;
       for (int s = 1; s < nsegs && ok; ++s) ok = wait_flag(a.flags + slot0 + s, a.epoch, g);
       *merge_ok = ok ? 1 : 0;
     }
-    if (!group_sync(sm.bar(kBarGroup), gphase, g)) return false;
-    if (!*merge_ok) return false;
+    if (!group_sync(sm.bar(kBarGroup), gphase, g)) return -1;
+    if (!*merge_ok) return -1;
   }
   const uint32_t otile = sm.v(k2);   // staged: the output tile (two 128-byte-swizzled panels)
   if (staged)
@@ -705,7 +724,7 @@ __device__ __noinline__ bool segment_epilogue(const Smem& sm, const QueryArgs& a
   }
   tc_fence_before();
   warp_arrive(sm.bar(kBarOEmpty));
-  return true;
+  return static_cast<int>(gphase - gphase0);
 }
 
 // Warp 3. (1) Raises the flag of each partial record this CTA stores, once the softmax
@@ -771,15 +790,21 @@ template <bool kHybrid>
 __device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const QueryArgs& a, int warp,
                              const CUtensorMap* tm_o, const Guard& g) {
   const int quarter = warp & 3;
-  const int half = (warp - 4) >> 2;                         // 0: columns 0-63, 1: columns 64-127
+  // In the epilogue and the Q' packing a thread owns row r (its TMEM lane) and the column
+  // half `half`; in the tile loop the same warp owns 16 whole rows of its quarter instead
+  // (rows 16 half .. 16 half + 15; see row_max2).
+  const int half = (warp - 4) >> 2;
   const uint32_t r = quarter * 32 + (threadIdx.x & 31);     // tile row == TMEM lane
   const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+  const uint32_t lane16_off = static_cast<uint32_t>(quarter * 32 + 16 * half) << 16;
+  const int g4 = static_cast<int>(threadIdx.x & 3);
+  const uint32_t row0 = quarter * 32 + 16 * half + ((threadIdx.x & 31) >> 2);   // rows row0, row0 + 8
   const uint32_t tO = tmem + lane_off + kColO;
-  float* xch = reinterpret_cast<float*>(ctl + kCtlX);      // [2 slots][2 halves][128]
+  float* xch = reinterpret_cast<float*>(ctl + kCtlX);      // [2 slots][m | l][128]
   volatile int* merge_ok = reinterpret_cast<volatile int*>(ctl + kCtlMisc + 8);
   const uint32_t pair_bar = sm.bar(kBarPair + quarter);
   const int d = a.d;
-  const int c0 = 64 * half;                                 // first column of this thread's half
+  const int c0 = 64 * half;                                 // first output column of this thread's half
   const int ncols = max(0, min(64, d - c0));                // output columns of this half
   uint32_t nseg = 0, nhead = 0, tile = 0, gphase = 0, nx = 0, ring = 0;
   // Test hook: a wait that can only run out (the bounded-wait path, without a fault).
@@ -790,49 +815,55 @@ __device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const 
     const uint32_t t0 = tile, n = sg.ke - sg.kb;
     const int rs = ring_stage(ring + n);   // ring stage of the readout operands (staged merges)
     ring += n + ((kHybrid && sg.head) ? 1u : 0u);
-    float m = -INFINITY, l = 0.f;
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};   // rows row0, row0 + 8
     for (uint32_t i = 0; i < n; ++i) {
       const uint32_t t = t0 + i;
       const int sb = sbuf(t);
       if (!mbar_wait_warp(sm.bar(kBarSFull + sb), sphase(t), g)) return;
       tc_fence_after();
-      const uint32_t tS = tmem + lane_off + 128u * sb;
+      const uint32_t tS = tmem + lane16_off + 128u * sb;
       const int valid = a.kv_len - (sg.kb + static_cast<int>(i)) * kRows;   // >= 1
-      // This half's scores, then the row max: the two warps holding these rows (one per
-      // half) swap their half-row maxima. Each half reads and writes only its own columns.
       uint32_t sv[2][32];
-      tmem_ld32x2_wait(tS + c0, sv[0], tS + c0 + 32, sv[1]);
-      float h0, h1;
-      if (!pair_swap(pair_bar, xch, nx, half, r, half_max(sv, c0, valid), h0, h1, g)) return;
-      const float mt = fmaxf(h0, h1) * a.scale_log2;
-      float m_new = m;
-      bool rescale = false;
-      if (i == 0) {
-        m_new = mt;
-      } else if (mt > m + kRescaleThreshold) {
-        m_new = mt;
-        rescale = true;
+      tmem_ld16dp256_x8x2_wait(tS, sv[0], tS + 64u, sv[1]);
+      float mt[2];
+      row_max2(sv, g4, valid, mt);
+      float m_new[2];
+      bool rescale[2] = {false, false};
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        mt[h] *= a.scale_log2;
+        m_new[h] = m[h];
+        if (i == 0) {
+          m_new[h] = mt[h];
+        } else if (mt[h] > m[h] + kRescaleThreshold) {
+          m_new[h] = mt[h];
+          rescale[h] = true;
+        }
       }
-      if (__any_sync(0xffffffffu, rescale)) {
-        // O holds the sum up to tile t-1: wait for that P.V MMA, then scale this half-row.
+      if (__any_sync(0xffffffffu, rescale[0] || rescale[1])) {
+        // O holds the sum up to tile t-1: wait for that P.V MMA, then scale these rows.
         if (!mbar_wait_warp(sm.bar(kBarPVDone + sbuf(t - 1)), sphase(t - 1), g)) return;
         tc_fence_after();
-        const float corr = rescale ? ex2_approx(m - m_new) : 1.f;
+        const float corr0 = rescale[0] ? ex2_approx(m[0] - m_new[0]) : 1.f;
+        const float corr1 = rescale[1] ? ex2_approx(m[1] - m_new[1]) : 1.f;
+        const uint32_t tO16 = tmem + lane16_off + kColO;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t ov[16];
-          tmem_ld16_wait(tO + c0 + 16u * c, ov);
+          tmem_ld16dp256_x4_wait(tO16 + 32u * c, ov);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
-          tmem_st16(tO + c0 + 16u * c, ov);
+          for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * ((e & 2) ? corr1 : corr0));
+          tmem_st16dp256_x4(tO16 + 32u * c, ov);
         }
-        l *= corr;
+        l[0] *= corr0;
+        l[1] *= corr1;
       }
-      m = m_new;
+      m[0] = m_new[0];
+      m[1] = m_new[1];
       uint32_t pk[32];
-      l += half_probs(sv, m, a.scale_log2, pk);
-      // P overwrites the first 32 of this half's score columns.
-      tmem_st32(tS + c0, pk);
+      row_probs2(sv, m, a.scale_log2, pk, l);
+      // P (bf16 pairs) overwrites the first 64 columns of the rows' scores.
+      tmem_st16dp128_x16(tS, pk);
       tmem_wait_st();
       tc_fence_before();
       warp_arrive(sm.bar(kBarPFull + sb));
@@ -865,14 +896,37 @@ __device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const 
       warp_arrive(sm.bar(kBarQpReady));
       ++nhead;
     }
-    // Every MMA of the segment (the readout included) is done; combine the half-row sums.
+    // Every MMA of the segment (the readout included) is done. Each row's max and sum go
+    // from the tile-loop layout (16 rows a warp, four threads a row) to the epilogue's
+    // (thread = row) through shared memory; the two warps of the quarter meet on their pair
+    // barrier. Slots alternate by exchange count, so a slot is rewritten only after the
+    // other warp has passed the next exchange, and so has read it.
     if (!mbar_wait_warp(sm.bar(kBarOFull), nseg & 1, g)) return;
     tc_fence_after();
-    float l0, l1;
-    if (!pair_swap(pair_bar, xch, nx, half, r, l, l0, l1, g)) return;
-    if (!segment_epilogue<kHybrid>(sm, a, sg, sch.first_rec, sch.last_nsegs, r, half, c0, ncols, tO, tX, m, l0 + l1,
-                                   gphase, merge_ok, reinterpret_cast<const float*>(ctl - kTileRegion), rs, tm_o, g))
-      return;
+    {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        l[h] += __shfl_xor_sync(0xffffffffu, l[h], 1);
+        l[h] += __shfl_xor_sync(0xffffffffu, l[h], 2);
+      }
+      float* ml = xch + (nx & 1) * 256;
+      if (g4 == 0) {
+        ml[row0] = m[0];
+        ml[row0 + 8] = m[1];
+        ml[kRows + row0] = l[0];
+        ml[kRows + row0 + 8] = l[1];
+      }
+      warp_arrive(pair_bar);
+      const bool ok = mbar_wait_warp(pair_bar, nx & 1, g);
+      ++nx;
+      if (!ok) return;
+    }
+    const float* ml = xch + ((nx - 1) & 1) * 256;
+    const int syncs = segment_epilogue<kHybrid>(sm, a, sg, sch.first_rec, sch.last_nsegs, r, half, c0, ncols, tO, tX,
+                                                ml[r], ml[kRows + r], gphase, merge_ok,
+                                                reinterpret_cast<const float*>(ctl - kTileRegion), rs, tm_o, g);
+    if (syncs < 0) return;
+    gphase += static_cast<uint32_t>(syncs);
     ++nseg;
   }
 }
