@@ -17,10 +17,11 @@
 // Reduction through L2. Every CTA writes its partial U (fp32, column-quad-major so that a
 // warp's stores are contiguous) and its sum of alpha to a scratch slot of its own, then the
 // cluster meets once at a barrier (release/acquire: the partials are visible after it). CTA
-// g then owns a block of columns of S_N: for each of its elements it sums the G partials in
-// a fixed order (the result does not depend on timing), adds abar S_{N-1} and writes S_N in
-// fp32 and bf16. The scratch is private to the launch's own clusters and is fully written
-// before it is read, so it never needs clearing.
+// g then owns a block of columns of S_N: it bulk-copies that block of every group's partial
+// into shared memory, sums the G partials of each element in a fixed order (the result does
+// not depend on timing), adds abar S_{N-1} and writes S_N in fp32 and bf16. The scratch is
+// private to the launch's own clusters and is fully written before it is read, so it never
+// needs clearing.
 //
 // Roles (192 threads): warp 0 TMA, warp 1 TMEM owner and MMA issuer (warp-wide loop, one
 // elected lane issues), warps 2-5 row warps (thread = token row for K' and R, = state row k
@@ -56,9 +57,10 @@ enum : int {
   kBarR = 13,         // R bf16 over the V tile (one arrival per row warp)
   kBarU = 14,         // U complete
   kBarFinal = 15,     // every MMA done (drain before TMEM is freed)
-  kNumBars = 16
+  kBarOwn = 16,       // the owned columns of every group's partial landed in shared memory
+  kNumBars = 17
 };
-constexpr uint32_t kCtlMisc = 128;           // tmem slot, abort flag, rows-failed flag, warp alpha sums
+constexpr uint32_t kCtlMisc = 192;           // tmem slot, abort flag, rows-failed flag, warp alpha sums
 constexpr uint32_t kSmemBytes = kCtlOff + kCtlMisc + 64;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;   // room to align the base to 1 KiB
 static_assert(kNumBars * 8 <= kCtlMisc, "barriers must fit their slot");
@@ -391,19 +393,23 @@ __global__ void __launch_bounds__(kThreadsC, 1)
       rd.part_alpha[bh * G + rank] = (warp_sums[0] + warp_sums[1]) + (warp_sums[2] + warp_sums[3]);
     }
   }
-  // This CTA's columns of S_{N-1} go to L2 ahead of the barrier (no other CTA writes them):
-  // for each row, the 128-byte lines that hold the first and last of its columns.
+  // CTA `rank` owns column quads [q0, q1) of S_N, every row. Its columns of S_{N-1} go to L2
+  // ahead of the barrier (no other CTA writes them): for each row, the 128-byte lines that
+  // hold the first and last of its columns.
   const int quads = d / 4;
   const int qpo = (quads + G - 1) / G;   // column quads owned per CTA
   const int q0 = min(quads, rank * qpo), q1 = min(quads, q0 + qpo);
+  const int nq_own = q1 - q0;
   const size_t dd = static_cast<size_t>(d) * d;
-  if (ok_here && q1 > q0) {
+  if (ok_here && nq_own > 0) {
     for (int i = threadIdx.x; i < 2 * d; i += kThreadsC) {
       const int k = i >> 1, col = (i & 1) ? 4 * q1 - 1 : 4 * q0;
       prefetch_l2(rd.S_old + bh * dd + static_cast<size_t>(k) * d + col);
     }
   }
-  __threadfence();
+  // The partials were written through the generic proxy and are read below by bulk copies
+  // (the async proxy); the cluster barrier's release/acquire makes them visible.
+  fence_proxy_async_global();
   tc_fence_before();
   cluster_sync();   // every CTA's partial is written and visible
   if (warp == 1) {   // every TMEM read of this CTA happened before the barrier
@@ -414,38 +420,74 @@ __global__ void __launch_bounds__(kThreadsC, 1)
   }
   if (!ok_here) return;
 
-  // Owner phase: S_N over columns [4 q0, 4 q1), every row, from the G partials summed in a
-  // fixed order. Item (row k, quad q), rows fastest, so a warp's partial loads are contiguous.
+  // Owner phase. The G partial blocks of the owned columns (contiguous in the column-quad-
+  // major slots: nq_own x 128 float4 each, one bulk copy per group; many small copies would
+  // cost far more than these few large ones) come into shared memory over the chunk tiles
+  // that are idle now, while each thread loads the S_{N-1} values and the alpha sums it
+  // needs; then every item (row k, quad q; rows fastest) sums the G partials in a fixed
+  // order, adds abar S_{N-1} and writes S_N in fp32 and bf16.
+  const uint32_t own_bytes = static_cast<uint32_t>(nq_own) * kRows * 16;
+  const uint32_t recv = sm.k(0);
+  if (nq_own > 0 && warp == 0) {
+    if (lane == 0) {
+      fence_proxy_async_global();
+      mbar_expect_tx(sm.bar(kBarOwn), own_bytes * G);
+    }
+    __syncwarp();
+    for (int j = lane; j < G; j += 32)
+      bulk_load(recv + j * own_bytes, part_slot(rd.part_u, bh, G, j) + static_cast<size_t>(q0) * kRows, own_bytes,
+                sm.bar(kBarOwn));
+  }
+  float al[kMaxCluster];
+#pragma unroll
+  for (int j = 0; j < kMaxCluster; ++j) al[j] = j < G ? __ldcg(rd.part_alpha + bh * G + j) : 0.f;
   float asum = 0.f;
-  for (int j = 0; j < G; ++j) asum += __ldcg(rd.part_alpha + bh * G + j);
+#pragma unroll
+  for (int j = 0; j < kMaxCluster; ++j) asum += al[j];
   const float abar = asum * rd.inv_T;
   const float* S_old = rd.S_old + bh * dd;
   float* S_new = rd.S_new + bh * dd;
   uint16_t* S_new_bf16 = rd.S_new_bf16 + bh * dd;
-  const float4* part0 = part_slot(rd.part_u, bh, G, 0);
-  const int items = d * (q1 - q0);
+  const float4* own = reinterpret_cast<const float4*>(gbase + (recv - base));
+  const int items = d * nq_own;
+  constexpr int kBatch = 4;   // items a thread loads S_{N-1} for before it sums them
+  bool landed = false;
 #pragma unroll 1
-  for (int it = threadIdx.x; it < items; it += kThreadsC) {
-    const int k = it % d, q = q0 + it / d;
-    const float4 so = *reinterpret_cast<const float4*>(S_old + static_cast<size_t>(k) * d + 4 * q);
-    float4 u[kMaxCluster];
+  for (int it0 = threadIdx.x; it0 < items; it0 += kBatch * kThreadsC) {
+    float4 so[kBatch];
 #pragma unroll
-    for (int j = 0; j < kMaxCluster; ++j)
-      if (j < G) u[j] = __ldcg(part0 + (static_cast<size_t>(j) * 32 + q) * kRows + k);
-    float4 acc = make_float4(abar * so.x, abar * so.y, abar * so.z, abar * so.w);
-#pragma unroll
-    for (int j = 0; j < kMaxCluster; ++j) {
-      if (j < G) {
-        acc.x += u[j].x;
-        acc.y += u[j].y;
-        acc.z += u[j].z;
-        acc.w += u[j].w;
-      }
+    for (int e = 0; e < kBatch; ++e) {
+      const int it = it0 + e * kThreadsC;
+      if (it < items)
+        so[e] = *reinterpret_cast<const float4*>(S_old + static_cast<size_t>(it % d) * d + 4 * (q0 + it / d));
     }
-    *reinterpret_cast<float4*>(S_new + static_cast<size_t>(k) * d + 4 * q) = acc;
-    *reinterpret_cast<uint2*>(S_new_bf16 + static_cast<size_t>(k) * d + 4 * q) =
-        make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+    if (!landed) {
+      if (!mbar_wait(sm.bar(kBarOwn), 0, g)) break;
+      landed = true;
+    }
+#pragma unroll
+    for (int e = 0; e < kBatch; ++e) {
+      const int it = it0 + e * kThreadsC;
+      if (it >= items) break;
+      const int k = it % d, qo = it / d;
+      float4 acc = make_float4(abar * so[e].x, abar * so[e].y, abar * so[e].z, abar * so[e].w);
+#pragma unroll
+      for (int j = 0; j < kMaxCluster; ++j) {
+        if (j < G) {
+          const float4 u = own[(j * nq_own + qo) * kRows + k];
+          acc.x += u.x;
+          acc.y += u.y;
+          acc.z += u.z;
+          acc.w += u.w;
+        }
+      }
+      const size_t o = static_cast<size_t>(k) * d + 4 * (q0 + qo);
+      *reinterpret_cast<float4*>(S_new + o) = acc;
+      *reinterpret_cast<uint2*>(S_new_bf16 + o) = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+    }
   }
+  // The copies must land before the CTA may exit (matters only after a time-out).
+  if (nq_own > 0 && warp == 0) mbar_wait_drain(sm.bar(kBarOwn), 0);
 }
 
 __global__ void arl2_state_import_kernel(const float* __restrict__ src, float* __restrict__ S,
