@@ -32,6 +32,9 @@ Readings of what the pages leave open (plain readings, fixed for this library):
   R5 The softmax scale is 1/sqrt(d) and no mask is applied inside the frame.
   R6 The two branches are summed: O = O_intra + O_inter.
   R7 Inputs arrive already rounded to bfloat16 and are widened exactly to fp64.
+  R8 The per-token gates, where they are produced from the hidden state rather than given,
+     are a linear projection of the token's hidden state per head plus a bias, through a
+     sigmoid, which keeps both in (0, 1) as a forget gate and a rate must be.
 
 Array layout: q, k, v are [B, T, H, d] (token-major); feature-map weights are
 [H, d_in, d_out]; the state is [B, H, d_k, d_v]; alpha and beta are [B, H, T].
@@ -161,6 +164,36 @@ class Layer:
         self.S = frame_commit(k, v, alpha, beta, self.Wk, self.Wv, self.S)
         self.frame += 1
         return self.S
+
+
+def gates_from_hidden(x, Wa, ba, Wb, bb):
+    """Per-token forget gate and rate from the token's hidden state (§2.1: alpha and beta are
+    per-token learned projections; reading R8 fixes their form):
+
+        alpha[b, h, t] = sigmoid(x[b, t, :] . Wa[h, :] + ba[h])
+        beta[b, h, t]  = sigmoid(x[b, t, :] . Wb[h, :] + bb[h])
+
+    x is [B, T, D] (D: the layer's model width); Wa, Wb are [H, D]; ba, bb are [H]. Returns
+    (alpha, beta), each [B, H, T].
+    """
+    x, Wa, Wb, ba, bb = _f64(x), _f64(Wa), _f64(Wb), _f64(ba), _f64(bb)
+    B, T, _ = x.shape
+    H = Wa.shape[0]
+    alpha = np.empty((B, H, T))
+    beta = np.empty((B, H, T))
+    for b in range(B):
+        for h in range(H):
+            za = x[b] @ Wa[h] + ba[h]
+            zb = x[b] @ Wb[h] + bb[h]
+            alpha[b, h] = 1.0 / (1.0 + np.exp(-za))
+            beta[b, h] = 1.0 / (1.0 + np.exp(-zb))
+    return alpha, beta
+
+
+def frame_commit_gated(x, k, v, Wa, ba, Wb, bb, Wk, Wv, S) -> np.ndarray:
+    """The clean-pass commit with its gates produced from the hidden state x (gates_from_hidden)."""
+    alpha, beta = gates_from_hidden(x, Wa, ba, Wb, bb)
+    return frame_commit(k, v, alpha, beta, Wk, Wv, S)
 
 
 def kv_cache_attention(q, k_cache, v_cache, length: int, rows=None) -> np.ndarray:

@@ -19,6 +19,7 @@ import numpy as np
 
 TENSOR_Q, TENSOR_K, TENSOR_V, TENSOR_ALPHA, TENSOR_BETA = 0, 1, 2, 3, 4
 TENSOR_WQ, TENSOR_WK, TENSOR_WV, TENSOR_STATE = 5, 6, 7, 8
+TENSOR_X, TENSOR_WA, TENSOR_WB = 9, 10, 11
 CLEAN_PASS = 4
 _WEIGHT_FRAME = 0xFFFF  # frame slot used for the per-layer phi weights
 
@@ -69,6 +70,25 @@ def feature_maps(seed: int, config: int, H: int, d: int):
         w = g.standard_normal((H, d, d), dtype=np.float32) / np.float32(np.sqrt(d))
         out.append(bf16_bits(w.astype(np.float32)))
     return tuple(out)
+
+
+def hidden(seed: int, config: int, frame: int, B: int, T: int, D: int) -> np.ndarray:
+    """The clean pass's hidden states x ~ N(0, 1), bfloat16 bits [B, T, D] (D: model width)."""
+    g = rng(seed, config, frame, CLEAN_PASS, TENSOR_X)
+    return bf16_bits(g.standard_normal((B, T, D), dtype=np.float32))
+
+
+def gate_weights(seed: int, config: int, H: int, D: int):
+    """Gate projections for gates produced from x: Wa, Wb as bfloat16 bits [H, D] and biases
+    ba, bb as float32 [H]. Wa ~ N(0, std 0.5/sqrt(D)) with ba = 2 and Wb ~ N(0, std 1/sqrt(D))
+    with bb = 0, so that for x ~ N(0, 1) alpha = sigmoid(N(2, 0.5)) and beta = sigmoid(N(0, 1)),
+    the same distributions as the gates drawn directly."""
+    ga = rng(seed, config, _WEIGHT_FRAME, 0, TENSOR_WA)
+    gb = rng(seed, config, _WEIGHT_FRAME, 0, TENSOR_WB)
+    wa = ga.standard_normal((H, D), dtype=np.float32) * np.float32(0.5 / np.sqrt(D))
+    wb = gb.standard_normal((H, D), dtype=np.float32) / np.float32(np.sqrt(D))
+    return (bf16_bits(wa.astype(np.float32)), np.full(H, 2.0, np.float32),
+            bf16_bits(wb.astype(np.float32)), np.zeros(H, np.float32))
 
 
 def state(seed: int, config: int, B: int, H: int, d: int, scale: float = 1.0) -> np.ndarray:

@@ -306,3 +306,80 @@ def test_planted_mistakes_are_caught(mistake):
     g0 = _golden("commit_normalised_keys.json")
     caught |= not np.allclose(_commit_from_fixture(g0, bad), np.array(g0["S_next"]), atol=1e-12)
     assert caught, f"planted mistake {mistake!r} passed both commit fixtures"
+
+
+# ---------------------------------------------------------------- gate producer
+def _gates_fixture():
+    g = _golden("gates_from_hidden.json")
+    x = np.array(g["x"], float)[None]
+    return g, x, np.array(g["Wa"], float), np.array(g["ba"], float), np.array(g["Wb"], float), np.array(g["bb"], float)
+
+
+def test_gates_golden():
+    g, x, Wa, ba, Wb, bb = _gates_fixture()
+    a, b = orc.gates_from_hidden(x, Wa, ba, Wb, bb)
+    np.testing.assert_allclose(a[0], np.array(g["alpha"]), rtol=0, atol=1e-15)
+    np.testing.assert_allclose(b[0], np.array(g["beta"]), rtol=0, atol=1e-15)
+
+
+def test_gates_of_a_zero_hidden_state_are_the_bias_sigmoid():
+    rng = np.random.default_rng(3)
+    H, D = 3, 8
+    Wa, Wb = rng.standard_normal((H, D)), rng.standard_normal((H, D))
+    ba, bb = rng.standard_normal(H), rng.standard_normal(H)
+    a, b = orc.gates_from_hidden(np.zeros((2, 5, D)), Wa, ba, Wb, bb)
+    for h in range(H):
+        assert np.all(a[:, h] == 1.0 / (1.0 + np.exp(-ba[h])))
+        assert np.all(b[:, h] == 1.0 / (1.0 + np.exp(-bb[h])))
+
+
+def test_gate_logits_are_affine_in_the_hidden_state():
+    # logit(alpha(x1 + x2)) = logit(alpha(x1)) + logit(alpha(x2)) - ba, per head and token.
+    rng = np.random.default_rng(4)
+    B, T, D, H = 2, 6, 16, 3
+    x1, x2 = rng.standard_normal((B, T, D)) * 0.3, rng.standard_normal((B, T, D)) * 0.3
+    Wa, Wb = rng.standard_normal((H, D)) * 0.5, rng.standard_normal((H, D)) * 0.5
+    ba, bb = rng.standard_normal(H), rng.standard_normal(H)
+    logit = lambda p: np.log(p) - np.log1p(-p)
+    a1, b1 = orc.gates_from_hidden(x1, Wa, ba, Wb, bb)
+    a2, b2 = orc.gates_from_hidden(x2, Wa, ba, Wb, bb)
+    a12, b12 = orc.gates_from_hidden(x1 + x2, Wa, ba, Wb, bb)
+    np.testing.assert_allclose(logit(a12), logit(a1) + logit(a2) - ba[None, :, None], atol=1e-12)
+    np.testing.assert_allclose(logit(b12), logit(b1) + logit(b2) - bb[None, :, None], atol=1e-12)
+
+
+def test_gated_commit_is_the_commit_with_produced_gates():
+    rng = np.random.default_rng(5)
+    B, T, H, d = 1, 9, 2, 4
+    D = H * d
+    x = rng.standard_normal((B, T, D))
+    k, v = rng.standard_normal((B, T, H, d)), rng.standard_normal((B, T, H, d))
+    Wa, Wb = rng.standard_normal((H, D)), rng.standard_normal((H, D))
+    ba, bb = rng.standard_normal(H), rng.standard_normal(H)
+    Wk, Wv = rng.standard_normal((H, d, d)), rng.standard_normal((H, d, d))
+    S = rng.standard_normal((B, H, d, d))
+    # The same commit with hand-computed gates (a loop over tokens, not the oracle's matmul).
+    a = np.empty((B, H, T))
+    b = np.empty((B, H, T))
+    for h in range(H):
+        for t in range(T):
+            a[0, h, t] = 1.0 / (1.0 + np.exp(-(sum(x[0, t, j] * Wa[h, j] for j in range(D)) + ba[h])))
+            b[0, h, t] = 1.0 / (1.0 + np.exp(-(sum(x[0, t, j] * Wb[h, j] for j in range(D)) + bb[h])))
+    np.testing.assert_allclose(orc.frame_commit_gated(x, k, v, Wa, ba, Wb, bb, Wk, Wv, S),
+                               orc.frame_commit(k, v, a, b, Wk, Wv, S), atol=1e-12)
+
+
+def test_planted_gate_mistakes_are_caught():
+    g, x, Wa, ba, Wb, bb = _gates_fixture()
+    sig = lambda z: 1.0 / (1.0 + np.exp(-z))
+    mistakes = {
+        "no bias": lambda: (sig(x[0] @ Wa.T).T, sig(x[0] @ Wb.T).T),
+        "gates swapped": lambda: (sig(x[0] @ Wb.T + bb).T, sig(x[0] @ Wa.T + ba).T),
+        "weights transposed": lambda: (sig(x[0] @ Wa + ba).T, sig(x[0] @ Wb + bb).T),
+        "tanh for sigmoid": lambda: (np.tanh(x[0] @ Wa.T + ba).T, np.tanh(x[0] @ Wb.T + bb).T),
+        "minus sign": lambda: (sig(-(x[0] @ Wa.T) + ba).T, sig(-(x[0] @ Wb.T) + bb).T),
+    }
+    for name, wrong in mistakes.items():
+        a, b = wrong()
+        ok = np.allclose(a, g["alpha"], atol=1e-12) and np.allclose(b, g["beta"], atol=1e-12)
+        assert not ok, f"the gate fixture does not catch: {name}"
