@@ -20,7 +20,9 @@ technical summary of arXiv 2605.16579 on gist.science (zh/pt/fr pages):
       - clean-pass update: denoising passes only read S; S is written
         once per frame, after the clean pass.
 
-Readings of what the pages leave open (plain readings, fixed for this library):
+Readings of what the pages leave open (plain readings, fixed for this library; the numbers
+follow the library's one list of readings, and those missing here fix the schedule, the
+input distributions and the tolerances, not this module's arithmetic):
   R1 The update as printed has no transpose and is ill-formed for K' (T x d_k)
      and S (d_k x d_v); it is read as K'^T (V' - K' S).
   R2 alpha and beta are per token; S is per frame. The frame's forget factor is
@@ -31,10 +33,17 @@ Readings of what the pages leave open (plain readings, fixed for this library):
      Only K' is L2-normalised per token, as k / max(||k||_2, 1e-12).
   R5 The softmax scale is 1/sqrt(d) and no mask is applied inside the frame.
   R6 The two branches are summed: O = O_intra + O_inter.
-  R7 Inputs arrive already rounded to bfloat16 and are widened exactly to fp64.
-  R8 The per-token gates, where they are produced from the hidden state rather than given,
-     are a linear projection of the token's hidden state per head plus a bias, through a
-     sigmoid, which keeps both in (0, 1) as a forget gate and a rate must be.
+  R9 Inputs arrive already rounded to bfloat16 and are widened exactly to fp64.
+  R13 The per-token gates, where they are produced from the hidden state rather than given,
+      are a linear projection of the token's hidden state per head plus a bias, through a
+      sigmoid, which keeps both in (0, 1) as a forget gate and a rate must be.
+  R15 Token-level access (the ablation of §4 that the pages contrast with frame-level
+      access, without giving its form): inside a pass the state advances token by token
+      in the frame's token order, with the update rule of §2.1 applied to one token at a
+      time (its own alpha_t as the forget gate and beta_t as the rate, the residual against
+      the undecayed state as in R3), starting from S_{N-1}. Token t reads the state left by
+      tokens 0..t-1, the token-level counterpart of every token reading S_{N-1}. The clean
+      pass's final state is S_N.
 
 Array layout: q, k, v are [B, T, H, d] (token-major); feature-map weights are
 [H, d_in, d_out]; the state is [B, H, d_k, d_v]; alpha and beta are [B, H, T].
@@ -168,7 +177,7 @@ class Layer:
 
 def gates_from_hidden(x, Wa, ba, Wb, bb):
     """Per-token forget gate and rate from the token's hidden state (§2.1: alpha and beta are
-    per-token learned projections; reading R8 fixes their form):
+    per-token learned projections; reading R13 fixes their form):
 
         alpha[b, h, t] = sigmoid(x[b, t, :] . Wa[h, :] + ba[h])
         beta[b, h, t]  = sigmoid(x[b, t, :] . Wb[h, :] + bb[h])
@@ -194,6 +203,48 @@ def frame_commit_gated(x, k, v, Wa, ba, Wb, bb, Wk, Wv, S) -> np.ndarray:
     """The clean-pass commit with its gates produced from the hidden state x (gates_from_hidden)."""
     alpha, beta = gates_from_hidden(x, Wa, ba, Wb, bb)
     return frame_commit(k, v, alpha, beta, Wk, Wv, S)
+
+
+def token_level_scan(q, k, v, alpha, beta, Wq, Wk, Wv, S):
+    """Token-level access (R15): per (batch, head), starting from S_{N-1}, for t = 0..T-1
+
+        o_inter[t] = q'_t S                                    (the state before token t)
+        S          = alpha_t S + beta_t k'_t^T (v'_t - k'_t S)   (one token of the §2.1 rule)
+
+    with q' = phi_q(q), k' = rownorm(phi_k(k)), v' = phi_v(v) as in the frame-level layer.
+    Returns (O_inter [B, T, H, d_v], the final state [B, H, d_k, d_v]). q may be None (the
+    commit needs only the final state)."""
+    kp = l2_normalize_rows(feature_map(k, Wk))
+    vp = feature_map(v, Wv)
+    qp = None if q is None else feature_map(q, Wq)
+    alpha, beta, S = _f64(alpha), _f64(beta), _f64(S)
+    B, T, H, _ = kp.shape
+    o_inter = None if q is None else np.empty((B, T, H, S.shape[-1]))
+    S_end = np.empty_like(S)
+    for b in range(B):
+        for h in range(H):
+            St = S[b, h].copy()
+            for t in range(T):
+                if qp is not None:
+                    o_inter[b, t, h] = qp[b, t, h] @ St
+                k_t = kp[b, t, h]
+                St = alpha[b, h, t] * St + beta[b, h, t] * np.outer(k_t, vp[b, t, h] - k_t @ St)
+            S_end[b, h] = St
+    return o_inter, S_end
+
+
+def frame_query_token(q, k, v, alpha, beta, Wq, Wk, Wv, S):
+    """One query pass with token-level access (R15): O = O_intra + O_inter, the intra branch as
+    in the frame-level layer and the inter branch read token by token. The pass's own k, v and
+    gates advance the state inside the pass; the layer's state S_{N-1} is not changed."""
+    o_inter, _ = token_level_scan(q, k, v, alpha, beta, Wq, Wk, Wv, S)
+    return intra_attention(q, k, v) + o_inter
+
+
+def frame_commit_token(k, v, alpha, beta, Wk, Wv, S) -> np.ndarray:
+    """The clean-pass commit with token-level access (R15): S_N is the state after the clean
+    pass's last token."""
+    return token_level_scan(None, k, v, alpha, beta, None, Wk, Wv, S)[1]
 
 
 def kv_cache_attention(q, k_cache, v_cache, length: int, rows=None) -> np.ndarray:

@@ -383,3 +383,127 @@ def test_planted_gate_mistakes_are_caught():
         a, b = wrong()
         ok = np.allclose(a, g["alpha"], atol=1e-12) and np.allclose(b, g["beta"], atol=1e-12)
         assert not ok, f"the gate fixture does not catch: {name}"
+
+
+# ---- Token-level access (reading R15) ------------------------------------------------------
+
+def _token_fixture():
+    g = _golden("token_scan_two_tokens.json")
+    q, k, v = (np.array(g[n], float)[None, :, None, :] for n in ("q", "k", "v"))
+    a = np.array(g["alpha"], float)[None, None, :]
+    b = np.array(g["beta"], float)[None, None, :]
+    S0 = np.array(g["S0"], float)[None, None]
+    I = np.eye(2)[None]
+    return g, q, k, v, a, b, I, S0
+
+
+def test_token_scan_golden():
+    g, q, k, v, a, b, I, S0 = _token_fixture()
+    o, S = orc.token_level_scan(q, k, v, a, b, I, I, I, S0)
+    np.testing.assert_allclose(o[0, :, 0], np.array(g["o_inter"]), rtol=0, atol=1e-14)
+    np.testing.assert_allclose(S[0, 0], np.array(g["S_end"]), rtol=0, atol=1e-14)
+    np.testing.assert_allclose(orc.frame_commit_token(k, v, a, b, I, I, S0)[0, 0], np.array(g["S_end"]), atol=1e-14)
+
+
+def test_token_scan_of_one_token_is_the_frame_level_layer():
+    # T = 1: the frame's mean gate is the token's gate and beta/T = beta, so token-level and
+    # frame-level access agree, for the readout and the commit.
+    rng = np.random.default_rng(21)
+    B, H, d = 2, 3, 4
+    q, k, v = (rng.standard_normal((B, 1, H, d)) for _ in range(3))
+    Wq, Wk, Wv = (rng.standard_normal((H, d, d)) for _ in range(3))
+    S = rng.standard_normal((B, H, d, d))
+    a, b = rng.uniform(0.1, 0.9, (B, H, 1)), rng.uniform(0.1, 0.9, (B, H, 1))
+    o, S_end = orc.token_level_scan(q, k, v, a, b, Wq, Wk, Wv, S)
+    np.testing.assert_allclose(o, orc.readout(q, Wq, S), atol=1e-12)
+    np.testing.assert_allclose(S_end, orc.frame_commit(k, v, a, b, Wk, Wv, S), atol=1e-12)
+
+
+def test_token_scan_is_a_sequence_of_one_token_frames():
+    # Token-level access over T tokens = T frame-level commits of one-token frames, each token
+    # reading the state its predecessors left.
+    rng = np.random.default_rng(22)
+    B, T, H, d = 1, 7, 2, 4
+    q, k, v = (rng.standard_normal((B, T, H, d)) for _ in range(3))
+    Wq, Wk, Wv = (rng.standard_normal((H, d, d)) / 2 for _ in range(3))
+    S = rng.standard_normal((B, H, d, d))
+    a, b = rng.uniform(0.5, 1.0, (B, H, T)), rng.uniform(0.0, 1.0, (B, H, T))
+    o, S_end = orc.token_level_scan(q, k, v, a, b, Wq, Wk, Wv, S)
+    St = S
+    for t in range(T):
+        np.testing.assert_allclose(o[:, t:t + 1], orc.readout(q[:, t:t + 1], Wq, St), atol=1e-12)
+        St = orc.frame_commit(k[:, t:t + 1], v[:, t:t + 1], a[:, :, t:t + 1], b[:, :, t:t + 1], Wk, Wv, St)
+    np.testing.assert_allclose(S_end, St, atol=1e-12)
+
+
+def test_token_scan_closed_forms():
+    rng = np.random.default_rng(23)
+    B, T, H, d = 1, 6, 2, 6
+    q, k, v = (rng.standard_normal((B, T, H, d)) for _ in range(3))
+    I = np.stack([np.eye(d)] * H)
+    S = rng.standard_normal((B, H, d, d))
+    # alpha = 1, beta = 0: nothing moves; every token reads S.
+    o, S_end = orc.token_level_scan(q, k, v, np.ones((B, H, T)), np.zeros((B, H, T)), I, I, I, S)
+    np.testing.assert_array_equal(S_end, S)
+    np.testing.assert_allclose(o, orc.readout(q, I, S), atol=1e-12)
+    # beta = 0: pure decay, token t reads (prod of the gates before it) S.
+    a = rng.uniform(0.3, 0.99, (B, H, T))
+    o, S_end = orc.token_level_scan(q, k, v, a, np.zeros((B, H, T)), I, I, I, S)
+    for h in range(H):
+        np.testing.assert_allclose(S_end[0, h], np.prod(a[0, h]) * S[0, h], atol=1e-12)
+        for t in range(T):
+            np.testing.assert_allclose(o[0, t, h], np.prod(a[0, h, :t]) * (q[0, t, h] @ S[0, h]), atol=1e-12)
+    # Orthonormal keys and alpha = 1: the tokens' updates do not interact, so
+    # S_end = S + sum_t beta_t k_t^T (v_t - k_t S).
+    Qm = np.linalg.qr(rng.standard_normal((d, d)))[0]
+    k_on = np.broadcast_to(Qm[:T][None, :, None, :], (B, T, H, d)).copy()
+    b = rng.uniform(0.1, 1.0, (B, H, T))
+    _, S_end = orc.token_level_scan(None, k_on, v, np.ones((B, H, T)), b, None, I, I, S)
+    for h in range(H):
+        want = S[0, h] + sum(b[0, h, t] * np.outer(k_on[0, t, h], v[0, t, h] - k_on[0, t, h] @ S[0, h])
+                             for t in range(T))
+        np.testing.assert_allclose(S_end[0, h], want, atol=1e-12)
+
+
+def test_token_query_adds_the_scan_readout_to_intra_attention():
+    rng = np.random.default_rng(24)
+    B, T, H, d = 1, 5, 2, 4
+    q, k, v = (rng.standard_normal((B, T, H, d)) for _ in range(3))
+    W = [rng.standard_normal((H, d, d)) for _ in range(3)]
+    S = rng.standard_normal((B, H, d, d))
+    a, b = rng.uniform(0.5, 1.0, (B, H, T)), rng.uniform(0.0, 1.0, (B, H, T))
+    o_inter, _ = orc.token_level_scan(q, k, v, a, b, *W, S)
+    np.testing.assert_allclose(orc.frame_query_token(q, k, v, a, b, *W, S),
+                               orc.intra_attention(q, k, v) + o_inter, atol=1e-12)
+
+
+def test_planted_token_scan_mistakes_are_caught():
+    # Test-local copies of the scan, each with one plausible slip; the golden fixture must
+    # reject every one of them.
+    g, q, k, v, a, b, I, S0 = _token_fixture()
+    qv, kv, vv = q[0, :, 0], k[0, :, 0], v[0, :, 0]
+    al, be = a[0, 0], b[0, 0]
+
+    def scan(after=False, beta_over_T=False, decayed=False, reverse=False, no_norm=False, mean_alpha=False):
+        S = S0[0, 0].copy()
+        T = len(al)
+        order = range(T - 1, -1, -1) if reverse else range(T)
+        o = np.zeros((T, 2))
+        for t in order:
+            kt = kv[t] if no_norm else kv[t] / np.linalg.norm(kv[t])
+            at = al.mean() if mean_alpha else al[t]
+            bt = be[t] / T if beta_over_T else be[t]
+            res = vv[t] - kt @ (at * S if decayed else S)
+            S_next = at * S + bt * np.outer(kt, res)
+            o[t] = qv[t] @ (S_next if after else S)
+            S = S_next
+        return o, S
+
+    ok_o, ok_S = scan()
+    np.testing.assert_allclose(ok_o, np.array(g["o_inter"]), atol=1e-14)
+    np.testing.assert_allclose(ok_S, np.array(g["S_end"]), atol=1e-14)
+    for slip in ("after", "beta_over_T", "decayed", "reverse", "no_norm", "mean_alpha"):
+        o, S = scan(**{slip: True})
+        caught = (not np.allclose(o, np.array(g["o_inter"]), atol=1e-9) or
+                  not np.allclose(S, np.array(g["S_end"]), atol=1e-9))
+        assert caught, slip
