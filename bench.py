@@ -31,6 +31,13 @@ The bench prints one JSON line (rank 0):
     and device memory (cudaMemGetInfo) before and after.
   - sweep: frames/s and the two kernels' roofline fractions at B in {1, 4} and
     T in {390, 1560, 3600} (device-generated seeded inputs, larger than L2 per cycle).
+  - hybrid_stack: timing-only 30-layer stacks with 0%, 50% and 75% of the layers ARL2 and
+    the rest softmax over a growing KV cache: time per frame and N-dependent memory at
+    frame N = 1, 21, 60, 120.
+  - token_level: the token-level access ablation (4 queries + 1 commit per frame, each call
+    alone), its scan against the SMs' fp32 rate.
+  - clean_pass: frames with the fused clean pass (4 queries + clean pass) against frames with
+    its two calls (4 queries + query + commit), and the clean pass alone against the pair.
   - cpu_baseline: the fp64 oracle on this host's cores over a bounded sample.
   - clocks: SM clocks and throttle reasons sampled with NVML during the timed region.
 With --gpus N under torchrun, each rank runs its own independent layer (the layer has no
@@ -92,12 +99,15 @@ FRAME_BYTES = QUERIES * QUERY_BYTES + COMMIT_BYTES
 DATASHEET_BF16_TFLOPS = 2250.0
 
 
+KERNEL_HEADERS = {"arl2_query.cu": ("arl2_query_body.cuh",)}
+
+
 def kernel_sources_sha256(kernel_file: str) -> str:
     """SHA-256 over a kernel's source file and the headers it includes."""
     import hashlib
     csrc = os.path.join(ROOT, "softmax_attention_ar_b200", "csrc")
     digest = hashlib.sha256()
-    for f in (kernel_file, "arl2_device.cuh", "arl2_kernels.h"):
+    for f in (kernel_file, *KERNEL_HEADERS.get(kernel_file, ()), "arl2_device.cuh", "arl2_kernels.h"):
         with open(os.path.join(csrc, f), "rb") as fh:
             digest.update(fh.read())
     return digest.hexdigest()
@@ -287,6 +297,84 @@ def kv_cache_baseline(frames, dev, layer_ms_per_frame, layer_bytes):
             "arl2_ms_per_frame": layer_ms_per_frame, "arl2_state_bytes": layer_bytes}
 
 
+def hybrid_stack(frames, dev, stream, layers=30, Ns=(1, 21, 60, 120), shares=(0.0, 0.5, 0.75)):
+    """Timing-only stack of `layers` attention layers at the 480p shapes: a share of them ARL2
+    layers, the rest softmax attention over a growing KV cache (the layers ARL2 replaces). For
+    frame N: the time of one frame of the whole stack (per layer its 4 denoising queries and
+    the clean pass's commit, or cache append), CUDA events over two consecutive frames, and
+    the device memory that depends on N (the KV caches; each ARL2 layer's state is constant).
+    Synthetic weights and inputs: this reproduces the shape of the memory and time curves with
+    video length, not any model's quality."""
+    import torch
+
+    from softmax_attention_ar_b200.arl2 import ARL2Layer, KVCacheBaseline
+    Nmax = max(Ns) + 2
+    frame_kv = B * T * H * D * 2 * 2                 # one frame's K and V, bf16
+    n_soft_max = max(layers - int(round(s * layers)) for s in shares)
+    n_arl2_max = max(int(round(s * layers)) for s in shares)
+    caches = [KVCacheBaseline(H, T, D, B, max_frames=Nmax) for _ in range(n_soft_max)]
+    arl2s = [ARL2Layer(H, T, D, B) for _ in range(n_arl2_max)]
+    wq = torch.randn((H, D, D), device=dev, dtype=torch.float32).div_(D ** 0.5).to(torch.bfloat16)
+    for lay in arl2s:
+        lay.set_feature_maps(wq, wq, wq)
+        lay.set_launch_overlap(True)
+    o = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
+    state_bytes = B * H * D * D * (4 + 4 + 2 + 2)    # fp32 state, its other buffer and their bf16 copies
+    out = {"layers": layers, "what": "timing-only: 4 queries + 1 commit (or cache append) per layer per frame; "
+                                     "softmax layers attend over every cached frame plus the current one",
+           "kv_bytes_per_frame_per_softmax_layer": frame_kv, "arl2_state_bytes_per_layer": state_bytes, "shares": {}}
+    for share in shares:
+        n_arl2 = int(round(share * layers))
+        n_soft = layers - n_arl2
+        rows = []
+        for N in Ns:
+            for c in caches[:n_soft]:
+                c.reset()
+                for f in range(N - 1):
+                    _, k, v = frames[f % CYCLE][0][QUERIES][:3]
+                    c.commit(k, v)
+            for lay in arl2s[:n_arl2]:
+                lay.reset()
+
+            def stack_frame(f):
+                passes, a, b = frames[f % CYCLE]
+                for i in range(layers):
+                    if i < n_arl2:      # ARL2 layers first; order does not change the total
+                        lay = arl2s[i]
+                        for p in range(QUERIES):
+                            lay.query(*passes[p][:3], out=o)
+                        _, k, v = passes[QUERIES][:3]
+                        lay.commit(k, v, a, b)
+                    else:
+                        c = caches[i - n_arl2]
+                        for p in range(QUERIES):
+                            c.query(*passes[p][:3], out=o)
+                        _, k, v = passes[QUERIES][:3]
+                        c.commit(k, v)
+
+            torch.cuda.synchronize()
+            # A softmax layer's query also copies the frame's k and v into the cache: count
+            # every copy as a launch.
+            queue_ahead(2 * (n_arl2 * (QUERIES + 1) + n_soft * (3 * QUERIES + 2)) + 2)
+            st, en = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            st.record(stream)
+            stack_frame(N - 1)
+            stack_frame(N)
+            en.record(stream)
+            torch.cuda.synchronize()
+            rows.append({"N": N, "ms_per_frame": st.elapsed_time(en) / 2, "kv_bytes": n_soft * N * frame_kv,
+                         "arl2_state_bytes": n_arl2 * state_bytes})
+        out["shares"][f"{share:.2f}"] = {"arl2_layers": n_arl2, "softmax_layers": n_soft, "frames": rows}
+    status = [c.status() for c in caches] + [lay.status() for lay in arl2s]
+    out["status"] = max(status) if status else 0
+    for c in caches:
+        c.close()
+    for lay in arl2s:
+        lay.close()
+    torch.cuda.empty_cache()
+    return out
+
+
 def max_over_ranks(values, device, world):
     """Each rank's timings -> the maximum over ranks, elementwise (the job is as slow as its
     slowest rank). Uses the default process group when world > 1."""
@@ -320,6 +408,8 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# fp32 FMA rate of the SMs (no tensor cores): 148 SMs x 128 lanes x 2 flops x 1.965 GHz.
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 HOST_MS_PER_LAUNCH = 0.05   # generous bound on the host's cost to enqueue one launch or event
 
 
@@ -486,6 +576,122 @@ def stream_leg(layer, frames, stream, barrier, n=240):
             "layer_bytes": layer.memory_bytes, "frame_index_after": layer.frame_index}
 
 
+def clean_pass_leg(frames, maps, stream, barrier, n_windows=20, window=10, splits=(0,)):
+    """The fused clean pass against the two calls it replaces, with launch overlap on:
+    frames of 4 denoising queries + the fused clean pass (5 launches) against frames of
+    4 queries + the clean pass's query + the commit (6 launches), in alternating windows of
+    `window` frames (events around each window); and the clean pass alone, back to back,
+    against a query and a commit back to back. Both schedules produce the same outputs:
+    the clean pass's o, and S_N."""
+    from softmax_attention_ar_b200.arl2 import ARL2Layer
+    out = {"what": "per frame: 4 queries + fused clean pass, against 4 queries + query + commit",
+           "frames_per_window": window, "windows": n_windows, "splits": []}
+    for split in splits:
+        fused, sep = ARL2Layer(H, T, D, B), ARL2Layer(H, T, D, B)
+        for lay in (fused, sep):
+            lay.set_feature_maps(*maps)
+            lay.set_launch_overlap(True)
+        if split:
+            fused.set_clean_split(split)
+
+        def frame_fused(i):
+            passes, a, b = frames[i % len(frames)]
+            for p in range(QUERIES):
+                fused.query(*passes[p][:3], out=passes[p][3])
+            q, k, v, o = passes[QUERIES]
+            fused.clean_pass(q, k, v, a, b, out=o)
+
+        def frame_sep(i):
+            passes, a, b = frames[i % len(frames)]
+            for p in range(QUERIES):
+                sep.query(*passes[p][:3], out=passes[p][3])
+            q, k, v, o = passes[QUERIES]
+            sep.query(q, k, v, out=o)
+            sep.commit(k, v, a, b)
+
+        def clean_only(i):
+            passes, a, b = frames[i % len(frames)]
+            q, k, v, o = passes[QUERIES]
+            fused.clean_pass(q, k, v, a, b, out=o)
+
+        def pair_only(i):
+            passes, a, b = frames[i % len(frames)]
+            q, k, v, o = passes[QUERIES]
+            sep.query(q, k, v, out=o)
+            sep.commit(k, v, a, b)
+
+        for i in range(5):
+            frame_fused(i)
+            frame_sep(i)
+        f_rates, s_rates, c_rates, p_rates = [], [], [], []
+        for w in range(n_windows):
+            f_rates += _time_windows(frame_fused, stream, 1, window, w * window, barrier)
+            s_rates += _time_windows(frame_sep, stream, 1, window, w * window, barrier)
+            c_rates += _time_windows(clean_only, stream, 1, window, w * window, barrier)
+            p_rates += _time_windows(pair_only, stream, 1, window, w * window, barrier)
+        st = max(fused.status(), sep.status())
+        if st != 0:
+            raise RuntimeError(f"device status {st} in the clean-pass leg")
+        med = statistics.median
+        out["splits"].append({
+            "commit_sms": fused.clean_split, "requested": split,
+            "frames_per_s_fused": med(f_rates), "frames_per_s_separate": med(s_rates),
+            "us_per_frame_fused": 1e6 / med(f_rates), "us_per_frame_separate": 1e6 / med(s_rates),
+            "us_clean_pass_fused": 1e6 / med(c_rates), "us_query_plus_commit": 1e6 / med(p_rates)})
+        fused.close()
+        sep.close()
+    return out
+
+
+def token_level_leg(frames, maps, stream, barrier, n_windows=10, window=5):
+    """Token-level access (the ablation): frames of 4 token-level queries + 1 token-level
+    commit, and each call alone in back-to-back windows. A token-level query is three launches
+    (the intra branch, the projections, the scan), a commit two (the projections, the scan).
+    The scan is fp32 on the CUDA cores: its rate is reported against the SMs' fp32 peak."""
+    from softmax_attention_ar_b200.arl2 import ARL2Layer
+    lay = ARL2Layer(H, T, D, B)
+    lay.set_feature_maps(*maps)
+
+    def frame(i):
+        passes, a, b = frames[i % len(frames)]
+        for p in range(QUERIES):
+            lay.query_token(*passes[p][:3], a, b, out=passes[p][3])
+        _, k, v, _ = passes[QUERIES]
+        lay.commit_token(k, v, a, b)
+
+    def query_only(i):
+        passes, a, b = frames[i % len(frames)]
+        lay.query_token(*passes[0][:3], a, b, out=passes[0][3])
+
+    def commit_only(i):
+        passes, a, b = frames[i % len(frames)]
+        _, k, v, _ = passes[QUERIES]
+        lay.commit_token(k, v, a, b)
+
+    for i in range(3):
+        frame(i)
+    f_rates = _time_windows(frame, stream, n_windows, window, 0, barrier)
+    q_rates = _time_windows(query_only, stream, n_windows, window, 0, barrier)
+    c_rates = _time_windows(commit_only, stream, n_windows, window, 0, barrier)
+    if lay.status() != 0:
+        raise RuntimeError("device status in the token-level leg")
+    lay.close()
+    med = statistics.median
+    q_us, c_us = 1e6 / med(q_rates), 1e6 / med(c_rates)
+    # Scan arithmetic per token and column of S: k'.s and q'.s (2d flops each) and the update
+    # s = alpha s + (beta u) k' (3d flops); a commit has no q'.s.
+    scan_q = B * H * T * 7 * D * D
+    scan_c = B * H * T * 5 * D * D
+    return {"what": "token-level access: per frame 4 queries (intra + projections + scan) and 1 commit "
+                    "(projections + scan)",
+            "frames_per_s": med(f_rates), "us_per_frame": 1e6 / med(f_rates),
+            "us_query": q_us, "us_commit": c_us,
+            "scan_flops_query": scan_q, "scan_flops_commit": scan_c,
+            "fp32_peak_tflops": FP32_PEAK_TFLOPS,
+            "commit_tflops": scan_c / (c_us * 1e-6) / 1e12,
+            "commit_frac_of_fp32_peak": scan_c / (c_us * 1e-6) / 1e12 / FP32_PEAK_TFLOPS}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -622,6 +828,13 @@ def run_ours(args, rank, world, local_rank):
         line["sweep"] = sweep_info
     if not args.no_kv_baseline:
         line["kv_cache_baseline"] = kv_cache_baseline(frames, dev, elapsed_ms / args.steps, layer.memory_bytes)
+    if not args.no_hybrid_stack:
+        line["hybrid_stack"] = hybrid_stack(frames, dev, stream)
+    if not args.no_token_level:
+        line["token_level"] = token_level_leg(frames, maps, stream, barrier)
+    if not args.no_clean_pass:
+        line["clean_pass"] = clean_pass_leg(frames, maps, stream, barrier,
+                                            splits=tuple(int(x) for x in args.clean_splits.split(",")))
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     print(json.dumps(line), flush=True)
@@ -638,6 +851,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer (e2e) measurement")
     ap.add_argument("--no-kv-baseline", action="store_true", help="skip the growing-KV-cache comparison")
     ap.add_argument("--no-sweep", action="store_true", help="skip the token/batch sweep")
+    ap.add_argument("--no-hybrid-stack", action="store_true", help="skip the 30-layer hybrid stack timing")
+    ap.add_argument("--no-clean-pass", action="store_true", help="skip the fused clean pass comparison")
+    ap.add_argument("--no-token-level", action="store_true", help="skip the token-level access timing")
+    ap.add_argument("--clean-splits", default="0", help="commit SMs of the fused clean pass to time (0: automatic)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -31,7 +31,8 @@
  *     alpha and beta are fp32 [B, H, T]. The state is fp32 [B, H, d_k, d_v].
  *   - The caller owns every buffer it passes. The library owns the two state buffers, its
  *     copies of the feature maps, its scratch and its staging buffers. It allocates all of
- *     them in arl2_create and frees them in arl2_destroy, so no call allocates memory.
+ *     them in arl2_create and frees them in arl2_destroy, so no per-frame call allocates
+ *     memory (only the tuning call arl2_set_clean_split may).
  *   - Supported shapes: d_k == d_v == d in {32, 64, 128}; 1 <= T <= 4096; B >= 1; H >= 1;
  *     B * H <= 65535. Other shapes return ARL2_ERR_UNSUPPORTED. The device must be sm_100.
  *   - A context is not thread-safe. Calls on one context must be ordered by the caller,
@@ -91,7 +92,50 @@ arl2_status arl2_frame_query(arl2_ctx* ctx, const arl2_bf16* q, const arl2_bf16*
 arl2_status arl2_frame_commit(arl2_ctx* ctx, const arl2_bf16* k, const arl2_bf16* v,
                               const float* alpha, const float* beta, arl2_stream stream);
 
-/* Host-buffer forms of the two calls above, for callers whose data is in host memory.
+/* The clean pass of frame N in one launch: the query of arl2_frame_query and the commit of
+ * arl2_frame_commit on the same k and v (§2.2 clean-pass update: the final, clean forward
+ * pass both reads S_{N-1} for its own output and writes S_N). The result equals calling
+ * arl2_frame_query(q, k, v, o) then arl2_frame_commit(k, v, alpha, beta) on the same stream,
+ * up to the order of floating-point sums: o reads S_{N-1}, S_N goes into the other state
+ * buffer and the frame count advances. Part of the GPU runs the query while the rest runs
+ * the commit, so the commit's latency hides behind the query. Arguments as for those two
+ * calls; o must not overlap q, k, v, alpha or beta. */
+arl2_status arl2_frame_clean_pass(arl2_ctx* ctx, const arl2_bf16* q, const arl2_bf16* k,
+                                  const arl2_bf16* v, arl2_bf16* o, const float* alpha,
+                                  const float* beta, arl2_stream stream);
+
+/* How many SMs the clean pass gives the commit (the rest run the query). 0 (the default)
+ * picks the number from a cost model of the two parts; n > 0 asks for n, clamped to
+ * [1, B * H * ceil(T / 128)] and to leave one SM for the query. Synchronises the device, and
+ * allocates when the new split needs more scratch (ARL2_ERR_OOM if that fails; the old split
+ * then stays). For tuning and tests; results differ between splits only in the order of
+ * floating-point sums. */
+arl2_status arl2_set_clean_split(arl2_ctx* ctx, int commit_sms);
+
+/* The SMs the clean pass currently gives the commit; -1 for a NULL context. */
+int arl2_clean_split(const arl2_ctx* ctx);
+
+/* ---- Token-level access (the ablation of §4, "Ablations") ------------------------------
+ * The pages report that letting the state advance token by token inside a frame, instead of
+ * every token reading S_{N-1}, degrades quality; they give no form. This library reads it as
+ * the §2.1 update applied to one token at a time, in token order, from S_{N-1}: per (batch,
+ * head), for t = 0..T-1,
+ *   o_inter[t] = q'_t S,    S <- alpha_t S + beta_t k'_t^T (v'_t - k'_t S)
+ * with q' = q Wq_h, k' = rownorm(k Wk_h), v' = v Wv_h, and the per-token gates alpha_t (not
+ * their mean) and beta_t (not beta_t / T). Layouts and alignment as above.
+ *   query:  o = softmax(q k^T / sqrt(d)) v + o_inter, the scan running over this pass's own
+ *           k, v and gates; never writes the state.
+ *   commit: S_N = the state after the last token of the clean pass; advances the frame count.
+ * The scan is sequential in the tokens: these calls run an fp32 scan on the CUDA cores, far
+ * slower than the frame-level calls. o must not overlap q, k, v, alpha or beta. */
+arl2_status arl2_frame_query_token(arl2_ctx* ctx, const arl2_bf16* q, const arl2_bf16* k,
+                                   const arl2_bf16* v, arl2_bf16* o, const float* alpha,
+                                   const float* beta, arl2_stream stream);
+arl2_status arl2_frame_commit_token(arl2_ctx* ctx, const arl2_bf16* k, const arl2_bf16* v,
+                                    const float* alpha, const float* beta, arl2_stream stream);
+
+/* Host-buffer forms of arl2_frame_query and arl2_frame_commit, for callers whose data is in
+ * host memory.
  * Each call copies its inputs into library-owned staging, runs the kernel on the stream
  * and (for the query) copies o back. The copies run on two internal streams, and the
  * calls take two staging sets by turns: one call's input copy overlaps the previous
@@ -105,6 +149,32 @@ arl2_status arl2_frame_query_host(arl2_ctx* ctx, const arl2_bf16* q_host, const 
 arl2_status arl2_frame_commit_host(arl2_ctx* ctx, const arl2_bf16* k_host, const arl2_bf16* v_host,
                                    const float* alpha_host, const float* beta_host,
                                    arl2_stream stream);
+
+/* ---- Gates produced from the hidden state ----------------------------------------------
+ * §2.1 calls the forget gate alpha and the rate beta per-token learned projections without
+ * giving their form. This library reads them as a linear projection of the token's hidden
+ * state per head plus a bias, through a sigmoid (both stay in (0, 1)):
+ *   alpha[b, h, t] = sigmoid(x[b, t, :] . Wa[h, :] + ba[h])
+ *   beta[b, h, t]  = sigmoid(x[b, t, :] . Wb[h, :] + bb[h])
+ * x is the layer's hidden state, bf16 [B, T, D] with D = H * d (the model width), 16-byte
+ * aligned. Supported when 2H <= 64 (H <= 32); otherwise these calls return
+ * ARL2_ERR_UNSUPPORTED and the gates are passed to arl2_frame_commit as before. */
+
+/* Copy the gate projections into the library: Wa, Wb bf16 [H, D] (rows of the model width),
+ * ba, bb fp32 [H]; device or host memory, stream-ordered like arl2_set_feature_maps. */
+arl2_status arl2_set_gate_weights(arl2_ctx* ctx, const arl2_bf16* Wa, const arl2_bf16* Wb,
+                                  const float* ba, const float* bb, arl2_stream stream);
+
+/* The gates alone: alpha, beta fp32 [B, H, T] (device memory, 4-byte aligned) from x.
+ * ARL2_ERR_STATE before arl2_set_gate_weights. */
+arl2_status arl2_frame_gates(arl2_ctx* ctx, const arl2_bf16* x, float* alpha, float* beta,
+                             arl2_stream stream);
+
+/* The clean-pass commit of frame N with its gates produced from x (the clean pass's hidden
+ * state): the gate kernel writes alpha and beta into library-owned buffers, then the commit
+ * runs as arl2_frame_commit on them. k, v as for arl2_frame_commit. */
+arl2_status arl2_frame_commit_gated(arl2_ctx* ctx, const arl2_bf16* x, const arl2_bf16* k,
+                                    const arl2_bf16* v, arl2_stream stream);
 
 /* Reset the state to S_0 = 0 and the frame count to 0 (the start of a new video). */
 arl2_status arl2_reset(arl2_ctx* ctx, arl2_stream stream);

@@ -32,6 +32,14 @@ SIGNATURES = {
     "arl2_frame_commit": (_S, [_P, _P, _P, _P, _P, _P]),
     "arl2_frame_query_host": (_S, [_P, _P, _P, _P, _P, _P]),
     "arl2_frame_commit_host": (_S, [_P, _P, _P, _P, _P, _P]),
+    "arl2_frame_clean_pass": (_S, [_P, _P, _P, _P, _P, _P, _P, _P]),
+    "arl2_set_clean_split": (_S, [_P, _I]),
+    "arl2_clean_split": (_I, [_P]),
+    "arl2_frame_query_token": (_S, [_P, _P, _P, _P, _P, _P, _P, _P]),
+    "arl2_frame_commit_token": (_S, [_P, _P, _P, _P, _P, _P]),
+    "arl2_set_gate_weights": (_S, [_P, _P, _P, _P, _P, _P]),
+    "arl2_frame_gates": (_S, [_P, _P, _P, _P, _P]),
+    "arl2_frame_commit_gated": (_S, [_P, _P, _P, _P, _P]),
     "arl2_reset": (_S, [_P, _P]),
     "arl2_get_state": (_S, [_P, _P, _P]),
     "arl2_set_state": (_S, [_P, _P, _P]),
@@ -184,6 +192,51 @@ class ARL2Layer:
                                            _cuda(alpha, torch.float32, g, "alpha"), _cuda(beta, torch.float32, g, "beta"),
                                            _stream(stream)), "arl2_frame_commit")
 
+    def clean_pass(self, q, k, v, alpha, beta, out=None, stream=None) -> torch.Tensor:
+        """The clean pass in one launch: out = the query of (q, k, v) on S_{N-1}, and the commit
+        of (k, v, alpha, beta) into S_N."""
+        if out is None:
+            out = torch.empty(self.act_shape, dtype=torch.bfloat16, device=q.device)
+        s, g = self.act_shape, self.gate_shape
+        _check(self._lib.arl2_frame_clean_pass(self._ctx, _cuda(q, torch.bfloat16, s, "q"),
+                                               _cuda(k, torch.bfloat16, s, "k"), _cuda(v, torch.bfloat16, s, "v"),
+                                               _cuda(out, torch.bfloat16, s, "o"),
+                                               _cuda(alpha, torch.float32, g, "alpha"),
+                                               _cuda(beta, torch.float32, g, "beta"), _stream(stream)),
+               "arl2_frame_clean_pass")
+        return out
+
+    def set_clean_split(self, commit_sms: int) -> None:
+        """SMs the clean pass gives the commit (0: chosen by the library's cost model)."""
+        _check(self._lib.arl2_set_clean_split(self._ctx, int(commit_sms)), "arl2_set_clean_split")
+
+    @property
+    def clean_split(self) -> int:
+        """SMs the clean pass currently gives the commit."""
+        return self._lib.arl2_clean_split(self._ctx)
+
+    def query_token(self, q, k, v, alpha, beta, out=None, stream=None) -> torch.Tensor:
+        """Token-level access: intra attention plus the token-by-token readout of this pass."""
+        if out is None:
+            out = torch.empty(self.act_shape, dtype=torch.bfloat16, device=q.device)
+        s, g = self.act_shape, self.gate_shape
+        _check(self._lib.arl2_frame_query_token(self._ctx, _cuda(q, torch.bfloat16, s, "q"),
+                                                _cuda(k, torch.bfloat16, s, "k"), _cuda(v, torch.bfloat16, s, "v"),
+                                                _cuda(out, torch.bfloat16, s, "o"),
+                                                _cuda(alpha, torch.float32, g, "alpha"),
+                                                _cuda(beta, torch.float32, g, "beta"), _stream(stream)),
+               "arl2_frame_query_token")
+        return out
+
+    def commit_token(self, k, v, alpha, beta, stream=None) -> None:
+        """Token-level access: S_N = the state after the clean pass's last token."""
+        s, g = self.act_shape, self.gate_shape
+        _check(self._lib.arl2_frame_commit_token(self._ctx, _cuda(k, torch.bfloat16, s, "k"),
+                                                 _cuda(v, torch.bfloat16, s, "v"),
+                                                 _cuda(alpha, torch.float32, g, "alpha"),
+                                                 _cuda(beta, torch.float32, g, "beta"), _stream(stream)),
+               "arl2_frame_commit_token")
+
     def query_host(self, q, k, v, out, stream=None) -> torch.Tensor:
         """Host-buffer query: q, k, v, out are CPU tensors (pinned for asynchrony)."""
         s = self.act_shape
@@ -200,6 +253,36 @@ class ARL2Layer:
                                                 _host(alpha, torch.float32, g, "alpha"),
                                                 _host(beta, torch.float32, g, "beta"), _stream(stream)),
                "arl2_frame_commit_host")
+
+    def set_gate_weights(self, Wa, Wb, ba, bb, stream=None) -> None:
+        """Gate projections for gates produced from the hidden state: Wa, Wb bf16 [H, H*d];
+        ba, bb fp32 [H]."""
+        D = self.H * self.d
+        _check(self._lib.arl2_set_gate_weights(self._ctx, _dev(Wa, torch.bfloat16, (self.H, D), "Wa"),
+                                               _dev(Wb, torch.bfloat16, (self.H, D), "Wb"),
+                                               _dev(ba, torch.float32, (self.H,), "ba"),
+                                               _dev(bb, torch.float32, (self.H,), "bb"), _stream(stream)),
+               "arl2_set_gate_weights")
+
+    def gates(self, x, alpha=None, beta=None, stream=None):
+        """alpha, beta fp32 [B, H, T] from the hidden state x bf16 [B, T, H*d]."""
+        if alpha is None:
+            alpha = torch.empty(self.gate_shape, dtype=torch.float32, device=x.device)
+        if beta is None:
+            beta = torch.empty(self.gate_shape, dtype=torch.float32, device=x.device)
+        xs, g = (self.B, self.T, self.H * self.d), self.gate_shape
+        _check(self._lib.arl2_frame_gates(self._ctx, _cuda(x, torch.bfloat16, xs, "x"),
+                                          _cuda(alpha, torch.float32, g, "alpha"),
+                                          _cuda(beta, torch.float32, g, "beta"), _stream(stream)),
+               "arl2_frame_gates")
+        return alpha, beta
+
+    def commit_gated(self, x, k, v, stream=None) -> None:
+        """The clean-pass commit with its gates produced from the hidden state x."""
+        xs, s = (self.B, self.T, self.H * self.d), self.act_shape
+        _check(self._lib.arl2_frame_commit_gated(self._ctx, _cuda(x, torch.bfloat16, xs, "x"),
+                                                 _cuda(k, torch.bfloat16, s, "k"), _cuda(v, torch.bfloat16, s, "v"),
+                                                 _stream(stream)), "arl2_frame_commit_gated")
 
     def reset(self, stream=None) -> None:
         _check(self._lib.arl2_reset(self._ctx, _stream(stream)), "arl2_reset")

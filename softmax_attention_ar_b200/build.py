@@ -18,8 +18,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libarl2.so")
 BUILD_DIR = os.path.join(PKG, "_build")
-SOURCES = ["arl2_api.cu", "arl2_query.cu", "arl2_commit.cu", "arl2_noalloc.cu"]
-HEADERS = ["arl2_device.cuh", "arl2_kernels.h"]
+SOURCES = ["arl2_api.cu", "arl2_query.cu", "arl2_commit.cu", "arl2_clean.cu", "arl2_token.cu", "arl2_gates.cu",
+           "arl2_noalloc.cu"]
+HEADERS = ["arl2_device.cuh", "arl2_kernels.h", "arl2_query_body.cuh", "arl2_commit_rows.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

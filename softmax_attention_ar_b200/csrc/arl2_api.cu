@@ -63,6 +63,22 @@ bool make_mat_map(CUtensorMap* m, const void* ptr, int n, int d) {
   return make_map(m, ptr, 3, dims, str, box);
 }
 
+// [B, T, D] hidden states: dims (D, T, B), box (64, 128, 1).
+bool make_hidden_map(CUtensorMap* m, const void* ptr, int B, int T, int D) {
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)B};
+  const cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)T * D * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  return make_map(m, ptr, 3, dims, str, box);
+}
+
+// [rows, D] gate projections: dims (D, rows), box (64, box_rows); rows past `rows` read as zero.
+bool make_gate_map(CUtensorMap* m, const void* ptr, int rows, int D, int box_rows) {
+  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  const cuuint64_t str[1] = {(cuuint64_t)D * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  return make_map(m, ptr, 2, dims, str, box);
+}
+
 bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
@@ -134,6 +150,9 @@ cudaError_t device_setup(int dev) {
   if (dev >= 0 && dev < 64 && g_setup_done[dev]) return cudaSuccess;
   cudaError_t e = arl2::query_setup();
   if (e == cudaSuccess) e = arl2::commit_setup();
+  if (e == cudaSuccess) e = arl2::clean_setup();
+  if (e == cudaSuccess) e = arl2::token_setup();
+  if (e == cudaSuccess) e = arl2::gates_setup();
   if (e == cudaSuccess && dev >= 0 && dev < 64) g_setup_done[dev] = true;
   return e;
 }
@@ -183,6 +202,20 @@ struct arl2_ctx {
   unsigned host_turn = 0;
   arl2::QueryPlan qplan{};        // stream-K split of the query kernel
   float* cscratch = nullptr;      // the commit's per-group partial U and alpha sums
+  arl2::CleanPlan cplan{};        // split of the fused clean pass
+  float* clscratch = nullptr;     // its commit segments' partial U and alpha sums
+  size_t clscratch_floats = 0;
+  unsigned int* clcounters = nullptr;   // its per-(batch, head) arrival counters
+  size_t qscratch_floats = 0;     // query scratch and flags, sized for both query splits
+  size_t qflag_count = 0;
+  float* tscratch = nullptr;      // token-level access: q', k', v' of one pass (fp32)
+  // Gates produced from the hidden state (only when 2H <= kMaxGateCols): Wg = [Wa; Wb] bf16
+  // [2H, D], its bias [2H] and the gates of the last gated commit, alpha then beta [B, H, T].
+  uint16_t* Wg = nullptr;
+  float* bg = nullptr;
+  float* gate_buf = nullptr;
+  bool gates_set = false;
+  CUtensorMap tm_wg;
   float* qscratch = nullptr;      // its partial records
   int* qflags = nullptr;          // their published flags
   int qepoch = 0;                 // epoch of the last query launch
@@ -223,6 +256,13 @@ struct arl2_kvcache {
 };
 
 namespace {
+
+// Gates produced from the hidden state: 2H projection rows, rounded up to 16 for the MMA.
+int gate_cols(int H) { return (2 * H + 15) / 16 * 16; }
+bool gates_supported(int H, int D) { return gate_cols(H) <= arl2::kMaxGateCols && D % 8 == 0; }
+
+// Launch the gate producer: alpha, beta [B, H, T] from x [B, T, D] (the context's Wg, bg).
+arl2_status gates_impl(arl2_ctx* c, const void* x, float* alpha, float* beta, cudaStream_t st);
 
 // Point a query launch at its stream-K plan and scratch.
 // Epochs of successive launches on one set of flags: nonzero, never the previous one.
@@ -274,6 +314,12 @@ void free_ctx(arl2_ctx* c) {
   cudaFree(c->qscratch);
   cudaFree(c->qflags);
   cudaFree(c->cscratch);
+  cudaFree(c->clscratch);
+  cudaFree(c->clcounters);
+  cudaFree(c->tscratch);
+  cudaFree(c->Wg);
+  cudaFree(c->bg);
+  cudaFree(c->gate_buf);
   delete c;
 }
 
@@ -342,9 +388,178 @@ arl2_status commit_impl(arl2_ctx* c, const void* k, const void* v, const float* 
   return ARL2_OK;
 }
 
+arl2_status clean_impl(arl2_ctx* c, const void* q, const void* k, const void* v, void* o, const float* alpha,
+                       const float* beta, cudaStream_t st) {
+  const CUtensorMap* mq = c->acts.get(q, c->B, c->T, c->H, c->d);
+  const CUtensorMap* mk = c->acts.get(k, c->B, c->T, c->H, c->d);
+  const CUtensorMap* mv = c->acts.get(v, c->B, c->T, c->H, c->d);
+  const CUtensorMap* mo = c->outs.get(o, c->B, c->T, c->H, c->d);
+  if (!mq || !mk || !mv || !mo) return ARL2_ERR_CUDA;
+  arl2::QueryArgs a{};
+  a.o = static_cast<uint16_t*>(o);
+  a.T = c->T;
+  a.kv_len = c->T;
+  a.B = c->B;
+  a.H = c->H;
+  a.d = c->d;
+  a.state_slot = c->cur;
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->d)));
+  a.err = c->err;
+  a.timeout_ns = c->timeout_ns;
+  a.stall = c->stall_next ? 1 : 0;
+  c->stall_next = false;
+  set_plan(&a, c->cplan.q, c->qscratch, c->qflags, next_epoch(&c->qepoch));
+  const arl2::CleanPlan& p = c->cplan;
+  a.first_cta = p.commit_ctas;   // the commit CTAs come first in the grid
+  arl2::CommitStreamArgs m{};
+  m.alpha = alpha;
+  m.beta = beta;
+  m.S_old = c->S[c->cur];
+  m.S_new = c->S[c->cur ^ 1];
+  m.S_new_bf16 = c->S_bf16 + (size_t)(c->cur ^ 1) * c->state_elems();
+  const size_t slots = (size_t)c->B * c->H * p.max_pieces;
+  m.part_u = c->clscratch;
+  m.part_alpha = c->clscratch + slots * 32 * 128 * 4;
+  m.counters = c->clcounters;
+  m.T = c->T;
+  m.B = c->B;
+  m.H = c->H;
+  m.d = c->d;
+  m.state_slot = c->cur;
+  m.inv_T = 1.0f / static_cast<float>(c->T);
+  m.nchunks = p.nchunks;
+  m.units = p.cunits;
+  m.num_ctas = p.commit_ctas;
+  m.max_pieces = p.max_pieces;
+  m.err = c->err;
+  m.timeout_ns = c->timeout_ns;
+  const size_t act = c->act_elems() * 2, gate = (size_t)c->B * c->H * c->T * 4;
+  const bool dependent = c->overlap && clear_of_last_output(st, {{q, act}, {k, act}, {v, act}, {alpha, gate},
+                                                                 {beta, gate}});
+  record_query_output(st, o, act);
+  if (arl2::launch_clean(*mq, *mk, *mv, c->tm_w[0], c->tm_s, *mo, c->tm_w[1], c->tm_w[2], a, m, st, dependent) !=
+      cudaSuccess)
+    return ARL2_ERR_CUDA;
+  c->cur ^= 1;
+  ++c->frame;
+  return ARL2_OK;
+}
+
+// Token-level access: the projections of the pass to scratch, then the scan. A query first
+// writes the intra branch into o (the query kernel without its readout); the scan adds o_inter.
+arl2_status token_impl(arl2_ctx* c, const void* q, const void* k, const void* v, void* o, const float* alpha,
+                       const float* beta, cudaStream_t st) {
+  const bool query = q != nullptr;
+  const CUtensorMap* mk = c->acts.get(k, c->B, c->T, c->H, c->d);
+  const CUtensorMap* mv = c->acts.get(v, c->B, c->T, c->H, c->d);
+  const CUtensorMap* mq = query ? c->acts.get(q, c->B, c->T, c->H, c->d) : mk;
+  if (!mk || !mv || !mq) return ARL2_ERR_CUDA;
+  if (query) {
+    const CUtensorMap* mo = c->outs.get(o, c->B, c->T, c->H, c->d);
+    if (!mo) return ARL2_ERR_CUDA;
+    arl2::QueryArgs a{};
+    a.o = static_cast<uint16_t*>(o);
+    a.T = c->T;
+    a.kv_len = c->T;
+    a.B = c->B;
+    a.H = c->H;
+    a.d = c->d;
+    a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->d)));
+    a.err = c->err;
+    a.timeout_ns = c->timeout_ns;
+    set_plan(&a, c->qplan, c->qscratch, c->qflags, next_epoch(&c->qepoch));
+    if (arl2::launch_query(false, *mq, *mk, *mv, c->tm_w[0], c->tm_s, *mo, a, st, false) != cudaSuccess)
+      return ARL2_ERR_CUDA;
+  }
+  arl2::TokenArgs t{};
+  const size_t rows = (size_t)c->B * c->H * c->T;
+  const int P = c->d + 4 * arl2::kTokenParts;
+  t.alpha = alpha;
+  t.beta = beta;
+  t.k_out = c->tscratch;
+  t.q_out = query ? c->tscratch + rows * P : nullptr;
+  t.v_out = c->tscratch + 2 * rows * P;
+  t.S_old = c->S[c->cur];
+  t.S_new = c->S[c->cur ^ 1];
+  t.S_new_bf16 = c->S_bf16 + (size_t)(c->cur ^ 1) * c->state_elems();
+  t.o = query ? static_cast<uint16_t*>(o) : nullptr;
+  t.T = c->T;
+  t.B = c->B;
+  t.H = c->H;
+  t.d = c->d;
+  t.err = c->err;
+  t.timeout_ns = c->timeout_ns;
+  if (arl2::launch_token_project(*mq, *mk, *mv, c->tm_w[0], c->tm_w[1], c->tm_w[2], t, st) != cudaSuccess ||
+      arl2::launch_token_scan(t, st) != cudaSuccess)
+    return ARL2_ERR_CUDA;
+  if (query) {
+    record_query_output(st, o, c->act_elems() * 2);
+  } else {
+    c->cur ^= 1;
+    ++c->frame;
+  }
+  return ARL2_OK;
+}
+
+arl2_status gates_impl(arl2_ctx* c, const void* x, float* alpha, float* beta, cudaStream_t st) {
+  CUtensorMap tm_x;
+  if (!make_hidden_map(&tm_x, x, c->B, c->T, c->H * c->d)) return ARL2_ERR_CUDA;
+  arl2::GateArgs g{};
+  g.bias = c->bg;
+  g.alpha = alpha;
+  g.beta = beta;
+  g.B = c->B;
+  g.T = c->T;
+  g.H = c->H;
+  g.D = c->H * c->d;
+  g.ngates = 2 * c->H;
+  g.ncols = gate_cols(c->H);
+  g.tmem_cols = g.ncols <= 32 ? 32 : 64;
+  g.err = c->err;
+  g.timeout_ns = c->timeout_ns;
+  return arl2::launch_gates(tm_x, c->tm_wg, g, st) == cudaSuccess ? ARL2_OK : ARL2_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
+
+arl2_status arl2_set_gate_weights(arl2_ctx* c, const arl2_bf16* Wa, const arl2_bf16* Wb, const float* ba,
+                                  const float* bb, arl2_stream stream) {
+  if (!c || !Wa || !Wb || !ba || !bb) return ARL2_ERR_INVALID_ARG;
+  if (!c->Wg) return ARL2_ERR_UNSUPPORTED;
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t rows = (size_t)c->H * c->H * c->d * 2;   // H rows of D = H d bf16
+  if (cudaMemcpyAsync(c->Wg, Wa, rows, cudaMemcpyDefault, st) != cudaSuccess ||
+      cudaMemcpyAsync(c->Wg + (size_t)c->H * c->H * c->d, Wb, rows, cudaMemcpyDefault, st) != cudaSuccess ||
+      cudaMemcpyAsync(c->bg, ba, (size_t)c->H * 4, cudaMemcpyDefault, st) != cudaSuccess ||
+      cudaMemcpyAsync(c->bg + c->H, bb, (size_t)c->H * 4, cudaMemcpyDefault, st) != cudaSuccess)
+    return ARL2_ERR_CUDA;
+  c->gates_set = true;
+  return ARL2_OK;
+}
+
+arl2_status arl2_frame_gates(arl2_ctx* c, const arl2_bf16* x, float* alpha, float* beta, arl2_stream stream) {
+  if (!c || !aligned16(x) || !aligned4(alpha) || !aligned4(beta)) return ARL2_ERR_INVALID_ARG;
+  if (!c->Wg) return ARL2_ERR_UNSUPPORTED;
+  if (!c->gates_set) return ARL2_ERR_STATE;
+  return gates_impl(c, x, alpha, beta, (cudaStream_t)stream);
+}
+
+arl2_status arl2_frame_commit_gated(arl2_ctx* c, const arl2_bf16* x, const arl2_bf16* k, const arl2_bf16* v,
+                                    arl2_stream stream) {
+  if (!c || !aligned16(x) || !aligned16(k) || !aligned16(v)) return ARL2_ERR_INVALID_ARG;
+  if (!c->Wg) return ARL2_ERR_UNSUPPORTED;
+  if (!c->gates_set || !c->maps_set) return ARL2_ERR_STATE;
+  cudaStream_t st = (cudaStream_t)stream;
+  float* alpha = c->gate_buf;
+  float* beta = c->gate_buf + (size_t)c->B * c->H * c->T;
+  arl2_status r = gates_impl(c, x, alpha, beta, st);
+  if (r != ARL2_OK) return r;
+  // The commit reads the gates from its first instructions, so it starts after the gate
+  // kernel has completed (a normal launch, not a programmatic dependent).
+  return commit_impl(c, k, v, alpha, beta, st, false);
+}
 
 arl2_status arl2_create(int H, int T, int d_k, int d_v, int B, arl2_ctx** out) {
   if (!out) return ARL2_ERR_INVALID_ARG;
@@ -375,9 +590,21 @@ arl2_status arl2_create(int H, int T, int d_k, int d_v, int B, arl2_ctx** out) {
     for (int i = 0; i < 2 && ok; ++i) ok = dev_alloc(&c->stage_f32[set][i], (size_t)B * H * T, &c->bytes);
   }
   c->qplan = arl2::plan_query(B, H, T, T, sms);
-  ok = ok && dev_alloc(&c->qscratch, arl2::query_scratch_floats(c->qplan), &c->bytes);
-  ok = ok && dev_alloc(&c->qflags, arl2::query_flag_count(c->qplan), &c->bytes);
+  c->cplan = arl2::plan_clean(B, H, T, sms, 0);
+  c->qscratch_floats = std::max(arl2::query_scratch_floats(c->qplan), arl2::query_scratch_floats(c->cplan.q));
+  c->qflag_count = std::max(arl2::query_flag_count(c->qplan), arl2::query_flag_count(c->cplan.q));
+  c->clscratch_floats = arl2::clean_scratch_floats(c->cplan);
+  ok = ok && dev_alloc(&c->qscratch, c->qscratch_floats, &c->bytes);
+  ok = ok && dev_alloc(&c->qflags, c->qflag_count, &c->bytes);
   ok = ok && dev_alloc(&c->cscratch, arl2::commit_scratch_floats(B, H, c->ngroups), &c->bytes);
+  ok = ok && dev_alloc(&c->clscratch, c->clscratch_floats, &c->bytes);
+  ok = ok && dev_alloc(&c->clcounters, (size_t)B * H, &c->bytes);
+  ok = ok && dev_alloc(&c->tscratch, arl2::token_scratch_floats(B, H, T, d_k), &c->bytes);
+  const int D = H * d_k;   // the model width the gate projections read
+  if (ok && gates_supported(H, D)) {
+    ok = dev_alloc(&c->Wg, (size_t)2 * H * D, &c->bytes) && dev_alloc(&c->bg, (size_t)2 * H, &c->bytes) &&
+         dev_alloc(&c->gate_buf, (size_t)2 * B * H * T, &c->bytes);
+  }
   if (!ok) {
     free_ctx(c);
     return ARL2_ERR_OOM;
@@ -391,10 +618,12 @@ arl2_status arl2_create(int H, int T, int d_k, int d_v, int B, arl2_ctx** out) {
   ok = ok && cudaMemset(c->S[0], 0, c->state_elems() * 4) == cudaSuccess &&
        cudaMemset(c->S[1], 0, c->state_elems() * 4) == cudaSuccess &&
        cudaMemset(c->S_bf16, 0, 2 * c->state_elems() * 2) == cudaSuccess &&
-       cudaMemset(c->qflags, 0, arl2::query_flag_count(c->qplan) * sizeof(int)) == cudaSuccess &&
+       cudaMemset(c->qflags, 0, c->qflag_count * sizeof(int)) == cudaSuccess &&
+       cudaMemset(c->clcounters, 0, (size_t)B * H * sizeof(unsigned int)) == cudaSuccess &&
        cudaMemset(c->err, 0, sizeof(unsigned int)) == cudaSuccess;
   for (int i = 0; i < 3 && ok; ++i) ok = make_mat_map(&c->tm_w[i], c->W[i], H, d_k);
   ok = ok && make_mat_map(&c->tm_s, c->S_bf16, 2 * B * H, d_k);
+  if (ok && c->Wg) ok = make_gate_map(&c->tm_wg, c->Wg, 2 * H, D, gate_cols(H));
   if (ok) ok = cudaDeviceSynchronize() == cudaSuccess;
   if (!ok) {
     free_ctx(c);
@@ -428,6 +657,79 @@ arl2_status arl2_frame_commit(arl2_ctx* c, const arl2_bf16* k, const arl2_bf16* 
   if (!c || !aligned16(k) || !aligned16(v) || !aligned4(alpha) || !aligned4(beta)) return ARL2_ERR_INVALID_ARG;
   if (!c->maps_set) return ARL2_ERR_STATE;
   return commit_impl(c, k, v, alpha, beta, (cudaStream_t)stream);
+}
+
+arl2_status arl2_frame_clean_pass(arl2_ctx* c, const arl2_bf16* q, const arl2_bf16* k, const arl2_bf16* v,
+                                  arl2_bf16* o, const float* alpha, const float* beta, arl2_stream stream) {
+  if (!c || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(alpha) ||
+      !aligned4(beta))
+    return ARL2_ERR_INVALID_ARG;
+  if (!c->maps_set) return ARL2_ERR_STATE;
+  return clean_impl(c, q, k, v, o, alpha, beta, (cudaStream_t)stream);
+}
+
+arl2_status arl2_set_clean_split(arl2_ctx* c, int commit_sms) {
+  if (!c || commit_sms < 0) return ARL2_ERR_INVALID_ARG;
+  const arl2::CleanPlan p = arl2::plan_clean(c->B, c->H, c->T, c->num_sms, commit_sms);
+  const size_t qs = std::max(c->qscratch_floats, arl2::query_scratch_floats(p.q));
+  const size_t qf = std::max(c->qflag_count, arl2::query_flag_count(p.q));
+  const size_t cl = std::max(c->clscratch_floats, arl2::clean_scratch_floats(p));
+  if (cudaDeviceSynchronize() != cudaSuccess) return ARL2_ERR_CUDA;   // no launch still uses the scratch
+  float *nqs = nullptr, *ncl = nullptr;
+  int* nqf = nullptr;
+  size_t added = 0;
+  bool ok = true;
+  if (qs > c->qscratch_floats) ok = dev_alloc(&nqs, qs, &added);
+  if (ok && qf > c->qflag_count) ok = dev_alloc(&nqf, qf, &added) && cudaMemset(nqf, 0, qf * sizeof(int)) == cudaSuccess;
+  if (ok && cl > c->clscratch_floats) ok = dev_alloc(&ncl, cl, &added);
+  if (!ok) {
+    cudaFree(nqs);
+    cudaFree(nqf);
+    cudaFree(ncl);
+    return ARL2_ERR_OOM;
+  }
+  if (nqs) {
+    cudaFree(c->qscratch);
+    c->bytes -= c->qscratch_floats * sizeof(float);
+    c->qscratch = nqs;
+    c->qscratch_floats = qs;
+  }
+  if (nqf) {
+    cudaFree(c->qflags);
+    c->bytes -= c->qflag_count * sizeof(int);
+    c->qflags = nqf;
+    c->qflag_count = qf;
+  }
+  if (ncl) {
+    cudaFree(c->clscratch);
+    c->bytes -= c->clscratch_floats * sizeof(float);
+    c->clscratch = ncl;
+    c->clscratch_floats = cl;
+  }
+  c->bytes += added;
+  // Every head's counter restarts at zero for the new segment counts.
+  if (cudaMemset(c->clcounters, 0, (size_t)c->B * c->H * sizeof(unsigned int)) != cudaSuccess)
+    return ARL2_ERR_CUDA;
+  c->cplan = p;
+  return ARL2_OK;
+}
+
+int arl2_clean_split(const arl2_ctx* c) { return c ? c->cplan.commit_ctas : -1; }
+
+arl2_status arl2_frame_query_token(arl2_ctx* c, const arl2_bf16* q, const arl2_bf16* k, const arl2_bf16* v,
+                                   arl2_bf16* o, const float* alpha, const float* beta, arl2_stream stream) {
+  if (!c || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(alpha) ||
+      !aligned4(beta))
+    return ARL2_ERR_INVALID_ARG;
+  if (!c->maps_set) return ARL2_ERR_STATE;
+  return token_impl(c, q, k, v, o, alpha, beta, (cudaStream_t)stream);
+}
+
+arl2_status arl2_frame_commit_token(arl2_ctx* c, const arl2_bf16* k, const arl2_bf16* v, const float* alpha,
+                                    const float* beta, arl2_stream stream) {
+  if (!c || !aligned16(k) || !aligned16(v) || !aligned4(alpha) || !aligned4(beta)) return ARL2_ERR_INVALID_ARG;
+  if (!c->maps_set) return ARL2_ERR_STATE;
+  return token_impl(c, nullptr, k, v, nullptr, alpha, beta, (cudaStream_t)stream);
 }
 
 arl2_status arl2_frame_query_host(arl2_ctx* c, const arl2_bf16* q, const arl2_bf16* k, const arl2_bf16* v,
@@ -486,7 +788,8 @@ arl2_status arl2_reset(arl2_ctx* c, arl2_stream stream) {
   cudaStream_t st = (cudaStream_t)stream;
   if (cudaMemsetAsync(c->S[0], 0, c->state_elems() * 4, st) != cudaSuccess ||
       cudaMemsetAsync(c->S[1], 0, c->state_elems() * 4, st) != cudaSuccess ||
-      cudaMemsetAsync(c->S_bf16, 0, 2 * c->state_elems() * 2, st) != cudaSuccess)
+      cudaMemsetAsync(c->S_bf16, 0, 2 * c->state_elems() * 2, st) != cudaSuccess ||
+      cudaMemsetAsync(c->clcounters, 0, (size_t)c->B * c->H * sizeof(unsigned int), st) != cudaSuccess)
     return ARL2_ERR_CUDA;
   c->cur = 0;
   c->frame = 0;

@@ -30,6 +30,7 @@
 // Shared memory: Wk | Wv | S | K0 K1 | V0 V1 (32 KiB tiles), then a control block.
 #include <algorithm>
 
+#include "arl2_commit_rows.cuh"
 #include "arl2_device.cuh"
 #include "arl2_kernels.h"
 
@@ -67,7 +68,6 @@ static_assert(kNumBars * 8 <= kCtlMisc, "barriers must fit their slot");
 static_assert(kSmemAlloc <= 232448, "shared memory per CTA");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColKp0 = 0, kColVp = 128, kColU = 256, kColKp1 = 384;
-constexpr float kNormEps = 1e-12f;
 constexpr int kRowWarps = 4;
 
 struct Smem {
@@ -194,8 +194,7 @@ __device__ void mma_issuer(const Smem& sm, uint32_t tmem, int nc, bool lead, con
 }
 
 // Warps 2-5: K' and R per chunk (thread = token row), then wait for U. Returns false if a
-// wait gave up. Sums of squares and the scalings run on paired fp32 operations with
-// independent accumulators, so the row's dependent chains stay short.
+// wait gave up.
 __device__ bool row_role(const Smem& sm, uint32_t tmem, const CommitArgs& a, int c0, int nc, int h, int b, int warp,
                          int lane, float* warp_sums, const Guard& g) {
   const int quarter = warp & 3;
@@ -223,67 +222,14 @@ __device__ bool row_role(const Smem& sm, uint32_t tmem, const CommitArgs& a, int
     // K' = Kp / max(|Kp|, eps) -> bf16, over the K tile (its MMA has finished).
     if (!mbar_wait_warp(sm.bar(kBarProjK + st), (i >> 1) & 1, g)) return false;
     tc_fence_after();
-    {
-      uint32_t kv[4][32];
-      tmem_ld32x2_wait(tmem + lane_off + col_kp(i), kv[0], tmem + lane_off + col_kp(i) + 32u, kv[1]);
-      tmem_ld32x2_wait(tmem + lane_off + col_kp(i) + 64u, kv[2], tmem + lane_off + col_kp(i) + 96u, kv[3]);
-      float2 ss[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) ss[j] = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float2 x = make_float2(__uint_as_float(kv[c][e]), __uint_as_float(kv[c][e + 1]));
-          ss[(e >> 1) & 3] = __ffma2_rn(x, x, ss[(e >> 1) & 3]);
-        }
-      const float2 s01 = __fadd2_rn(__fadd2_rn(ss[0], ss[1]), __fadd2_rn(ss[2], ss[3]));
-      const float inv = 1.f / fmaxf(sqrtf(s01.x + s01.y), kNormEps);
-      const float2 inv2 = make_float2(inv, inv);
-      const uint32_t tile = sm.k(st);
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint32_t* x = kv[c] + 8 * q;
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 y = __fmul2_rn(make_float2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), inv2);
-            w[e] = pack_bf16x2(y.x, y.y);
-          }
-          st_shared_v4(tile + swz_chunk(r, 4 * c + q), w[0], w[1], w[2], w[3]);
-        }
-    }
+    commit_rows_normalise(tmem + lane_off + col_kp(i), sm.k(st), r);
     fence_proxy_async_smem();
     tc_fence_before();
     warp_arrive(sm.bar(kBarKn));
     // R = (Vp - K'S) * beta_t / T -> bf16, over the V tile (its MMA has finished).
     if (!mbar_wait_warp(sm.bar(kBarKS), i & 1, g)) return false;
     tc_fence_after();
-    {
-      const uint32_t tile = sm.v(st);
-      const float2 cf = make_float2(coef, coef);
-      uint32_t vp[2][32];
-#pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) {
-        tmem_ld32x2_wait(tmem + lane_off + kColVp + 64u * c2, vp[0], tmem + lane_off + kColVp + 64u * c2 + 32u,
-                         vp[1]);
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 y = __fmul2_rn(
-                  make_float2(__uint_as_float(vp[c][8 * q + 2 * e]), __uint_as_float(vp[c][8 * q + 2 * e + 1])), cf);
-              w[e] = pack_bf16x2(y.x, y.y);
-            }
-            st_shared_v4(tile + swz_chunk(r, 4 * (2 * c2 + c) + q), w[0], w[1], w[2], w[3]);
-          }
-      }
-    }
+    commit_rows_residual(tmem + lane_off + kColVp, sm.v(st), r, coef);
     fence_proxy_async_smem();
     tc_fence_before();
     warp_arrive(sm.bar(kBarR));

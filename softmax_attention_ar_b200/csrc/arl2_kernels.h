@@ -25,7 +25,8 @@ struct QueryArgs {
   // Persistent stream-K split (see QueryPlan) and its scratch.
   int nq, nkv;            // query tiles and key tiles per (batch, head)
   long long units;        // B * H * nq * nkv (query tile, key tile) pairs
-  int num_ctas;           // grid size
+  int num_ctas;           // CTAs of the split
+  int first_cta;          // the split's CTAs are blockIdx.x in [first_cta, first_cta + num_ctas)
   int max_segs;           // CTAs sharing one query tile, at most
   float* part_o;          // [qtiles * max_segs][32 column quads][128 rows] float4: partial O accumulators
   float* part_ml;         // [qtiles * max_segs, 2, 128] running max (log2 units) and sum
@@ -67,6 +68,88 @@ struct ReduceArgs {
   int d;
   float inv_T;
 };
+
+// The fused clean pass (arl2_clean.cu): one launch whose first CTAs run the commit as a
+// stream over the B*H*nchunks chunk units, cut into num_ctas contiguous ranges, and whose
+// other CTAs run the query's stream-K split (QueryArgs, first_cta = the commit CTAs). A head
+// whose chunks span several CTAs is reduced by its last-arriving segment from per-segment
+// scratch slots.
+struct CommitStreamArgs {
+  const float* alpha;     // [B, H, T]
+  const float* beta;      // [B, H, T]
+  const float* S_old;     // [B*H, d, d] fp32 S_{N-1}
+  float* S_new;           // [B*H, d, d] fp32 S_N
+  uint16_t* S_new_bf16;   // [B*H, d, d] its bf16 copy
+  float* part_u;          // [B*H*max_pieces][32 column quads][128 rows] float4 partial U
+  float* part_alpha;      // [B*H*max_pieces] alpha sums of the segments
+  unsigned int* counters; // [B*H] segments arrived, wrapping at the head's segment count
+  int T, B, H, d;
+  int state_slot;         // state buffer read (S_{N-1}), for the bf16 copy's tensor map
+  float inv_T;
+  int nchunks;            // 128-token chunks per (batch, head)
+  long long units;        // B * H * nchunks
+  int num_ctas;           // the commit CTAs are blockIdx.x in [0, num_ctas)
+  int max_pieces;         // segments of one head, at most (scratch slots per head)
+  unsigned int* err;
+  unsigned long long timeout_ns;
+};
+struct CleanPlan {
+  QueryPlan q;            // the query CTAs' split
+  int commit_ctas;        // commit CTAs
+  int nchunks;
+  long long cunits;       // chunk units
+  int max_pieces;
+};
+// commit_ctas = 0 picks the split from a cost model; otherwise that many commit CTAs (clamped
+// to [1, chunk units] and to leave at least one query CTA).
+CleanPlan plan_clean(int B, int H, int T, int num_sms, int commit_ctas);
+size_t clean_scratch_floats(const CleanPlan& p);   // part_u, then part_alpha
+cudaError_t clean_setup();
+cudaError_t launch_clean(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                         const CUtensorMap& tm_wq, const CUtensorMap& tm_s, const CUtensorMap& tm_o,
+                         const CUtensorMap& tm_wk, const CUtensorMap& tm_wv, const QueryArgs& qa,
+                         const CommitStreamArgs& ca, cudaStream_t stream, bool dependent);
+
+// Token-level access (arl2_token.cu): projections to scratch, then the per-token scan.
+constexpr int kTokenParts = 8;   // lanes per column of S in the scan; rows of q', k' come in 8 parts
+struct TokenArgs {
+  const float* alpha;     // [B, H, T]
+  const float* beta;      // [B, H, T]
+  float* q_out;           // [B*H, T, d + 32] q' (padded parts); null for a commit
+  float* k_out;           // [B*H, T, d + 32] k' normalised (padded parts; part 0's padding holds alpha, beta)
+  float* v_out;           // [B*H, T, d] v'
+  const float* S_old;     // [B*H, d, d] fp32 S_{N-1}
+  float* S_new;           // [B*H, d, d] the final state (commit only)
+  uint16_t* S_new_bf16;   // its bf16 copy
+  uint16_t* o;            // [B, T, H, d] bf16: holds the intra branch; the scan adds o_inter (query only)
+  int T, B, H, d;
+  unsigned int* err;
+  unsigned long long timeout_ns;
+};
+size_t token_scratch_floats(int B, int H, int T, int d);
+cudaError_t token_setup();
+cudaError_t launch_token_project(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                                 const CUtensorMap& tm_wq, const CUtensorMap& tm_wk, const CUtensorMap& tm_wv,
+                                 const TokenArgs& a, cudaStream_t stream);
+cudaError_t launch_token_scan(const TokenArgs& a, cudaStream_t stream);
+
+// Gates produced from the hidden state (arl2_gates.cu): alpha, beta [B, H, T] fp32 from
+// x [B, T, D] bf16 and the stacked projections Wg = [Wa; Wb] of 2H rows plus a bias of 2H.
+constexpr int kMaxGateCols = 64;   // 2H rounded up to 16 is at most this (H <= 32)
+struct GateArgs {
+  const float* bias;      // [2H]: ba then bb
+  float* alpha;           // [B, H, T]
+  float* beta;            // [B, H, T]
+  int B, T, H, D;
+  int ngates;             // 2H
+  int ncols;              // 2H rounded up to 16: the MMA's N and the Wg box rows
+  int tmem_cols;          // TMEM columns allocated (a power of two, at least 32)
+  unsigned int* err;
+  unsigned long long timeout_ns;
+};
+int gate_split(int D);   // CTAs per cluster (slices of D)
+cudaError_t gates_setup();
+cudaError_t launch_gates(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const GateArgs& a, cudaStream_t stream);
 
 // Helpers defined in arl2_api.cu: device check and set-up (returns an arl2_status), and
 // the bf16 tensor maps every kernel reads through.
