@@ -510,9 +510,10 @@ __device__ __forceinline__ void commit_cta(const CUtensorMap& tm_k, const CUtens
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // Any kernel launched behind this one waits for the whole grid before it reads the state or
-  // writes anything this grid reads (see the query CTAs), so it may start early.
-  griddep_launch_dependents();
+  // No early trigger here: a kernel launched behind this one starts its CTAs once these have
+  // exited. The commit CTAs run the longest serial chains of the launch; letting the next
+  // query in early would give its last CTAs (in launch order) the SMs these CTAs hold only at
+  // their end, and delay that whole query.
 
   if (warp == 0) {
     producer(sm, &tm_k, &tm_v, &tm_wk, &tm_wv, &tm_s, a, cta, elect_one(), g);
@@ -551,11 +552,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     query_cta<true>(tm_q, tm_k, tm_v, tm_wq, tm_s, tm_o, qa, smem_raw);
 }
 
-// Cost model of the split, in microseconds of one CTA's work, from B200 timings of the two
-// standalone kernels at 480p and larger shapes: a query CTA spends about 1.24 us per (query
-// tile, key tile) unit plus about 3 us per segment (epilogue, readout, merge) and 8 us of
-// start-up and tail; a commit CTA about 2 us per 128-token chunk, 3 us per segment (its
-// weights and the epilogue), 2 us for a split head's reduction and 4 us of start-up.
+// Cost model of the split, in microseconds of one CTA's work, fitted to B200 timings of the
+// fused kernel and the standalone query at 480p and larger shapes: a query CTA spends about
+// 1.24 us per (query tile, key tile) unit plus about 3 us per segment (epilogue, readout,
+// merge) and 8 us of start-up and tail; a commit CTA about 5.5 us per 128-token chunk (its
+// four-MMA chain with two row passes between, next to the query CTAs), 3 us per segment, 2 us
+// for a split head's reduction and 4 us of start-up.
 double query_cta_cost(long long units, int ctas) {
   const double per = static_cast<double>((units + ctas - 1) / ctas);
   return 8.0 + 1.24 * per + 3.0 * 2.0;
@@ -563,7 +565,7 @@ double query_cta_cost(long long units, int ctas) {
 double commit_cta_cost(long long cunits, int nchunks, int ctas) {
   const long long per = (cunits + ctas - 1) / ctas;
   const long long segs = (per + nchunks - 1) / nchunks + 1;
-  return 4.0 + 2.0 * static_cast<double>(per) + 3.0 * static_cast<double>(segs) + 2.0;
+  return 4.0 + 5.5 * static_cast<double>(per) + 3.0 * static_cast<double>(segs) + 2.0;
 }
 
 }  // namespace
