@@ -336,9 +336,11 @@ def hybrid_stack(frames, dev, stream, layers=30, Ns=(1, 21, 60, 120), shares=(0.
             for lay in arl2s[:n_arl2]:
                 lay.reset()
 
-            def stack_frame(f):
+            def stack_frame(f, mid=None):
                 passes, a, b = frames[f % CYCLE]
                 for i in range(layers):
+                    if i == n_arl2 and mid is not None:
+                        mid.record(stream)   # the ARL2 layers are done, the softmax layers start
                     if i < n_arl2:      # ARL2 layers first; order does not change the total
                         lay = arl2s[i]
                         for p in range(QUERIES):
@@ -356,14 +358,19 @@ def hybrid_stack(frames, dev, stream, layers=30, Ns=(1, 21, 60, 120), shares=(0.
             # A softmax layer's query also copies the frame's k and v into the cache: count
             # every copy as a launch.
             queue_ahead(2 * (n_arl2 * (QUERIES + 1) + n_soft * (3 * QUERIES + 2)) + 2)
-            st, en = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            st, md, mid, en = (torch.cuda.Event(enable_timing=True) for _ in range(4))
             st.record(stream)
             stack_frame(N - 1)
-            stack_frame(N)
+            md.record(stream)
+            stack_frame(N, mid)
             en.record(stream)
             torch.cuda.synchronize()
-            rows.append({"N": N, "ms_per_frame": st.elapsed_time(en) / 2, "kv_bytes": n_soft * N * frame_kv,
-                         "arl2_state_bytes": n_arl2 * state_bytes})
+            row = {"N": N, "ms_per_frame": st.elapsed_time(en) / 2, "kv_bytes": n_soft * N * frame_kv,
+                   "arl2_state_bytes": n_arl2 * state_bytes}
+            if 0 < n_arl2 < layers:   # the second frame split at the last ARL2 layer
+                row["ms_arl2_layers"] = md.elapsed_time(mid)
+                row["ms_softmax_layers"] = mid.elapsed_time(en)
+            rows.append(row)
         out["shares"][f"{share:.2f}"] = {"arl2_layers": n_arl2, "softmax_layers": n_soft, "frames": rows}
     status = [c.status() for c in caches] + [lay.status() for lay in arl2s]
     out["status"] = max(status) if status else 0
