@@ -96,8 +96,7 @@ enum : int {
   kBarRecLoad = 35,   // the merge inputs of the CTA's last segment are staged in shared memory
   kBarLastPV = 36,    // the last P.V MMA of a staged merge's segment is done (V stages idle)
   kBarLastQK = 37,    // its last score MMA is done (K stages idle): staging may start
-  kBarVGo = 38,       // the CTA's first K tile landed: the V ring may start filling (completes once)
-  kNumBars = 39
+  kNumBars = 38
 };
 // Tiles at the (1 KiB-aligned) base of dynamic shared memory, then the control block.
 constexpr uint32_t kQOff = 0;
@@ -243,108 +242,187 @@ __device__ __forceinline__ int o_inter_tile(uint32_t t0, uint32_t n, bool last) 
 }
 __device__ __forceinline__ uint32_t sphase(uint32_t t) { return (t / kSBufs) & 1; }
 
-// K producer (kIsK) or V producer. Per segment: its key tiles, then, when the segment
-// holds key tile 0 of its query tile, the readout operand (Wq or S), all through this
-// producer's ring. The K producer also loads each segment's Q tile.
-template <bool kHybrid, bool kIsK>
-__device__ void producer(const Smem& sm, const CUtensorMap* tm_q, const CUtensorMap* tm_kv, const CUtensorMap* tm_rd,
-                         const QueryArgs& a, const Guard& g, bool lead) {
-  const int full0 = kIsK ? kBarKFull : kBarVFull, empty0 = kIsK ? kBarKEmpty : kBarVEmpty;
-  uint32_t nissued[kStages] = {0, 0, 0};
+// Producer (warp 0): per segment its Q tile, then per key tile the K tile and the V tile,
+// each through its own three-stage ring; when the segment holds key tile 0 of its query
+// tile, the readout operands follow its key tiles (Wq_h through the K ring, the bf16 state
+// copy S_h through the V ring).
+template <bool kHybrid>
+__device__ void producer(const Smem& sm, const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                         const CUtensorMap* tm_w, const CUtensorMap* tm_s, const QueryArgs& a, const Guard& g,
+                         bool lead) {
+  uint32_t nk[kStages] = {0, 0, 0}, nv[kStages] = {0, 0, 0};   // loads issued per stage
   uint32_t nseg = 0, ring = 0;
   Sched sch(a, static_cast<int>(blockIdx.x) - a.first_cta);
   Seg sg;
   bool ok = true;
-  bool waited = false;   // V producer: griddepcontrol.wait done before the first state load
-  auto slot_wait = [&](uint32_t gidx) -> bool {
+  bool waited = false;   // griddepcontrol.wait done before the first state load
+  auto slot_wait = [&](int empty0, uint32_t gidx) -> bool {
     return gidx < kStages || mbar_wait_warp(sm.bar(empty0 + ring_stage(gidx)), ring_phase(gidx - kStages), g);
   };
-  auto tile_addr = [&](int s) { return kIsK ? sm.k(s) : sm.v(s); };
   // q, k and v are this launch's activations: evict-first in L2, so they do not push out
   // what later launches reuse. (A key tile's other readers in this launch still hit L2: the
   // launch's working set is far below its size.)
   const uint64_t stream_policy = l2_evict_first_policy();
+  auto load_kv = [&](const CUtensorMap* map, uint32_t dst, int bar, const Seg& s, int j) {
+    if (lead) {
+      mbar_expect_tx(sm.bar(bar), kTileBytes);
+      for (int p = 0; p < 2; ++p)
+        tma_load_4d_hint(dst + p * kPanelBytes, map, sm.bar(bar), 64 * p, s.h, j * kRows, s.b, stream_policy);
+    }
+  };
+  auto load_op = [&](const CUtensorMap* map, uint32_t dst, int bar, int c2) {
+    if (lead) {
+      mbar_expect_tx(sm.bar(bar), kTileBytes);
+      for (int p = 0; p < 2; ++p) tma_load_3d(dst + p * kPanelBytes, map, sm.bar(bar), 64 * p, 0, c2);
+    }
+  };
   while (ok && sch.next(sg)) {
-    if (kIsK) {
-      // The next segment's Q tile goes to L2 now, so that its load (issued only once this
-      // segment's MMAs are done with Q) does not wait on HBM.
-      if (lead && sch.u < sch.u1)
-        for (int p = 0; p < 2; ++p) tma_prefetch_4d(tm_q, 64 * p, sch.h, sch.qt * kRows, sch.b);
-      if (nseg > 0 && !mbar_wait_warp(sm.bar(kBarQEmpty), (nseg - 1) & 1, g)) break;
-      if (lead) {
-        mbar_expect_tx(sm.bar(kBarQFull), kTileBytes);
-        for (int p = 0; p < 2; ++p)
-          tma_load_4d_hint(sm.q() + p * kPanelBytes, tm_q, sm.bar(kBarQFull), 64 * p, sg.h, sg.qt * kRows, sg.b,
-                           stream_policy);
-      }
+    // The next segment's Q tile goes to L2 now, so that its load (issued only once this
+    // segment's MMAs are done with Q) does not wait on HBM.
+    if (lead && sch.u < sch.u1)
+      for (int p = 0; p < 2; ++p) tma_prefetch_4d(tm_q, 64 * p, sch.h, sch.qt * kRows, sch.b);
+    if (nseg > 0 && !mbar_wait_warp(sm.bar(kBarQEmpty), (nseg - 1) & 1, g)) break;
+    if (lead) {
+      mbar_expect_tx(sm.bar(kBarQFull), kTileBytes);
+      for (int p = 0; p < 2; ++p)
+        tma_load_4d_hint(sm.q() + p * kPanelBytes, tm_q, sm.bar(kBarQFull), 64 * p, sg.h, sg.qt * kRows, sg.b,
+                         stream_policy);
     }
     ++nseg;
     for (int j = sg.kb; j < sg.ke; ++j, ++ring) {
-      // Start-up order: the first Q tile and first K tile go out alone (they gate the
-      // first score MMA); the rest of both rings fills once that K tile has landed. The K
-      // producer waits for it right after issuing it (phase 0 of K stage 0, which only it
-      // refills, so the phase cannot pass unseen) and then opens the V ring through a
-      // barrier that completes once. The V producer must not wait on the K stage barrier
-      // itself: if it started late, that barrier could already be in its third phase, and
-      // a parity wait for phase 0 would then wait for a phase that never comes.
-      if (!kIsK && ring == 0 && !mbar_wait_warp(sm.bar(kBarVGo), 0, g)) {
-        ok = false;
-        break;
-      }
-      if (!slot_wait(ring)) {
-        ok = false;
-        break;
-      }
       const int s = ring_stage(ring);
-      if (lead) {
-        mbar_expect_tx(sm.bar(full0 + s), kTileBytes);
-        for (int p = 0; p < 2; ++p)
-          tma_load_4d_hint(tile_addr(s) + p * kPanelBytes, tm_kv, sm.bar(full0 + s), 64 * p, sg.h, j * kRows, sg.b,
-                           stream_policy);
+      if (!slot_wait(kBarKEmpty, ring)) {
+        ok = false;
+        break;
       }
-      ++nissued[s];
-      if (kIsK && ring == 0) {
-        if (!mbar_wait_warp(sm.bar(kBarKFull), 0, g)) {
-          ok = false;
-          break;
-        }
-        if (lead) mbar_arrive(sm.bar(kBarVGo));
-        __syncwarp();
+      load_kv(tm_k, sm.k(s), kBarKFull + s, sg, j);
+      ++nk[s];
+      // Start-up order: the first Q tile and first K tile go out alone (they gate the
+      // first score MMA); the rest of both rings fills once that K tile has landed.
+      if (ring == 0 && !mbar_wait_warp(sm.bar(kBarKFull), 0, g)) {
+        ok = false;
+        break;
       }
+      if (!slot_wait(kBarVEmpty, ring)) {
+        ok = false;
+        break;
+      }
+      load_kv(tm_v, sm.v(s), kBarVFull + s, sg, j);
+      ++nv[s];
     }
     if (ok && kHybrid && sg.head) {
-      // The readout operand (Wq_h or the bf16 state copy S_h) follows the key tiles.
-      // S_{N-1} may be the output of the commit right before this launch: when this grid
-      // was launched as its programmatic dependent, that commit's writes are visible only
-      // after griddepcontrol.wait. The V producer waits once, before its first state load
-      // (a no-op for a normal launch, and long past by then behind another query).
-      if (!kIsK && !waited) {
+      // The readout operands follow the key tiles. S_{N-1} may be the output of the commit
+      // right before this launch: when this grid was launched as its programmatic
+      // dependent, that commit's writes are visible only after griddepcontrol.wait, which
+      // comes once, before the first state load (a no-op for a normal launch, and long past
+      // by then behind another query).
+      const int s = ring_stage(ring);
+      if (!slot_wait(kBarKEmpty, ring)) break;
+      load_op(tm_w, sm.k(s), kBarKFull + s, sg.h);
+      ++nk[s];
+      if (!waited) {
         griddep_wait();
         waited = true;
       }
-      if (!slot_wait(ring)) break;
-      const int s = ring_stage(ring);
-      const int c2 = kIsK ? sg.h : a.state_slot * a.B * a.H + sg.b * a.H + sg.h;
-      if (lead) {
-        mbar_expect_tx(sm.bar(full0 + s), kTileBytes);
-        for (int p = 0; p < 2; ++p) tma_load_3d(tile_addr(s) + p * kPanelBytes, tm_rd, sm.bar(full0 + s), 64 * p, 0, c2);
-      }
-      ++nissued[s];
+      if (!slot_wait(kBarVEmpty, ring)) break;
+      load_op(tm_s, sm.v(s), kBarVFull + s, a.state_slot * a.B * a.H + sg.b * a.H + sg.h);
+      ++nv[s];
       ++ring;
     }
   }
+  __syncwarp();
   // Every load issued must land before the CTA may exit (matters only after an abort).
-  if (kIsK && nseg > 0) mbar_wait_drain(sm.bar(kBarQFull), (nseg - 1) & 1);
-  for (int s = 0; s < kStages; ++s)
-    if (nissued[s]) mbar_wait_drain(sm.bar(full0 + s), (nissued[s] - 1) & 1);
+  if (nseg > 0) mbar_wait_drain(sm.bar(kBarQFull), (nseg - 1) & 1);
+  for (int s = 0; s < kStages; ++s) {
+    if (nk[s]) mbar_wait_drain(sm.bar(kBarKFull + s), (nk[s] - 1) & 1);
+    if (nv[s]) mbar_wait_drain(sm.bar(kBarVFull + s), (nv[s] - 1) & 1);
+  }
 }
 
-
+// Two MMA issuers, each a warp whose elected lane issues and commits; a tcgen05.mma issue
+// blocks until the tensor pipe takes the instruction, so with one issuer the pipe idled
+// whenever that thread waited on a barrier between its MMA groups. Here one warp issues
+// the score MMAs (and Q' = Q Wq_h), the other the P.V MMAs (and O_inter = Q' S_h): while
+// one waits, the other feeds the pipe. A commit tracks only its own thread's MMAs, so every
+// reuse of TMEM columns the other issuer's MMA reads is ordered by a barrier:
+//   - score tile t overwrites S buffer t % 3 once the P.V MMA of tile t - 3 (which read P
+//     from it) is done;
+//   - after a head segment (not the CTA's last), the next segment's first score tile goes
+//     into the buffer that held Q': it waits until the readout MMA is done (OFull); the
+//     buffer holding O_inter is next written once the epilogue has read it (OEmpty);
+//   - the P.V MMA of a segment's first tile overwrites O once the epilogue has read it.
+// S buffers cycle with the tile count: tile t in buffer t % 3. A segment holding key tile 0
+// puts Q' in the buffer of tile t0 + n and O_inter in that of the last tile (t0 + n - 1),
+// or, in the CTA's last segment, of tile t0 + n - 2 (see o_inter_tile).
+template <bool kHybrid>
+__device__ void score_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, const Guard& g, bool lead) {
+  constexpr uint32_t id_kk = idesc_bf16(128, 128, false, false);   // A, B K-major
+  constexpr uint32_t id_kmn = idesc_bf16(128, 128, false, true);   // A K-major, B MN-major
+  uint32_t nseg = 0, tile = 0, ring = 0;
+  int qp_buf = -1, x_buf = -1;        // buffers still read by the previous segment's readout / epilogue
+  uint32_t qp_phase = 0, x_phase = 0;
+  Sched sch(a, static_cast<int>(blockIdx.x) - a.first_cta);
+  Seg sg;
+  // Before an MMA writes the S buffer of tile t: the earlier readers of that buffer are done.
+  auto buffer_free = [&](uint32_t t) -> bool {
+    const int sb = sbuf(t);
+    if (t >= kSBufs && !mbar_wait_warp(sm.bar(kBarPVDone + sb), sphase(t - kSBufs), g)) return false;
+    if (sb == qp_buf) {
+      if (!mbar_wait_warp(sm.bar(kBarOFull), qp_phase, g)) return false;
+      qp_buf = -1;
+    }
+    if (sb == x_buf) {
+      if (!mbar_wait_warp(sm.bar(kBarOEmpty), x_phase, g)) return false;
+      x_buf = -1;
+    }
+    tc_fence_after();
+    return true;
+  };
+  while (sch.next(sg)) {
+    const bool rd = kHybrid && sg.head;
+    const uint32_t t0 = tile, n = sg.ke - sg.kb;
+    const bool staged = sg.head && !sg.tail && staged_merge(sch.last_nsegs);   // the CTA's last segment
+    if (!mbar_wait_warp(sm.bar(kBarQFull), nseg & 1, g)) return;
+    for (uint32_t i = 0; i < n; ++i) {
+      const uint32_t t = t0 + i, r = ring + i;
+      const int sb = sbuf(t), ks = ring_stage(r);
+      if (!buffer_free(t) || !mbar_wait_warp(sm.bar(kBarKFull + ks), ring_phase(r), g)) return;
+      tc_fence_after();
+      if (lead) {
+        mma8_ss<false, false>(tmem + 128u * sb, desc_kmajor(sm.q(), 0), desc_kmajor(sm.k(ks), 0), id_kk, 0u);
+        mma_commit(sm.bar(kBarKEmpty + ks));
+        mma_commit(sm.bar(kBarSFull + sb));
+      }
+    }
+    if (lead && staged) mma_commit(sm.bar(kBarLastQK));   // K stages other than the readout's are idle
+    if (rd) {
+      // Q' = Q Wq_h into the S buffer of tile t0 + n (Wq_h in the K ring after the key tiles).
+      const int rs = ring_stage(ring + n);
+      if (!buffer_free(t0 + n) || !mbar_wait_warp(sm.bar(kBarKFull + rs), ring_phase(ring + n), g)) return;
+      tc_fence_after();
+      if (lead) {
+        mma8_ss<false, true>(tmem + 128u * sbuf(t0 + n), desc_kmajor(sm.q(), 0), desc_mnmajor(sm.k(rs), 0), id_kmn,
+                             0u);
+        mma_commit(sm.bar(kBarKEmpty + rs));
+        mma_commit(sm.bar(kBarQEmpty));
+        mma_commit(sm.bar(kBarQp));
+      }
+      qp_buf = sbuf(t0 + n);
+      qp_phase = nseg & 1;
+      x_buf = o_inter_tile(t0, n, sg.last);
+      x_phase = nseg & 1;
+    } else if (lead) {
+      mma_commit(sm.bar(kBarQEmpty));
+    }
+    tile += n;
+    ring += n + (rd ? 1u : 0u);
+    ++nseg;
+  }
+}
 
 template <bool kHybrid>
-__device__ void mma_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, const Guard& g, bool lead) {
-  constexpr uint32_t id_kk = idesc_bf16(128, 128, false, false);   // A, B K-major
-  constexpr uint32_t id_kmn = idesc_bf16(128, 128, false, true);   // A K-major (smem or TMEM), B MN-major
+__device__ void pv_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, const Guard& g, bool lead) {
+  constexpr uint32_t id_kmn = idesc_bf16(128, 128, false, true);   // A K-major (TMEM), B MN-major
   const uint32_t tO = tmem + kColO;
   // A operands in TMEM, by K step of 16: P packed by the softmax's .16x128b stores (its
   // 64 words in order), and Q' packed in place by column halves (words 0-31 and 64-95).
@@ -353,91 +431,31 @@ __device__ void mma_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, co
   uint32_t nseg = 0, nhead = 0, tile = 0, ring = 0;
   Sched sch(a, static_cast<int>(blockIdx.x) - a.first_cta);
   Seg sg;
-  // Score tile t (S buffer t % 3) from the K tile in ring slot r. The buffer's previous
-  // tile (t - 3) was consumed by a P.V MMA issued earlier, so in-order execution keeps it.
-  auto issue_qk = [&](uint32_t t, uint32_t r) -> bool {
-    const int sb = sbuf(t), ks = ring_stage(r);
-    if (!mbar_wait_warp(sm.bar(kBarKFull + ks), ring_phase(r), g)) return false;
-    tc_fence_after();
-    const uint32_t tS = tmem + 128u * sb;
-    if (lead) {
-      mma8_ss<false, false>(tS, desc_kmajor(sm.q(), 0), desc_kmajor(sm.k(ks), 0), id_kk, 0u);
-      mma_commit(sm.bar(kBarKEmpty + ks));
-      mma_commit(sm.bar(kBarSFull + sb));
-    }
-    return true;
-  };
-  // First readout MMA, Q' = Q Wq_h into the S buffer of tile t0 + n (Y). Issued right
-  // after the segment's last score MMA (never before the O wait, as Y may be the buffer
-  // of the previous segment's O_inter): Y last held tile t0 + n - 3, whose P.V MMA is
-  // already queued, and Q is free once this MMA is done.
-  auto issue_qwq = [&](uint32_t t0, uint32_t n, uint32_t r_rd) -> bool {
-    const int rs = ring_stage(r_rd);
-    if (!mbar_wait_warp(sm.bar(kBarKFull + rs), ring_phase(r_rd), g)) return false;
-    tc_fence_after();
-    if (lead) {
-      mma8_ss<false, true>(tmem + 128u * sbuf(t0 + n), desc_kmajor(sm.q(), 0), desc_mnmajor(sm.k(rs), 0), id_kmn,
-                           0u);
-      mma_commit(sm.bar(kBarKEmpty + rs));
-      mma_commit(sm.bar(kBarQEmpty));
-      mma_commit(sm.bar(kBarQp));
-    }
-    return true;
-  };
   while (sch.next(sg)) {
     const bool rd = kHybrid && sg.head;
     const uint32_t t0 = tile, n = sg.ke - sg.kb;
-    bool staged = false;   // a staged merge: the K, then V, stages it uses are signalled idle
-    if (sg.head && !sg.tail) staged = staged_merge(sch.last_nsegs);   // the CTA's last segment
-    const uint32_t r0 = ring, r_rd = ring + n;   // first key tile's ring slot, the readout operands' slot
-    // Score tiles issued before the P.V loop: two. Afterwards the scores of tile t + 2 are
-    // issued right behind the P.V MMA of tile t: they go to the buffer whose P was read by
-    // the P.V MMA before that one, so adjacent MMA groups never touch the same TMEM columns
-    // (an MMA that overwrites columns the MMA just ahead of it still reads stalls the pipe).
-    const uint32_t npre = min(n, 2u);
-    if (!mbar_wait_warp(sm.bar(kBarQFull), nseg & 1, g)) return;
-    tc_fence_after();
-    for (uint32_t i = 0; i < npre; ++i)
-      if (!issue_qk(t0 + i, r0 + i)) return;
-    // O (and the previous segment's O_inter, in the buffer of tile t0 + 2) must have been
-    // read before either is rewritten.
+    const bool staged = sg.head && !sg.tail && staged_merge(sch.last_nsegs);
+    // O (and the previous segment's O_inter) must have been read before O is rewritten.
     if (nseg > 0 && !mbar_wait_warp(sm.bar(kBarOEmpty), (nseg - 1) & 1, g)) return;
-    tc_fence_after();
-    if (n <= npre) {   // every score tile is issued
-      if (lead && staged) mma_commit(sm.bar(kBarLastQK));
-      if (rd && !issue_qwq(t0, n, r_rd)) return;
-      if (lead && !rd) mma_commit(sm.bar(kBarQEmpty));
-    }
-    const uint32_t nissued = npre;   // score tiles issued ahead of the P.V loop
     for (uint32_t i = 0; i < n; ++i) {
-      const uint32_t t = t0 + i, r = r0 + i;
+      const uint32_t t = t0 + i, r = ring + i;
       const int sb = sbuf(t), vs = ring_stage(r);
       if (!mbar_wait_warp(sm.bar(kBarPFull + sb), sphase(t), g)) return;
       if (!mbar_wait_warp(sm.bar(kBarVFull + vs), ring_phase(r), g)) return;
       tc_fence_after();
-      const uint32_t tP = tmem + 128u * sb;
       if (lead) {
-        mma8_ts(tO, tP, kPackedP, desc_mnmajor(sm.v(vs), 0), id_kmn, i > 0 ? 1u : 0u);
+        mma8_ts(tO, tmem + 128u * sb, kPackedP, desc_mnmajor(sm.v(vs), 0), id_kmn, i > 0 ? 1u : 0u);
         mma_commit(sm.bar(kBarPVDone + sb));
         mma_commit(sm.bar(kBarVEmpty + vs));
       }
-      if (i + nissued < n) {
-        if (!issue_qk(t + nissued, r + nissued)) return;
-        if (i + nissued + 1 == n) {   // that was the last score tile
-          if (lead && staged) mma_commit(sm.bar(kBarLastQK));
-          if (rd && !issue_qwq(t0, n, r_rd)) return;
-          if (lead && !rd) mma_commit(sm.bar(kBarQEmpty));
-        }
-      }
     }
-    if (lead && staged) mma_commit(sm.bar(kBarLastPV));
+    if (lead && staged) mma_commit(sm.bar(kBarLastPV));   // V stages other than the readout's are idle
     if (rd) {
-      // Second readout MMA, after the last P.V: O_inter = Q' S_{N-1}, with Q' packed to
-      // bf16 in place by the softmax threads, into X (see o_inter_tile).
+      // O_inter = Q' S_{N-1}, with Q' packed to bf16 in place by the softmax threads.
       const uint32_t tY = tmem + 128u * sbuf(t0 + n), tX = tmem + 128u * o_inter_tile(t0, n, sg.last);
-      const int rs = ring_stage(r_rd);
+      const int rs = ring_stage(ring + n);
       if (!mbar_wait_warp(sm.bar(kBarQpReady), nhead & 1, g)) return;
-      if (!mbar_wait_warp(sm.bar(kBarVFull + rs), ring_phase(r_rd), g)) return;
+      if (!mbar_wait_warp(sm.bar(kBarVFull + rs), ring_phase(ring + n), g)) return;
       tc_fence_after();
       if (lead) {
         mma8_ts(tX, tY, kPackedQ, desc_mnmajor(sm.v(rs), 0), id_kmn, 0u);
@@ -447,7 +465,7 @@ __device__ void mma_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, co
     }
     if (lead) mma_commit(sm.bar(kBarOFull));   // every MMA of the segment, the readout included
     tile += n;
-    ring = r0 + n + (rd ? 1u : 0u);
+    ring += n + (rd ? 1u : 0u);
     ++nseg;
   }
 }
@@ -460,9 +478,9 @@ __device__ void mma_issuer(const Smem& sm, uint32_t tmem, const QueryArgs& a, co
 // (t / 4) + 8h, column 64p + 8c + 2 (t % 4) + j. Row statistics need only shuffles among
 // those four lanes, never another warp.
 
-// Row maxima (raw units) of this thread's two rows over its 32 columns each, with keys at
-// or beyond `valid` masked to -inf, then over the row's four threads.
-__device__ __forceinline__ void row_max2(uint32_t (&sv)[2][32], int g4, int valid, float (&mx)[2]) {
+// Maxima (raw units) of this thread's two rows over its own 32 columns each, with keys at or
+// beyond `valid` masked to -inf. The row's other three threads hold the rest of the row.
+__device__ __forceinline__ void thread_max2(uint32_t (&sv)[2][32], int g4, int valid, float (&mx)[2]) {
   if (valid < kRows) {
 #pragma unroll
     for (int p = 0; p < 2; ++p)
@@ -482,6 +500,9 @@ __device__ __forceinline__ void row_max2(uint32_t (&sv)[2][32], int g4, int vali
         m4[c & 1] = fmax3(m4[c & 1], __uint_as_float(sv[p][4 * c + 2 * h]), __uint_as_float(sv[p][4 * c + 2 * h + 1]));
     mx[h] = fmaxf(m4[0], m4[1]);
   }
+}
+// The maxima over each row's four threads (consecutive lanes).
+__device__ __forceinline__ void row_reduce_max2(float (&mx)[2]) {
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
@@ -793,7 +814,7 @@ __device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const 
   const int quarter = warp & 3;
   // In the epilogue and the Q' packing a thread owns row r (its TMEM lane) and the column
   // half `half`; in the tile loop the same warp owns 16 whole rows of its quarter instead
-  // (rows 16 half .. 16 half + 15; see row_max2).
+  // (rows 16 half .. 16 half + 15; see thread_max2).
   const int half = (warp - 4) >> 2;
   const uint32_t r = quarter * 32 + (threadIdx.x & 31);     // tile row == TMEM lane
   const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
@@ -826,19 +847,31 @@ __device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const 
       const int valid = a.kv_len - (sg.kb + static_cast<int>(i)) * kRows;   // >= 1
       uint32_t sv[2][32];
       tmem_ld16dp256_x8x2_wait(tS, sv[0], tS + 64u, sv[1]);
+      // The running max changes only on a segment's first tile or when a row's max exceeds
+      // it by more than the threshold. Each thread first checks its own columns; only if
+      // one of the warp's threads sees such a column do the rows' four threads combine
+      // their maxima (scaling by the positive scale_log2 commutes with the max, so the
+      // rows get exactly the maxima the full reduction gives).
       float mt[2];
-      row_max2(sv, g4, valid, mt);
-      float m_new[2];
+      thread_max2(sv, g4, valid, mt);
+      float m_new[2] = {m[0], m[1]};
       bool rescale[2] = {false, false};
+      bool raise = i == 0;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         mt[h] *= a.scale_log2;
-        m_new[h] = m[h];
-        if (i == 0) {
-          m_new[h] = mt[h];
-        } else if (mt[h] > m[h] + kRescaleThreshold) {
-          m_new[h] = mt[h];
-          rescale[h] = true;
+        raise = raise || mt[h] > m[h] + kRescaleThreshold;
+      }
+      if (__any_sync(0xffffffffu, raise)) {
+        row_reduce_max2(mt);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (i == 0) {
+            m_new[h] = mt[h];
+          } else if (mt[h] > m[h] + kRescaleThreshold) {
+            m_new[h] = mt[h];
+            rescale[h] = true;
+          }
         }
       }
       if (__any_sync(0xffffffffu, rescale[0] || rescale[1])) {
@@ -970,7 +1003,7 @@ __device__ __forceinline__ void query_cta(const CUtensorMap& tm_q, const CUtenso
     mbar_init(sm.bar(kBarQpReady), kSoftmaxWarps);
     mbar_init(sm.bar(kBarOFull), 1);
     mbar_init(sm.bar(kBarOEmpty), kSoftmaxWarps);
-    mbar_init(sm.bar(kBarFinal), 1);
+    mbar_init(sm.bar(kBarFinal), 2);   // one commit per MMA issuer
     mbar_init(sm.bar(kBarGroup), kSoftmaxWarps);
     for (int q = 0; q < 4; ++q) mbar_init(sm.bar(kBarPair + q), 2);   // one arrival per warp
     mbar_init(sm.bar(kBarNever), 1);
@@ -978,18 +1011,17 @@ __device__ __forceinline__ void query_cta(const CUtensorMap& tm_q, const CUtenso
     mbar_init(sm.bar(kBarRecLoad), 1);
     mbar_init(sm.bar(kBarLastPV), 1);
     mbar_init(sm.bar(kBarLastQK), 1);
-    mbar_init(sm.bar(kBarVGo), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
-    if (kHybrid) prefetch_tmap(&tm_w);
-  }
-  if (warp == 2 && lane == 0) {
     prefetch_tmap(&tm_v);
-    if (kHybrid) prefetch_tmap(&tm_s);
+    if (kHybrid) {
+      prefetch_tmap(&tm_w);
+      prefetch_tmap(&tm_s);
+    }
   }
   if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
   tc_fence_before();
@@ -1003,20 +1035,21 @@ __device__ __forceinline__ void query_cta(const CUtensorMap& tm_q, const CUtenso
   // output may be this grid's) and before its first load of the state (a commit's output).
   griddep_launch_dependents();
 
-  // Producers and the MMA issuer run warp-wide (uniform control flow and waits); one
+  // The producer and the MMA issuers run warp-wide (uniform control flow and waits); one
   // elected lane issues each TMA copy, MMA and commit.
   if (warp == 0) {
-    producer<kHybrid, true>(sm, &tm_q, &tm_k, &tm_w, a, g, elect_one());
-  } else if (warp == 1) {
+    producer<kHybrid>(sm, &tm_q, &tm_k, &tm_v, &tm_w, &tm_s, a, g, elect_one());
+  } else if (warp == 1 || warp == 2) {
     const bool lead = elect_one();
-    mma_issuer<kHybrid>(sm, tmem, a, g, lead);
-    if (lead) mma_commit(sm.bar(kBarFinal));   // arrives once every MMA issued above has finished
+    if (warp == 1)
+      score_issuer<kHybrid>(sm, tmem, a, g, lead);
+    else
+      pv_issuer<kHybrid>(sm, tmem, a, g, lead);
+    if (lead) mma_commit(sm.bar(kBarFinal));   // arrives once every MMA this warp issued has finished
     __syncwarp();
-  } else if (warp == 2) {
-    producer<kHybrid, false>(sm, &tm_q, &tm_v, &tm_s, a, g, elect_one());
   } else if (warp == 3) {
     publisher<kHybrid>(sm, a, g);
-  } else if (warp >= 4) {
+  } else {
     softmax_role<kHybrid>(sm, ctl_ptr, tmem, a, warp, &tm_o, g);
   }
 
