@@ -26,11 +26,12 @@
 // Scratch records are column-quad-major, so every scratch access of a warp is coalesced.
 //
 // Roles (384 threads, one CTA per SM):
-//   warp 0      K producer: per segment the Q tile, then K tiles into a three-stage ring.
-//               When a segment starts a tile, Wq_h first goes through the ring like a tile.
-//   warp 1      TMEM owner; lane 0 issues every tcgen05.mma and commit.
-//   warp 2      V producer: V tiles into a three-stage ring. When a segment starts a tile,
-//               the bf16 state copy S_h goes first, through the ring.
+//   warp 0      producer: per segment the Q tile, then per key tile its K and V tiles,
+//               each into a three-stage ring. When a segment starts a tile, Wq_h follows
+//               its key tiles through the K ring and the bf16 state copy S_h through the V
+//               ring.
+//   warp 1      TMEM owner and score issuer: one lane issues the score MMAs (and Q Wq_h).
+//   warp 2      P.V issuer: one lane issues the P.V MMAs (and the readout Q' S_h).
 //   warp 3      publisher: raises the flag of each partial record the CTA stores.
 //   warps 4-11  two softmax warpgroups. Warps w and w+4 share a TMEM lane quarter (the
 //               same SM sub-partition). In the tile loop, w takes the quarter's first 16
@@ -42,17 +43,16 @@
 //               also write outputs and partial records. Warp 3 stages the records a merge
 //               reads.
 // TMEM (512 columns):
-//   - cols 0, 128, 256: three S tiles. The score MMA of tile t+2 is queued right behind
-//     the P.V MMA of tile t and writes the buffer last read two MMA groups earlier, so no
-//     MMA group overwrites TMEM columns that the group just ahead of it still reads (that
-//     stalls the tensor pipe). P (bf16 pairs) overwrites the first 64 columns of its own S
-//     tile, keys in order, and feeds the P.V MMA straight from TMEM.
+//   - cols 0, 128, 256: three S tiles, tile t in buffer t % 3. The score MMA of tile t
+//     waits for the P.V MMA of tile t - 3, which read P from the same buffer. P (bf16
+//     pairs) overwrites the first 64 columns of its own S tile, keys in order, and feeds
+//     the P.V MMA straight from TMEM.
 //   - col 384: O.
-//   - Readout, after the last P.V MMA of a segment holding key tile 0: Q' = Q Wq_h goes to
-//     the S tile of tile t0 + n (fp32, then packed in place to bf16 like P), and
-//     O_inter = Q' S_h to the S tile of the segment's last tile. The next segment issues
-//     its first two score tiles into neither of them before its O wait, and its third
-//     (into O_inter's tile) only after that wait.
+//   - Readout of a segment holding key tile 0: after its last score MMA, Q' = Q Wq_h goes
+//     to the S tile of tile t0 + n (fp32, then packed in place to bf16 like P); after its
+//     last P.V MMA, O_inter = Q' S_h goes to the S tile of the segment's last tile. The
+//     next segment's score MMAs write the first of these once the readout is done and the
+//     second once the epilogue has read O_inter.
 // Shared memory: Q | K0 K1 K2 | V0 V1 V2 (32 KiB tiles) from its 1 KiB-aligned base, then a
 // small control block (mbarriers, flags, the row-statistics exchange slots).
 //
