@@ -527,6 +527,7 @@ __device__ __forceinline__ void commit_cta(const CUtensorMap& tm_k, const CUtens
   } else if (warp >= kFirstEpiWarp && warp < kFirstEpiWarp + kEpiWarps) {
     epilogue_role(sm, tmem, a, cta, warp, lane, last_flag, warp_sums, g);
   }
+  __syncwarp();   // roles end in per-lane drains: one arrival per warp at the barrier
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -305,6 +305,7 @@ __global__ void __launch_bounds__(kThreadsC, 1)
     const bool ok = row_role(sm, tmem, a, c0, nc, h, b, warp, lane, warp_sums, g);
     if (!__all_sync(0xffffffffu, ok) && lane == 0) *rows_failed = 1;
   }
+  __syncwarp();   // the producer ends in per-lane drains: one arrival per warp at the barrier
   tc_fence_before();
   __syncthreads();
   const int d = rd.d;

@@ -88,7 +88,7 @@ enum : int {
   kBarQpReady = 24,   // Q' is packed to bf16 (per-warp arrivals)
   kBarOFull = 25,     // the segment's MMAs (its readout included) are all done
   kBarOEmpty = 26,    // the segment's O and O_inter were read (per-warp arrivals)
-  kBarFinal = 27,
+  kBarFinal = 27,     // every MMA done and every softmax warp finished with TMEM (before it is freed)
   kBarGroup = 28,     // bounded rendezvous of the softmax threads (per-warp arrivals)
   kBarPair = 29,      // +row quarter (4): the quarter's two warps stored their rows' max and sum
   kBarNever = 33,     // never signalled: target of the failure-detection test hook
@@ -579,24 +579,17 @@ __device__ __forceinline__ void merge_rows(const QueryArgs& a, const Seg& sg, ui
     if constexpr (kStaged) return st4[(kKOff + (q < 16 ? k1 : k2) * kTileBytes) / 16 + (q & 15) * kRows + r];
     else return __ldcg(quad_ptr(a.part_o, slot0 + s, q, r));
   };
-  float ws[kMaxSegs];
+  // Weights of the other records. The staged merge has exactly one; otherwise the loops
+  // over records run as loops (not unrolled): this code runs once per query tile, so its
+  // size (instruction fetches from L2 on a cold instruction cache) costs more than its
+  // arithmetic, and most tiles have no other record at all.
   float M = m;
-#pragma unroll
-  for (int s = 1; s < kMaxSegs; ++s) {
-    if (s < nsegs) {
-      ws[s] = rec_m(s);
-      M = fmaxf(M, ws[s]);
-    }
-  }
+#pragma unroll 1
+  for (int s = 1; s < nsegs; ++s) M = fmaxf(M, rec_m(s));
   const float w_own = ex2_approx(m - M);
   float L = w_own * l_row;
-#pragma unroll
-  for (int s = 1; s < kMaxSegs; ++s) {
-    if (s < nsegs) {
-      ws[s] = ex2_approx(ws[s] - M);
-      L += ws[s] * rec_l(s);
-    }
-  }
+#pragma unroll 1
+  for (int s = 1; s < nsegs; ++s) L += ex2_approx(rec_m(s) - M) * rec_l(s);
   const float inv_L = 1.f / L;
   const int t_row = sg.qt * kRows + static_cast<int>(r);
   const bool row_ok = t_row < a.T;
@@ -604,26 +597,27 @@ __device__ __forceinline__ void merge_rows(const QueryArgs& a, const Seg& sg, ui
   // Four passes of 16 columns: the other records first, then the TMEM loads (O, and
   // O_inter for the layer) with their wait right behind them. No code sits between a TMEM
   // load and its wait: the load's destination registers are undefined until the wait, and
-  // anything in between gives the compiler room to copy them early.
-#pragma unroll
+  // anything in between gives the compiler room to copy them early. The passes run as a
+  // loop: this code runs once per tile, on a cold instruction cache, where its size costs
+  // more than the loop.
+#pragma unroll 1
   for (int c = 0; c < 4; ++c) {
     if (16 * c >= ncols) break;
     float4 acc[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+    for (int s = 1; s < nsegs; ++s) {
+      const float ws = ex2_approx(rec_m(s) - M);
+      float4 v[4];
 #pragma unroll
-    for (int s = 1; s < kMaxSegs; ++s) {
-      if (s < nsegs) {
-        float4 v[4];
+      for (int q = 0; q < 4; ++q) v[q] = rec_o(s, q0 + 4 * c + q);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) v[q] = rec_o(s, q0 + 4 * c + q);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          acc[q].x += ws[s] * v[q].x;
-          acc[q].y += ws[s] * v[q].y;
-          acc[q].z += ws[s] * v[q].z;
-          acc[q].w += ws[s] * v[q].w;
-        }
+      for (int q = 0; q < 4; ++q) {
+        acc[q].x += ws * v[q].x;
+        acc[q].y += ws * v[q].y;
+        acc[q].z += ws * v[q].z;
+        acc[q].w += ws * v[q].w;
       }
     }
     uint32_t ov[16], xv[16];
@@ -688,7 +682,7 @@ __device__ __noinline__ int segment_epilogue(const Smem sm, const QueryArgs& a, 
   const size_t slot0 = static_cast<size_t>(sg.Q) * a.max_segs;
   if (!sg.head) {   // the CTA's first segment
     const size_t slot = slot0 + first_rec;
-#pragma unroll
+#pragma unroll 1
     for (int c = 0; c < 4; ++c) {
       if (16 * c >= ncols) break;
       uint32_t ov[16];
@@ -914,7 +908,7 @@ __device__ void softmax_role(const Smem& sm, uint8_t* ctl, uint32_t tmem, const 
       tc_fence_after();
       // Two rounds of 32 columns; round h packs into columns c0 + 16h .. c0 + 16h + 15,
       // which round h has already read (round 1 writes only what round 0 read).
-#pragma unroll
+#pragma unroll 1
       for (int h = 0; h < 2; ++h) {
         uint32_t x0[16], x1[16], pk[16];
         tmem_ld16x2_wait(tY + c0 + 32u * h, x0, tY + c0 + 32u * h + 16u, x1);
@@ -1003,7 +997,7 @@ __device__ __forceinline__ void query_cta(const CUtensorMap& tm_q, const CUtenso
     mbar_init(sm.bar(kBarQpReady), kSoftmaxWarps);
     mbar_init(sm.bar(kBarOFull), 1);
     mbar_init(sm.bar(kBarOEmpty), kSoftmaxWarps);
-    mbar_init(sm.bar(kBarFinal), 2);   // one commit per MMA issuer
+    mbar_init(sm.bar(kBarFinal), 2 + kSoftmaxWarps);   // a commit per MMA issuer, an arrival per softmax warp
     mbar_init(sm.bar(kBarGroup), kSoftmaxWarps);
     for (int q = 0; q < 4; ++q) mbar_init(sm.bar(kBarPair + q), 2);   // one arrival per warp
     mbar_init(sm.bar(kBarNever), 1);
@@ -1051,8 +1045,15 @@ __device__ __forceinline__ void query_cta(const CUtensorMap& tm_q, const CUtenso
     publisher<kHybrid>(sm, a, g);
   } else {
     softmax_role<kHybrid>(sm, ctl_ptr, tmem, a, warp, &tm_o, g);
+    // Every TMEM access of this warp is done (whichever way the role ended): TMEM may be
+    // freed once both MMA issuers and all eight softmax warps have arrived.
+    tc_fence_before();
+    warp_arrive(sm.bar(kBarFinal));
   }
 
+  // The roles end in per-lane waits (drains), so a warp may arrive here split: reconverge
+  // it first, or its parts would count as several arrivals at the CTA barrier.
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -158,6 +158,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
       }
     }
   }
+  __syncwarp();   // rows past T and the producer's drains split warps: one arrival per warp
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
