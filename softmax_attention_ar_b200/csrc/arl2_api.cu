@@ -277,6 +277,7 @@ void set_plan(arl2::QueryArgs* a, const arl2::QueryPlan& p, float* scratch, int*
   a->units = p.units;
   a->num_ctas = p.num_ctas;
   a->max_segs = p.max_segs;
+  a->head_w = p.head_w;
   const size_t slots = static_cast<size_t>(p.qtiles) * p.max_segs;
   a->part_o = scratch;
   a->part_ml = scratch + slots * 128 * 128;

@@ -28,17 +28,37 @@ struct QueryArgs {
   int num_ctas;           // CTAs of the split
   int first_cta;          // the split's CTAs are blockIdx.x in [first_cta, first_cta + num_ctas)
   int max_segs;           // CTAs sharing one query tile, at most
+  int head_w;             // extra weight of a query tile's key tile 0 in the split (quarter units)
   float* part_o;          // [qtiles * max_segs][32 column quads][128 rows] float4: partial O accumulators
   float* part_ml;         // [qtiles * max_segs, 2, 128] running max (log2 units) and sum
   int* flags;             // [qtiles * max_segs] record-published flags, set to the launch's epoch
   int epoch;              // nonzero, different from the previous launch on the same flags
 };
 
-// The stream-K split of one query launch: CTA c takes units [c*U/P, (c+1)*U/P).
+// The stream-K split of one query launch. Units are weighted: 4 for a (query tile, key tile)
+// pair, 4 + head_w for key tile 0, whose segment also computes the readout and finishes the
+// tile; CTA c takes the units whose weighted start lies in [c W / P, (c + 1) W / P), W the
+// total weight (see split_start).
 struct QueryPlan {
-  int nq, nkv, num_ctas, max_segs;
+  int nq, nkv, num_ctas, max_segs, head_w;
   long long units, qtiles;
 };
+// Weighted split of `units` (query tile, key tile) units, nkv per query tile, over P CTAs: the
+// first unit of CTA c (c = P gives units), and the CTA that holds unit u. Host and device
+// share these two functions, so the plan and the kernels agree on every boundary.
+__host__ __device__ inline long long split_start(long long c, long long units, int nkv, int head_w, int P) {
+  const long long wt = 4ll * nkv + head_w;   // weight of one query tile
+  const long long wc = c * ((units / nkv) * wt) / P;
+  const long long k = wc / wt, r = wc - k * wt;
+  if (r == 0) return k * nkv;
+  const long long j = r > head_w ? (r - head_w + 3) / 4 : 1;   // W(k nkv + j) = k wt + head_w + 4 j >= wc
+  return k * nkv + (j > 1 ? j : 1);
+}
+__host__ __device__ inline int split_owner(long long u, long long units, int nkv, int head_w, int P) {
+  const long long wtot = (units / nkv) * (4ll * nkv + head_w);
+  const long long w = 4 * u + static_cast<long long>(head_w) * ((u + nkv - 1) / nkv);   // weight before unit u
+  return static_cast<int>(((w + 1) * P - 1) / wtot);
+}
 QueryPlan plan_query(int B, int H, int T, int kv_len, int num_sms);
 size_t query_scratch_floats(const QueryPlan& p);   // part_o + part_ml
 size_t query_flag_count(const QueryPlan& p);       // flags

@@ -35,13 +35,19 @@ QueryPlan plan_query(int B, int H, int T, int kv_len, int num_sms) {
   p.qtiles = static_cast<long long>(B) * H * p.nq;
   long long ctas = std::max<long long>(1, std::min<long long>(num_sms, p.units));
   while (true) {
+    // Key tile 0 of a query tile weighs more than the others: its segment also computes the
+    // readout and finishes the tile (merge, normalisation, store), which costs about as much
+    // as two and a half key tiles on the B200. The weight applies only while every CTA's
+    // weighted share spans a whole unit of the largest weight, so no range is empty.
+    const long long wtot = p.qtiles * (4ll * p.nkv + kHeadWeight);
+    p.head_w = wtot / ctas >= 4 + kHeadWeight + 1 ? kHeadWeight : 0;
     // Largest number of CTAs sharing one query tile under this grid.
     int worst = 1;
     for (long long Q = 0; Q < p.qtiles; ++Q) {
       const long long first = Q * p.nkv, last = first + p.nkv - 1;
-      const long long c0 = ((first + 1) * ctas - 1) / p.units;
-      const long long c1 = ((last + 1) * ctas - 1) / p.units;
-      worst = std::max<int>(worst, static_cast<int>(c1 - c0 + 1));
+      const int c0 = split_owner(first, p.units, p.nkv, p.head_w, static_cast<int>(ctas));
+      const int c1 = split_owner(last, p.units, p.nkv, p.head_w, static_cast<int>(ctas));
+      worst = std::max(worst, c1 - c0 + 1);
     }
     if (worst <= kMaxSegs || ctas == 1) {
       p.max_segs = worst;

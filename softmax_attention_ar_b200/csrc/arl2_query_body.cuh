@@ -116,6 +116,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 384;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kMaxSegs = 8;                // the host plan keeps segments per query tile at or below this
+constexpr int kHeadWeight = 10;            // key tile 0's extra split weight, quarter units (see QueryPlan)
 // Staged merge: a query tile split in two segments is finished by its head segment (the
 // CTA's last) from a shared-memory copy of the other record, taken while the head's last
 // tiles are still in flight. The readout still reads Q, and Wq_h and S_h in ring stage ws of
@@ -170,7 +171,7 @@ struct Seg {
 
 // The CTA whose unit range holds unit u.
 __device__ __forceinline__ int owner(long long u, const QueryArgs& a) {
-  return static_cast<int>(((u + 1) * a.num_ctas - 1) / a.units);
+  return split_owner(u, a.units, a.nkv, a.head_w, a.num_ctas);
 }
 
 // A CTA's walk over its unit range, one segment at a time. The divisions happen once, when
@@ -186,8 +187,8 @@ struct Sched {
   int first_rec;         // the first segment's record slot within its tile (this CTA - the tile's first CTA)
   int last_nsegs;        // CTAs sharing the last segment's tile (counted from this one)
   __device__ Sched(const QueryArgs& a, int c) : nq(a.nq), nkv(a.nkv), H(a.H) {
-    u = static_cast<long long>(c) * a.units / a.num_ctas;
-    u1 = static_cast<long long>(c + 1) * a.units / a.num_ctas;
+    u = split_start(c, a.units, a.nkv, a.head_w, a.num_ctas);
+    u1 = split_start(c + 1, a.units, a.nkv, a.head_w, a.num_ctas);
     Q = static_cast<int>(u / nkv);
     kb = static_cast<int>(u % nkv);
     const int bh = Q / nq;
