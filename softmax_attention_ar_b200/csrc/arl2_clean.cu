@@ -64,7 +64,7 @@ enum : int {
   kBarR = 13,         // R bf16 over the V tile (one arrival per row warp)
   kBarU = 14,         // every MMA of the segment is done: U complete, its W, S and tiles free
   kBarUFree = 15,     // the segment's epilogue has read U out of TMEM (one arrival per epilogue warp)
-  kBarFinal = 16,     // every MMA of the CTA is done (drain before TMEM is freed)
+  kBarFinal = 16,     // every MMA done and every row and epilogue warp finished with TMEM (before it is freed)
   kBarEpi = 17,       // rendezvous of the epilogue warps (one arrival per epilogue warp)
   kBarASum = 18,      // the segment's alpha sums are in shared memory (one arrival per row warp)
   kNumBars = 19
@@ -493,6 +493,7 @@ __device__ __forceinline__ void commit_cta(const CUtensorMap& tm_k, const CUtens
     for (int i = 0; i < kNumBars; ++i)
       mbar_init(sm.bar(i), (i == kBarKn || i == kBarR || i == kBarASum) ? kRowWarps
                            : (i == kBarUFree || i == kBarEpi)              ? kEpiWarps
+                           : i == kBarFinal                                ? 1 + kRowWarps + kEpiWarps
                                                                            : 1);
     *abort_flag = 0;
     *last_flag = 0;
@@ -524,8 +525,12 @@ __device__ __forceinline__ void commit_cta(const CUtensorMap& tm_k, const CUtens
     __syncwarp();
   } else if (warp >= kFirstRowWarp && warp < kFirstRowWarp + kRowWarps) {
     row_role(sm, tmem, a, cta, warp, lane, warp_sums, g);
+    tc_fence_before();
+    warp_arrive(sm.bar(kBarFinal));   // this warp's TMEM accesses are done, however the role ended
   } else if (warp >= kFirstEpiWarp && warp < kFirstEpiWarp + kEpiWarps) {
     epilogue_role(sm, tmem, a, cta, warp, lane, last_flag, warp_sums, g);
+    tc_fence_before();
+    warp_arrive(sm.bar(kBarFinal));
   }
   __syncwarp();   // roles end in per-lane drains: one arrival per warp at the barrier
   tc_fence_before();

@@ -40,7 +40,7 @@ constexpr uint32_t kPCtlOff = 6 * kTileBytes;
 constexpr uint32_t kPSmem = kPCtlOff + 64;
 constexpr uint32_t kPSmemAlloc = kPSmem + 1024;
 static_assert(kPSmemAlloc <= 232448, "shared memory per CTA");
-enum : int { kPBarLoad = 0, kPBarMma = 1 };
+enum : int { kPBarLoad = 0, kPBarMma = 1, kPBarRead = 3 };   // 16..23 of the control block: TMEM slot, abort flag
 
 __device__ __forceinline__ int part_len(int d) { return d / kTokenParts; }
 __device__ __forceinline__ int padded_row(int d) { return d + 4 * kTokenParts; }
@@ -57,6 +57,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 20);
   const uint32_t bar_load = base + kPCtlOff + 8u * kPBarLoad, bar_mma = base + kPCtlOff + 8u * kPBarMma;
+  const uint32_t bar_read = base + kPCtlOff + 8u * kPBarRead;   // the row warps are done reading TMEM
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const bool with_q = a.q_out != nullptr;
@@ -65,6 +66,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar_load, 1);
     mbar_init(bar_mma, 1);
+    mbar_init(bar_read, 4);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -160,10 +162,12 @@ __global__ void __launch_bounds__(kThreadsP, 1)
   }
   __syncwarp();   // rows past T and the producer's drains split warps: one arrival per warp
   tc_fence_before();
+  if (warp >= 2) warp_arrive(bar_read);   // every TMEM read of this warp is done
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
     mbar_wait_drain(bar_mma, 0);
+    mbar_wait_drain(bar_read, 0);
     __syncwarp();
     tmem_dealloc(tmem, 512);
   }
